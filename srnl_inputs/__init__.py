@@ -1,0 +1,137 @@
+"""Seeded synthetic inputs for the SRNL four-direction scan.
+
+This module is shared by the float64 oracle, the GPU parity tests and the
+benchmark.  It only *draws* numbers and packs them; it holds none of the
+method's arithmetic (no gates, no recurrence, no projection).
+
+Workloads mirror the feature maps the VisionHOPE pages run the operator on
+(VisionHOPE README, "Main results" / "Efficiency"; "VisionHOPE: Visual Backbones
+as Self-Modifying Learning Systems", results paragraph): the 224x224
+hierarchical backbone's stride-4 and stride-16 maps, the plain backbone's
+patch-16 map, and the stride-4 map of a 800x1216 dense-prediction input.
+
+Draw order for one config with seed s (numpy ``default_rng(s)``):
+  1. x ~ N(0, 1), shape [B, H, W, C] (float32)
+  2. ramp configs only: a ~ N(0, 1) of shape [B, H, C];
+     x[b, i, j, c] += 0.5 * a[b, i, c] * (2 j / (W - 1) - 1)
+  3. M_mem0, M_k0, M_v0 ~ N(0, 0.02^2), each [4, heads, d, d]
+  4. m_eta0, m_alpha0 ~ N(0, 0.1^2), each [4, heads, d]
+  5. W_q ~ N(0, 1 / C), shape [C, C]
+Channel scales are the constant 0.25 ([4, C]).  For bf16 configs x is rounded
+to bfloat16 (round to nearest even) and both sides receive those same values.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import numpy as np
+
+F32 = "f32"
+BF16 = "bf16"
+
+
+@dataclasses.dataclass(frozen=True)
+class ScanConfig:
+    name: str
+    B: int
+    H: int
+    W: int
+    C: int
+    heads: int
+    d: int
+    alpha: float
+    chunk_row: int = 0      # 0 -> W (full rows)
+    chunk_col: int = 0      # 0 -> H (full columns)
+    act_dtype: str = BF16
+    x_kind: str = "normal"  # "normal" | "ramp"
+    eps: float = 1e-6
+
+    @property
+    def N(self) -> int:
+        return self.H * self.W
+
+    def replace(self, **kw) -> "ScanConfig":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads.  Sizes, alpha, chunking and value distributions follow the
+# hot-path scope table; seed 0 throughout.
+CONFIGS: Dict[str, ScanConfig] = {
+    "pr1_8x8": ScanConfig("pr1_8x8", B=1, H=8, W=8, C=64, heads=2, d=32,
+                          alpha=0.95, act_dtype=F32),
+    "hier_s1_56x56": ScanConfig("hier_s1_56x56", B=32, H=56, W=56, C=64, heads=2,
+                                d=32, alpha=0.95, act_dtype=BF16),
+    "hier_s3_14x14": ScanConfig("hier_s3_14x14", B=64, H=14, W=14, C=256, heads=8,
+                                d=32, alpha=0.95, act_dtype=BF16, x_kind="ramp"),
+    "plain_14x14": ScanConfig("plain_14x14", B=128, H=14, W=14, C=384, heads=12,
+                              d=32, alpha=0.90, act_dtype=BF16),
+    "hires_200x304": ScanConfig("hires_200x304", B=2, H=200, W=304, C=64, heads=2,
+                                d=32, alpha=0.95, act_dtype=BF16),
+}
+
+
+def bf16_round_bits(x32: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (nearest, ties to even); return uint16 bits."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    bias = ((u >> 16) & 1) + 0x7FFF
+    return ((u + bias) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+@dataclasses.dataclass
+class ScanInputs:
+    cfg: ScanConfig
+    x32: np.ndarray                 # float32 [B,H,W,C]: the values both sides use
+    x_bits: Optional[np.ndarray]    # uint16 [B,H,W,C] for bf16 configs, else None
+    W_q: np.ndarray                 # float32 [C, C]
+    scales: np.ndarray              # float32 [4, C]
+    M_mem0: np.ndarray              # float32 [4, heads, d, d]
+    M_k0: np.ndarray
+    M_v0: np.ndarray
+    m_eta0: np.ndarray              # float32 [4, heads, d]
+    m_alpha0: np.ndarray
+
+    def x_device_payload(self) -> np.ndarray:
+        """The activation buffer as the device receives it (bf16 bits or float32)."""
+        return self.x_bits if self.x_bits is not None else self.x32
+
+    def params(self) -> Dict[str, np.ndarray]:
+        return dict(W_q=self.W_q, scales=self.scales, M_mem0=self.M_mem0,
+                    M_k0=self.M_k0, M_v0=self.M_v0, m_eta0=self.m_eta0,
+                    m_alpha0=self.m_alpha0)
+
+
+def make_inputs(cfg: ScanConfig, seed: int = 0, *, x_scale: float = 1.0,
+                mem_scale: float = 0.02, vec_scale: float = 0.1) -> ScanInputs:
+    """Draw one workload.  ``*_scale`` knobs exist for extra parity cases only."""
+    rng = np.random.default_rng(seed)
+    B, H, W, C, nh, d = cfg.B, cfg.H, cfg.W, cfg.C, cfg.heads, cfg.d
+    x = rng.standard_normal((B, H, W, C), dtype=np.float32) * np.float32(x_scale)
+    if cfg.x_kind == "ramp":
+        a = rng.standard_normal((B, H, C), dtype=np.float32)
+        denom = max(W - 1, 1)
+        ramp = (2.0 * np.arange(W, dtype=np.float32) / denom - 1.0).astype(np.float32)
+        x = x + np.float32(0.5) * a[:, :, None, :] * ramp[None, None, :, None]
+    elif cfg.x_kind != "normal":
+        raise ValueError(f"unknown x_kind {cfg.x_kind!r}")
+    x = x.astype(np.float32)
+    M_mem0 = (rng.standard_normal((4, nh, d, d)) * mem_scale).astype(np.float32)
+    M_k0 = (rng.standard_normal((4, nh, d, d)) * mem_scale).astype(np.float32)
+    M_v0 = (rng.standard_normal((4, nh, d, d)) * mem_scale).astype(np.float32)
+    m_eta0 = (rng.standard_normal((4, nh, d)) * vec_scale).astype(np.float32)
+    m_alpha0 = (rng.standard_normal((4, nh, d)) * vec_scale).astype(np.float32)
+    W_q = (rng.standard_normal((C, C)) / np.sqrt(C)).astype(np.float32)
+    scales = np.full((4, C), 0.25, dtype=np.float32)
+    x_bits = None
+    if cfg.act_dtype == BF16:
+        x_bits = bf16_round_bits(x)
+        x = bf16_bits_to_f32(x_bits).reshape(x.shape)
+    elif cfg.act_dtype != F32:
+        raise ValueError(f"unknown act_dtype {cfg.act_dtype!r}")
+    return ScanInputs(cfg=cfg, x32=np.ascontiguousarray(x), x_bits=x_bits, W_q=W_q,
+                      scales=scales, M_mem0=M_mem0, M_k0=M_k0, M_v0=M_v0,
+                      m_eta0=m_eta0, m_alpha0=m_alpha0)
