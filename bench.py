@@ -1,0 +1,350 @@
+"""Benchmark of the SRNL four-direction scan forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one full forward (query projection, the four route scans, restore +
+channel fusion) over one batch of the workload, inputs resident in HBM.  The
+L2 cache (126 MB) is flushed before every timed step by writing a 256 MiB
+buffer outside the timed events.  Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun, N > 1): the sequences are independent, so every rank runs
+its own replica of the workload with no collective on the data path (weak
+scaling); the time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle (the slow, plain definition
+the parity tests use) on the host cores over a bounded sample of the same
+workload; it is the baseline arm, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from srnl_inputs import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "SRNL 4-dir scan tokens/s (fwd, 1xB200) and % of roofline at 56x56x64"
+UNIT = "route-tokens/s"
+DEFAULT_CONFIG = "hier_s1_56x56"
+L2_FLUSH_BYTES = 256 << 20
+
+# Fallback peaks only when the measured file is absent.
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS,
+                bf16_tflops_sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+# ----------------------------------------------------------------- work model
+def work_model(cfg, gen_bf16=True):
+    """Algorithmic bytes and flops of one forward (per launch)."""
+    B, H, W, C, heads, d = cfg.B, cfg.H, cfg.W, cfg.C, cfg.heads, cfg.d
+    N = H * W
+    tokens = B * N
+    elt = 2 if cfg.act_dtype == "bf16" else 4
+    param_bytes = 4 * (C * C + 4 * C + 4 * heads * (3 * d * d + 2 * d))
+    hbm_bytes = 2 * tokens * C * elt + param_bytes          # x read once, y written once, params
+    seq_tokens = 4 * tokens * heads                          # (route, head) token steps
+    gen_flops = 2.0 * seq_tokens * (2 * d + 2) * d           # boundary generation contraction
+    qproj_flops = 2.0 * tokens * C * C
+    # Sequential update on the single-product state, per (route, head) token:
+    #   s = row . u (2 d^2), row <- alpha row - (eta s) k (3 d^2), z = row . q (2 d^2),
+    #   readout y = M_mem0 z (2 d^2); plus the boundary product G Q_b once per chunk.
+    upd_flops_tok = 9.0 * d * d
+    Lr = cfg.chunk_row or W
+    Lc = cfg.chunk_col or H
+    chunks = B * heads * 2 * (-(-N // Lr) + -(-N // Lc))
+    boundary_flops = 2.0 * chunks * (2 * d + 2) * d * d
+    scan_flops = seq_tokens * upd_flops_tok + gen_flops + boundary_flops
+    return dict(tokens=tokens, route_tokens=4 * tokens, hbm_bytes=hbm_bytes, gen_flops=gen_flops,
+                qproj_flops=qproj_flops, scan_flops=scan_flops, seq_tokens=seq_tokens)
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self._proc = None
+        self._thr = None
+
+    def start(self):
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self._proc = None
+            return
+        self._thr = threading.Thread(target=self._read, daemon=True)
+        self._thr.start()
+
+    def _read(self):
+        for line in self._proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+        if self._thr is not None:
+            self._thr.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------- CPU oracle arm
+def oracle_sample(cfg, n_images, seed=0):
+    """Time the float64 oracle on the first n_images of the workload (1 host thread)."""
+    from oracle import srnl_oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:  # pragma: no cover
+        threadpool_limits = None
+    inp = make_inputs(cfg, seed=seed)
+    ctx = threadpool_limits(1) if threadpool_limits else None
+    t0 = time.perf_counter()
+    try:
+        O.operator_forward(inp.x32[:n_images], inp.params(), alpha_max=cfg.alpha, eps=cfg.eps,
+                           chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, heads=cfg.heads)
+    finally:
+        if ctx is not None:
+            ctx.__exit__(None, None, None)
+    dt = time.perf_counter() - t0
+    return 4.0 * n_images * cfg.H * cfg.W / dt, dt
+
+
+def cpu_baseline(cfg, budget_s=12.0):
+    one_rate, one_dt = oracle_sample(cfg, 1)
+    n = max(1, min(cfg.B, int(budget_s / max(one_dt, 1e-3))))
+    rate, dt = oracle_sample(cfg, n) if n > 1 else (one_rate, one_dt)
+    return {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {cfg.B} images of {cfg.name}, float64 numpy, 1 thread, {dt:.1f} s"}
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return
+    per_step = []
+    n_images = 1
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_sample(cfg, n_images)
+    for _ in range(args.steps):
+        rate, dt = oracle_sample(cfg, n_images)
+        per_step.append(dt)
+    t = sum(per_step)
+    value = 4.0 * n_images * cfg.H * cfg.W * args.steps / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "W": cfg.W,
+                                            "C": cfg.C, "heads": cfg.heads, "d": cfg.d,
+                                            "step_sample_images": n_images},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{n_images} image of {cfg.name} per step, float64 numpy, 1 thread"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- GPU arm
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import self_referential_nested_b200 as S
+    from self_referential_nested_b200 import build as B
+
+    B.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    gen = args.gen or cfg.act_dtype
+    act = cfg.act_dtype
+    inp = make_inputs(cfg, seed=rank)
+    cfgd = dict(B=cfg.B, H=cfg.H, W=cfg.W, C=cfg.C, heads=cfg.heads, d=cfg.d, alpha=cfg.alpha,
+                eps=cfg.eps, chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, act_dtype=act,
+                gen_dtype=gen)
+    h = S.srnl_scan_create(cfgd, inp.params())
+    if act == "bf16":
+        x = torch.from_numpy(inp.x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    else:
+        x = torch.from_numpy(inp.x32).to(dev)
+    y = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    S.srnl_scan_enable_stage_timing(h, 0)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        S.srnl_scan_forward(h, x, y, None, stream)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    S.srnl_scan_enable_stage_timing(h, max(args.steps, 1))
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_((i + 1) & 0xFF)                 # evict x / workspace from L2 (untimed)
+        starts[i].record(stream)
+        S.srnl_scan_forward(h, x, y, None, stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    stage, n_timed = S.srnl_scan_stage_times(h)
+    assert n_timed == args.steps
+    S.srnl_scan_enable_stage_timing(h, 0)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(step_ms))
+
+    # end to end through the host-buffer entry point: pinned x in, y out, every step
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    for _ in range(2):
+        S.srnl_scan_forward_host(h, xh, yh, stream)
+    e2e_s, e2e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e2e_s.record(stream)
+    for _ in range(args.steps):
+        S.srnl_scan_forward_host(h, xh, yh, stream)
+    e2e_e.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks.stop()
+    e2e_ms = e2e_s.elapsed_time(e2e_e)
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+    h.close()
+    if rank != 0:
+        return
+
+    wm = work_model(cfg)
+    peaks = load_peaks()
+    ms_step = total_ms / args.steps
+    value = world * wm["route_tokens"] * args.steps / (total_ms * 1e-3)
+    e2e_value = world * wm["route_tokens"] * args.steps / (e2e_ms * 1e-3)
+    stage_ms = np.asarray(stage)
+    scan_ms = float(stage_ms[1])
+    # dominant kernel: the scan (fp32 SIMT recurrence) -> ALU roofline
+    fp32_peak_tflops = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+    scan_tflops = wm["scan_flops"] / (scan_ms * 1e-3) / 1e12
+    t_bytes_us = wm["hbm_bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
+    t_tensor_us = (wm["gen_flops"] + wm["qproj_flops"]) / (peaks["bf16_tflops"] * 1e12) * 1e6
+    roof_us = max(t_bytes_us, t_tensor_us)
+    elt = 2 if act == "bf16" else 4
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if gen == "bf16" else "f32",
+        "data": "synthetic (seeded normal features, random-init memories)",
+        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "W": cfg.W, "C": cfg.C,
+                   "heads": cfg.heads, "d": cfg.d, "alpha": cfg.alpha, "chunk_row": cfg.chunk_row or cfg.W,
+                   "chunk_col": cfg.chunk_col or cfg.H, "act_dtype": act, "gen_dtype": gen,
+                   "states": "f32", "l2": "flushed (256 MiB write before each timed step)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "raster_tokens_per_s": value / 4},
+        "roofline": {"bound": "alu", "achieved": scan_tflops, "peak": fp32_peak_tflops,
+                     "unit": "TFLOP/s", "frac": scan_tflops / fp32_peak_tflops, "traffic": None,
+                     "kernel": "srnl_scan_kernel", "kernel_ms": scan_ms,
+                     "peak_note": "fp32 FMA peak 148 SM x 128 lanes x 2 x sm_max_mhz (derived)"},
+        "north_star_roofline": {"bound": "hbm" if t_bytes_us >= t_tensor_us else "tensor",
+                                "roofline_us": roof_us, "forward_us": ms_step * 1e3,
+                                "frac": roof_us / (ms_step * 1e3),
+                                "hbm_bytes": wm["hbm_bytes"], "tensor_flops": wm["gen_flops"] + wm["qproj_flops"],
+                                "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TF/s bf16"},
+        "stage_ms": {"query_projection": float(stage_ms[0]), "scan": scan_ms, "fusion": float(stage_ms[2])},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * elt),
+                "d2h_bytes_per_step": int(y.numel() * elt), "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+        line["cpu_baseline"]["gpu_over_cpu"] = value / line["cpu_baseline"]["value"]
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--gen", default=None, choices=[None, "f32", "bf16"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world == 1 and args.gpus > 1:
+        print(json.dumps({"error": "launch N>1 with torchrun"}), flush=True)
+        sys.exit(2)
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * srnl_scan.h — C ABI of the B200 (sm_100a) SRNL four-direction chunked scan.
+ *
+ * The operation is the forward pass of the VisionHOPE operator's memory scan:
+ *   - "VisionHOPE" README (github PSRben/VisionHOPE), sections "Overview" and
+ *     "SRNL and VisionHOPE operator": image features in, same shape out, a new
+ *     memory sequence on every call, head_dim-sized heads, row/column chunks.
+ *   - "VisionHOPE Model Overview: Architecture, Benchmarks, and Practical
+ *     Limits", sections "How VisionHOPE's Five Memories Work" (three matrix and
+ *     two vector memories per head), "Four-Directional Scanning and Spatial
+ *     Chunking" (four routes, per-route memories, shared query projection,
+ *     boundary generation, restore and channel fusion) and "Why the Stability
+ *     Controls Matter" (soft injection cap, spectral clamp).
+ *   - "VisionHOPE: Visual Backbones as Self-Modifying Learning Systems"
+ *     (summary of arXiv 2609.33325), write-rule, stability and 2D-maps
+ *     paragraphs (retained delta gradient write, stabilized key normalisation,
+ *     retention clamp, chunks equal to rows or columns).
+ *
+ * Layout.  Activations are channels-last: x[B][H][W][C] and y[B][H][W][C],
+ * dense, row-major, element type act_dtype.  Channel c belongs to head
+ * c / d, lane c % d.  Token raster index p = i*W + j.
+ *
+ * Routes.  r = 0 forward row-major, 1 reverse row-major, 2 forward
+ * column-major (t = j*H + i), 3 reverse column-major.  Chunks hold chunk_row
+ * (default W) consecutive tokens on routes 0/1 and chunk_col (default H) on
+ * routes 2/3; the last chunk of a route may be shorter.
+ *
+ * Per (batch, head, route) the five memories M_mem, M_k, M_v (d x d) and
+ * m_eta, m_alpha (1 x d) start from the route's initial states.  At each
+ * chunk boundary they generate, for every token of the chunk,
+ *   k~ = M_k x, v = M_v x, a = m_eta x, beta = m_alpha x        (x: head slice)
+ * then  k = k~ / sqrt(|k~|^2 + eps),  alpha_t = min(sigmoid(beta), alpha),
+ *       eta0 = softplus(a), g = |k - v| |k|,
+ *       eta1 = eta0 * phi(eta0 g / (1 - alpha_t)),  phi(z) = tanh(z)/z,
+ *       eta  = min(eta1, 2 / |k|^2),
+ * and every memory X is written in token order
+ *       X <- X alpha_t (I - eta k k^T) - eta (X k - X v) k^T.
+ * The readout after token t's write is y_t = M_mem q_t with q = x W_q^T (all
+ * C channels, split per head).  Outputs of the four routes are restored to
+ * raster order and fused: y[p][c] = sum_r scales[r][c] * y_r[p][c] (r = 0..3).
+ *
+ * Precision.  Memory states and all recurrence arithmetic are fp32.
+ * gen_dtype = SRNL_BF16 rounds the generation operands (x, and the boundary
+ * states of the four generating memories) and the query-projection operands
+ * (x, W_q, and the stored q) to bfloat16, with fp32 accumulation.
+ *
+ * Errors.  Every entry point returns an srnl_status and never aborts.  On
+ * failure the outputs are unspecified and srnl_scan_last_error() describes
+ * the cause.  Kernels are asynchronous on the given stream: a CUDA error
+ * raised by a kernel surfaces from a later call or a stream synchronisation.
+ * No kernel of this library waits on another kernel, rank or flag.
+ *
+ * Threads.  A handle may be used from one host thread at a time; forward
+ * calls on one handle must not overlap on the device (they share the
+ * handle's workspace).
+ */
+#ifndef SRNL_SCAN_H_
+#define SRNL_SCAN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SRNL_API __attribute__((visibility("default")))
+#else
+#define SRNL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct srnl_scan srnl_scan; /* opaque; owned by the library */
+
+typedef enum {
+  SRNL_OK = 0,
+  SRNL_E_INVAL = -1,       /* bad argument: NULL, shape, alignment, range */
+  SRNL_E_UNSUPPORTED = -2, /* valid but not built (e.g. head dim other than 32) */
+  SRNL_E_CUDA = -3,        /* a CUDA runtime call failed */
+  SRNL_E_NOMEM = -4,       /* device or pinned allocation failed */
+  SRNL_E_TIMEOUT = -5      /* reserved: no kernel in this library waits */
+} srnl_status;
+
+typedef enum { SRNL_F32 = 0, SRNL_BF16 = 1 } srnl_dtype;
+
+typedef struct {
+  int B, H, W, C; /* batch, height, width, channels (C = heads * d) */
+  int heads, d;   /* heads and head dim; d = 32 is built */
+  float alpha;    /* retention cap, 0 < alpha < 1 (0.95 hierarchical, 0.9 plain) */
+  float eps;      /* key normalisation epsilon, > 0 (1e-6) */
+  int chunk_row;  /* chunk length on routes 0/1; 0 means W (full rows) */
+  int chunk_col;  /* chunk length on routes 2/3; 0 means H (full columns) */
+  int act_dtype;  /* srnl_dtype of x and y */
+  int gen_dtype;  /* srnl_dtype of generation / projection operands */
+} srnl_scan_config;
+
+/* Parameters, HOST pointers to dense fp32 arrays.  srnl_scan_create copies and
+ * repacks them into device memory owned by the handle; the caller may free
+ * them when create returns. */
+typedef struct {
+  const float* W_q;      /* [C][C]   q = x W_q^T (shared by all routes)      */
+  const float* scales;   /* [4][C]   channel fusion scales per route          */
+  const float* M_mem0;   /* [4][heads][d][d] initial content memory per route */
+  const float* M_k0;     /* [4][heads][d][d] initial key memory               */
+  const float* M_v0;     /* [4][heads][d][d] initial value memory             */
+  const float* m_eta0;   /* [4][heads][d]    initial step-size memory         */
+  const float* m_alpha0; /* [4][heads][d]    initial retention memory         */
+} srnl_scan_params;
+
+/* Validate the config, allocate the handle, its device workspace and its
+ * packed parameters on the CURRENT CUDA device.  *out is set to NULL on
+ * failure.  Allocates with cudaMalloc; synchronous. */
+SRNL_API srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
+                             const srnl_scan_params* params);
+
+/* Forward pass.  x and y are DEVICE pointers on the handle's device, 16-byte
+ * aligned, [B][H][W][C] of act_dtype; x and y must not overlap.
+ * final_states: optional DEVICE pointer to fp32
+ * [4][B][heads][3*d*d + 2*d] receiving the memories after the last token of
+ * each route (M_mem, M_k, M_v row-major, then m_eta, m_alpha); NULL skips it.
+ * stream: a cudaStream_t (NULL = legacy default stream).  Asynchronous. */
+SRNL_API srnl_status srnl_scan_forward(srnl_scan* h, const void* x, void* y,
+                              float* final_states, void* stream);
+
+/* Same forward with HOST buffers: copies x host->device, runs the forward and
+ * copies y device->host on `stream`, then synchronises the stream.  x/y are
+ * host pointers of B*H*W*C act_dtype elements; pinned memory gives full copy
+ * bandwidth.  Uses staging buffers owned by the handle. */
+SRNL_API srnl_status srnl_scan_forward_host(srnl_scan* h, const void* x_host, void* y_host,
+                                   void* stream);
+
+/* Test hook: the device computes the route map the scan kernels use and
+ * writes out[t] = raster index of the t-th token of `route`, t < H*W, into the
+ * DEVICE int32 buffer `out`.  Asynchronous. */
+SRNL_API srnl_status srnl_scan_route_index(const srnl_scan* h, int route, int32_t* out,
+                                  void* stream);
+
+/* Test hook: xr[b][t][c] = x[b][perm_route(t)][c] on the device (act_dtype,
+ * DEVICE pointers, 16-byte aligned).  Asynchronous. */
+SRNL_API srnl_status srnl_scan_gather(const srnl_scan* h, int route, const void* x, void* xr,
+                             void* stream);
+
+/* Stage timing.  srnl_scan_enable_stage_timing(h, n) with n > 0 makes each
+ * later forward record CUDA events on its stream before and after each of its
+ * three kernels (query projection, scan, fusion), keeping the events of the
+ * last n forwards (n <= 1024); n = 0 turns timing off.
+ * srnl_scan_stage_times waits for those events, writes the mean duration in
+ * milliseconds of each kernel over the kept forwards to ms_out[0..2] and the
+ * number of forwards averaged to *count (may be NULL), then starts a new
+ * window.  Returns SRNL_E_INVAL if timing is off or no forward ran. */
+SRNL_API srnl_status srnl_scan_enable_stage_timing(srnl_scan* h, int n);
+SRNL_API srnl_status srnl_scan_stage_times(srnl_scan* h, float* ms_out, int* count);
+
+/* Bytes of device workspace the handle holds (packed params excluded). */
+SRNL_API size_t srnl_scan_workspace_bytes(const srnl_scan* h);
+
+/* Message for the last failure on this handle; with h == NULL, the last
+ * failure of srnl_scan_create on the calling thread.  Never NULL. */
+SRNL_API const char* srnl_scan_last_error(const srnl_scan* h);
+
+/* Static name of a status code. */
+SRNL_API const char* srnl_status_string(int status);
+
+/* Free the handle and all its device memory.  Accepts NULL.  Synchronises the
+ * device before freeing. */
+SRNL_API void srnl_scan_destroy(srnl_scan* h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SRNL_SCAN_H_ */

@@ -1,0 +1,206 @@
+"""Python binding of the SRNL four-direction scan C ABI (``include/srnl_scan.h``).
+
+Argument marshalling only: every step of the forward runs in the CUDA kernels of
+``libsrnl_scan.so``.  There is no CPU fallback; importing works without a GPU,
+but creating a handle needs the built library and a CUDA device.
+
+    from self_referential_nested_b200 import srnl_scan_create, srnl_scan_forward
+    h = srnl_scan_create(cfg_dict, params_dict)      # params: float32 numpy arrays
+    srnl_scan_forward(h, x, y)                      # x, y: CUDA tensors [B,H,W,C]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsrnl_scan.so")
+
+SRNL_OK, SRNL_E_INVAL, SRNL_E_UNSUPPORTED, SRNL_E_CUDA, SRNL_E_NOMEM, SRNL_E_TIMEOUT = 0, -1, -2, -3, -4, -5
+SRNL_F32, SRNL_BF16 = 0, 1
+STATE_FLOATS_D32 = 3 * 32 * 32 + 2 * 32
+
+EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
+            "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
+            "srnl_scan_stage_times", "srnl_scan_workspace_bytes",
+            "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy")
+
+
+class SrnlError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        self.status = status
+        super().__init__(f"{where}: {message} [status {status}]")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int), ("C", ctypes.c_int),
+                ("heads", ctypes.c_int), ("d", ctypes.c_int), ("alpha", ctypes.c_float),
+                ("eps", ctypes.c_float), ("chunk_row", ctypes.c_int), ("chunk_col", ctypes.c_int),
+                ("act_dtype", ctypes.c_int), ("gen_dtype", ctypes.c_int)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W_q", "scales", "M_mem0", "M_k0", "M_v0",
+                                                "m_eta0", "m_alpha0")]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load ``libsrnl_scan.so``; raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m self_referential_nested_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.srnl_scan_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(_Config), ctypes.POINTER(_Params)]
+    lib.srnl_scan_forward.argtypes = [vp, vp, vp, vp, vp]
+    lib.srnl_scan_forward_host.argtypes = [vp, vp, vp, vp]
+    lib.srnl_scan_route_index.argtypes = [vp, i, vp, vp]
+    lib.srnl_scan_gather.argtypes = [vp, i, vp, vp, vp]
+    lib.srnl_scan_enable_stage_timing.argtypes = [vp, i]
+    lib.srnl_scan_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
+    lib.srnl_scan_workspace_bytes.argtypes = [vp]
+    lib.srnl_scan_workspace_bytes.restype = ctypes.c_size_t
+    lib.srnl_scan_last_error.argtypes = [vp]
+    lib.srnl_scan_last_error.restype = ctypes.c_char_p
+    lib.srnl_status_string.argtypes = [i]
+    lib.srnl_status_string.restype = ctypes.c_char_p
+    lib.srnl_scan_destroy.argtypes = [vp]
+    lib.srnl_scan_destroy.restype = None
+    for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
+                 "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
+                 "srnl_scan_stage_times"):
+        getattr(lib, name).restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(t) -> int:
+    """Raw address of a torch tensor, a numpy array or an int (0 for None)."""
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class SrnlScan:
+    """Owns one ``srnl_scan*`` handle; ``close()`` (or GC) destroys it."""
+
+    def __init__(self, handle: int, cfg: Dict):
+        self._h = handle
+        self.cfg = dict(cfg)
+
+    @property
+    def handle(self) -> int:
+        if not self._h:
+            raise RuntimeError("srnl_scan handle is closed")
+        return self._h
+
+    def _check(self, status: int, where: str):
+        if status != SRNL_OK:
+            msg = load_library().srnl_scan_last_error(self._h).decode()
+            raise SrnlError(status, where, msg)
+
+    def close(self):
+        if self._h:
+            load_library().srnl_scan_destroy(self._h)
+            self._h = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self) -> int:
+        return int(load_library().srnl_scan_workspace_bytes(self.handle))
+
+
+def srnl_scan_create(cfg: Dict, params: Dict[str, np.ndarray]) -> SrnlScan:
+    """cfg keys: B, H, W, C, heads, d, alpha, eps, chunk_row, chunk_col,
+    act_dtype, gen_dtype ("f32"/"bf16" or SRNL_F32/SRNL_BF16).  params: float32
+    host arrays W_q, scales, M_mem0, M_k0, M_v0, m_eta0, m_alpha0."""
+    lib = load_library()
+
+    def dt(v):
+        return {"f32": SRNL_F32, "bf16": SRNL_BF16}.get(v, v)
+
+    c = _Config(B=cfg["B"], H=cfg["H"], W=cfg["W"], C=cfg["C"], heads=cfg["heads"], d=cfg["d"],
+                alpha=cfg["alpha"], eps=cfg.get("eps", 1e-6), chunk_row=cfg.get("chunk_row", 0),
+                chunk_col=cfg.get("chunk_col", 0), act_dtype=dt(cfg["act_dtype"]),
+                gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])))
+    keep = {k: np.ascontiguousarray(params[k], dtype=np.float32)
+            for k in ("W_q", "scales", "M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")}
+    p = _Params(**{k: v.ctypes.data for k, v in keep.items()})
+    h = ctypes.c_void_p()
+    st = lib.srnl_scan_create(ctypes.byref(h), ctypes.byref(c), ctypes.byref(p))
+    if st != SRNL_OK:
+        raise SrnlError(st, "srnl_scan_create", lib.srnl_scan_last_error(None).decode())
+    return SrnlScan(h.value, cfg)
+
+
+def srnl_scan_forward(h: SrnlScan, x, y, final_states=None, stream=None) -> None:
+    st = load_library().srnl_scan_forward(h.handle, _ptr(x), _ptr(y), _ptr(final_states), _stream(stream))
+    h._check(st, "srnl_scan_forward")
+
+
+def srnl_scan_forward_host(h: SrnlScan, x_host, y_host, stream=None) -> None:
+    st = load_library().srnl_scan_forward_host(h.handle, _ptr(x_host), _ptr(y_host), _stream(stream))
+    h._check(st, "srnl_scan_forward_host")
+
+
+def srnl_scan_route_index(h: SrnlScan, route: int, out, stream=None) -> None:
+    st = load_library().srnl_scan_route_index(h.handle, route, _ptr(out), _stream(stream))
+    h._check(st, "srnl_scan_route_index")
+
+
+def srnl_scan_gather(h: SrnlScan, route: int, x, xr, stream=None) -> None:
+    st = load_library().srnl_scan_gather(h.handle, route, _ptr(x), _ptr(xr), _stream(stream))
+    h._check(st, "srnl_scan_gather")
+
+
+def srnl_scan_enable_stage_timing(h: SrnlScan, ring: int = 256) -> None:
+    """Keep per-kernel events of the last ``ring`` forwards (0 turns timing off)."""
+    h._check(load_library().srnl_scan_enable_stage_timing(h.handle, int(ring)),
+             "srnl_scan_enable_stage_timing")
+
+
+def srnl_scan_stage_times(h: SrnlScan):
+    """Mean (query projection, scan, fusion) kernel ms over the window, and its size."""
+    out = (ctypes.c_float * 3)()
+    n = ctypes.c_int(0)
+    h._check(load_library().srnl_scan_stage_times(h.handle, out, ctypes.byref(n)), "srnl_scan_stage_times")
+    return tuple(float(v) for v in out), int(n.value)
+
+
+def srnl_scan_destroy(h: SrnlScan) -> None:
+    h.close()
+
+
+def srnl_status_string(status: int) -> str:
+    return load_library().srnl_status_string(status).decode()
+
+
+def srnl_scan_last_error(h: Optional[SrnlScan] = None) -> str:
+    return load_library().srnl_scan_last_error(h._h if h is not None else None).decode()

@@ -1,0 +1,339 @@
+// C ABI of the SRNL four-direction scan (declared in include/srnl_scan.h).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "srnl_common.cuh"
+#include "srnl_launch.h"
+#include "srnl_scan.h"
+
+struct srnl_scan {
+  srnl_scan_config cfg{};
+  srnl::ScanGeom geom{};
+  int device = 0;
+  // packed parameters (device)
+  float* Wq = nullptr;
+  float* G = nullptr;
+  float* Mm = nullptr;
+  float* scales = nullptr;
+  // workspace (device)
+  void* q = nullptr;        // [B*N][C] fp32 or bf16
+  float* yr = nullptr;      // [4][B*N][C] fp32 route partials
+  void* x_stage = nullptr;  // staging for srnl_scan_forward_host
+  void* y_stage = nullptr;
+  size_t ws_bytes = 0;
+  // optional stage timing: a ring of event sets, 4 events per forward
+  std::vector<cudaEvent_t> ev;
+  int ring = 0;        // sets in the ring (0 = timing off)
+  int recorded = 0;    // forwards recorded in the current window
+  std::string err;
+};
+
+namespace {
+
+thread_local std::string g_create_error;
+
+srnl_status fail(srnl_scan* h, srnl_status st, const std::string& msg) {
+  if (h != nullptr) h->err = msg; else g_create_error = msg;
+  return st;
+}
+
+srnl_status cuda_fail(srnl_scan* h, cudaError_t e, const char* what) {
+  std::string msg = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return fail(h, e == cudaErrorMemoryAllocation ? SRNL_E_NOMEM : SRNL_E_CUDA, msg);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+float bf16_round_host(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+size_t act_bytes(const srnl_scan_config& c) {
+  return (size_t)c.B * c.H * c.W * c.C * (c.act_dtype == SRNL_BF16 ? 2 : 4);
+}
+
+void free_all(srnl_scan* h) {
+  void* ptrs[] = {h->Wq, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage};
+  for (void* p : ptrs)
+    if (p != nullptr) cudaFree(p);
+  h->Wq = h->G = h->Mm = h->scales = nullptr;
+  h->q = h->x_stage = h->y_stage = nullptr;
+  h->yr = nullptr;
+}
+
+srnl_status validate_config(const srnl_scan_config* c) {
+  if (c->B <= 0 || c->H <= 0 || c->W <= 0 || c->C <= 0 || c->heads <= 0 || c->d <= 0)
+    return fail(nullptr, SRNL_E_INVAL, "B, H, W, C, heads and d must be positive");
+  if ((int64_t)c->heads * c->d != c->C)
+    return fail(nullptr, SRNL_E_INVAL, "C must equal heads * d");
+  if (c->d != srnl::kD)
+    return fail(nullptr, SRNL_E_UNSUPPORTED, "only head dim d = 32 is built");
+  if (!(c->alpha > 0.f && c->alpha < 1.f))
+    return fail(nullptr, SRNL_E_INVAL, "alpha must lie in (0, 1)");
+  if (!(c->eps > 0.f) || !std::isfinite(c->eps))
+    return fail(nullptr, SRNL_E_INVAL, "eps must be positive and finite");
+  if (c->chunk_row < 0 || c->chunk_col < 0)
+    return fail(nullptr, SRNL_E_INVAL, "chunk lengths must be >= 0 (0 = full rows/columns)");
+  if ((c->act_dtype != SRNL_F32 && c->act_dtype != SRNL_BF16) ||
+      (c->gen_dtype != SRNL_F32 && c->gen_dtype != SRNL_BF16))
+    return fail(nullptr, SRNL_E_INVAL, "act_dtype and gen_dtype must be SRNL_F32 or SRNL_BF16");
+  const int64_t N = (int64_t)c->H * c->W;
+  if (N > (int64_t)1 << 30) return fail(nullptr, SRNL_E_INVAL, "H*W too large");
+  if ((int64_t)4 * c->B * c->heads > (int64_t)INT32_MAX)
+    return fail(nullptr, SRNL_E_INVAL, "4*B*heads too large");
+  if ((int64_t)c->B * N * c->C > ((int64_t)1 << 40))
+    return fail(nullptr, SRNL_E_INVAL, "B*H*W*C too large");
+  return SRNL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* srnl_status_string(int status) {
+  switch (status) {
+    case SRNL_OK: return "SRNL_OK";
+    case SRNL_E_INVAL: return "SRNL_E_INVAL";
+    case SRNL_E_UNSUPPORTED: return "SRNL_E_UNSUPPORTED";
+    case SRNL_E_CUDA: return "SRNL_E_CUDA";
+    case SRNL_E_NOMEM: return "SRNL_E_NOMEM";
+    case SRNL_E_TIMEOUT: return "SRNL_E_TIMEOUT";
+    default: return "SRNL_E_UNKNOWN";
+  }
+}
+
+const char* srnl_scan_last_error(const srnl_scan* h) {
+  return h != nullptr ? h->err.c_str() : g_create_error.c_str();
+}
+
+srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
+                             const srnl_scan_params* prm) {
+  g_create_error.clear();
+  if (out == nullptr) return fail(nullptr, SRNL_E_INVAL, "out is NULL");
+  *out = nullptr;
+  if (cfg == nullptr || prm == nullptr) return fail(nullptr, SRNL_E_INVAL, "cfg or params is NULL");
+  if (prm->W_q == nullptr || prm->scales == nullptr || prm->M_mem0 == nullptr ||
+      prm->M_k0 == nullptr || prm->M_v0 == nullptr || prm->m_eta0 == nullptr ||
+      prm->m_alpha0 == nullptr)
+    return fail(nullptr, SRNL_E_INVAL, "a parameter pointer is NULL");
+  srnl_status st = validate_config(cfg);
+  if (st != SRNL_OK) return st;
+
+  srnl_scan* h = new (std::nothrow) srnl_scan();
+  if (h == nullptr) return fail(nullptr, SRNL_E_NOMEM, "host allocation failed");
+  h->cfg = *cfg;
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaGetDevice"); delete h; return st; }
+
+  const srnl_scan_config& c = h->cfg;
+  const int d = srnl::kD, nh = c.heads;
+  srnl::ScanGeom& g = h->geom;
+  g.B = c.B; g.H = c.H; g.W = c.W; g.C = c.C; g.heads = nh;
+  g.Lrow = c.chunk_row > 0 ? c.chunk_row : c.W;
+  g.Lcol = c.chunk_col > 0 ? c.chunk_col : c.H;
+  g.alpha = c.alpha; g.eps = c.eps;
+  g.act_bf16 = c.act_dtype == SRNL_BF16;
+  g.gen_bf16 = c.gen_dtype == SRNL_BF16;
+
+  // ---- pack parameters on the host, then upload
+  std::vector<float> Wq((size_t)c.C * c.C);
+  for (size_t i = 0; i < Wq.size(); ++i) Wq[i] = g.gen_bf16 ? bf16_round_host(prm->W_q[i]) : prm->W_q[i];
+  std::vector<float> G((size_t)4 * nh * srnl::kGen * d);
+  for (int r = 0; r < 4; ++r)
+    for (int hh = 0; hh < nh; ++hh) {
+      float* dst = G.data() + ((size_t)r * nh + hh) * srnl::kGen * d;
+      const size_t mo = ((size_t)r * nh + hh) * d * d, vo = ((size_t)r * nh + hh) * d;
+      std::memcpy(dst, prm->M_k0 + mo, sizeof(float) * d * d);
+      std::memcpy(dst + d * d, prm->M_v0 + mo, sizeof(float) * d * d);
+      std::memcpy(dst + 2 * d * d, prm->m_eta0 + vo, sizeof(float) * d);
+      std::memcpy(dst + 2 * d * d + d, prm->m_alpha0 + vo, sizeof(float) * d);
+    }
+  const size_t n_mm = (size_t)4 * nh * d * d, n_sc = (size_t)4 * c.C;
+  const size_t tokens = (size_t)c.B * c.H * c.W;
+  const size_t q_bytes = tokens * c.C * (g.gen_bf16 ? 2 : 4);
+  const size_t yr_bytes = 4 * tokens * c.C * sizeof(float);
+  const size_t stage_bytes = act_bytes(c);
+
+  struct { void** p; size_t n; } allocs[] = {
+      {(void**)&h->Wq, Wq.size() * sizeof(float)}, {(void**)&h->G, G.size() * sizeof(float)},
+      {(void**)&h->Mm, n_mm * sizeof(float)},      {(void**)&h->scales, n_sc * sizeof(float)},
+      {&h->q, q_bytes},                            {(void**)&h->yr, yr_bytes},
+      {&h->x_stage, stage_bytes},                  {&h->y_stage, stage_bytes}};
+  for (auto& a : allocs) {
+    e = cudaMalloc(a.p, a.n);
+    if (e != cudaSuccess) {
+      st = cuda_fail(nullptr, e, "cudaMalloc");
+      free_all(h); delete h; return st;
+    }
+  }
+  h->ws_bytes = q_bytes + yr_bytes + 2 * stage_bytes;
+  struct { void* dst; const void* src; size_t n; } copies[] = {
+      {h->Wq, Wq.data(), Wq.size() * sizeof(float)}, {h->G, G.data(), G.size() * sizeof(float)},
+      {h->Mm, prm->M_mem0, n_mm * sizeof(float)},    {h->scales, prm->scales, n_sc * sizeof(float)}};
+  for (auto& cp : copies) {
+    e = cudaMemcpy(cp.dst, cp.src, cp.n, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemcpy (params)"); free_all(h); delete h; return st; }
+  }
+  e = srnl::prepare_kernels();
+  if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "kernel attributes"); free_all(h); delete h; return st; }
+  *out = h;
+  return SRNL_OK;
+}
+
+static srnl_status run_forward(srnl_scan* h, const void* x, void* y, float* finals, cudaStream_t s) {
+  srnl::ScanParamsDev p{h->Wq, h->G, h->Mm, h->scales};
+  cudaError_t e;
+  cudaEvent_t* ev = h->ring > 0 ? &h->ev[(size_t)(h->recorded % h->ring) * 4] : nullptr;
+  if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
+  e = srnl::launch_query_projection(h->geom, p, x, h->q, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
+  if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
+  e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, finals, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "scan launch");
+  if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
+  e = srnl::launch_fuse(h->geom, h->yr, y, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "fusion launch");
+  if (ev) {
+    if ((e = cudaEventRecord(ev[3], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
+    ++h->recorded;
+  }
+  return SRNL_OK;
+}
+
+static srnl_status check_device(srnl_scan* h) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaGetDevice");
+  if (dev != h->device)
+    return fail(h, SRNL_E_INVAL, "current CUDA device differs from the handle's device");
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_forward(srnl_scan* h, const void* x, void* y, float* final_states, void* stream) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (x == nullptr || y == nullptr) return fail(h, SRNL_E_INVAL, "x or y is NULL");
+  if (!aligned16(x) || !aligned16(y)) return fail(h, SRNL_E_INVAL, "x and y must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(final_states) & 3u) != 0)
+    return fail(h, SRNL_E_INVAL, "final_states must be 4-byte aligned");
+  const size_t n = act_bytes(h->cfg);
+  const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+  if (xa < ya + n && ya < xa + n) return fail(h, SRNL_E_INVAL, "x and y overlap");
+  srnl_status st = check_device(h);
+  if (st != SRNL_OK) return st;
+  return run_forward(h, x, y, final_states, static_cast<cudaStream_t>(stream));
+}
+
+srnl_status srnl_scan_forward_host(srnl_scan* h, const void* x_host, void* y_host, void* stream) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (x_host == nullptr || y_host == nullptr) return fail(h, SRNL_E_INVAL, "x or y is NULL");
+  srnl_status st = check_device(h);
+  if (st != SRNL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t n = act_bytes(h->cfg);
+  cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, n, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "host-to-device copy");
+  st = run_forward(h, h->x_stage, h->y_stage, nullptr, s);
+  if (st != SRNL_OK) return st;
+  e = cudaMemcpyAsync(y_host, h->y_stage, n, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "device-to-host copy");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_route_index(const srnl_scan* hc, int route, int32_t* out, void* stream) {
+  srnl_scan* h = const_cast<srnl_scan*>(hc);
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (out == nullptr) return fail(h, SRNL_E_INVAL, "out is NULL");
+  if (route < 0 || route > 3) return fail(h, SRNL_E_INVAL, "route must be 0..3");
+  cudaError_t e = srnl::launch_route_index(route, h->geom.H, h->geom.W, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "route index launch");
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_gather(const srnl_scan* hc, int route, const void* x, void* xr, void* stream) {
+  srnl_scan* h = const_cast<srnl_scan*>(hc);
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (x == nullptr || xr == nullptr) return fail(h, SRNL_E_INVAL, "x or xr is NULL");
+  if (!aligned16(x) || !aligned16(xr)) return fail(h, SRNL_E_INVAL, "x and xr must be 16-byte aligned");
+  if (route < 0 || route > 3) return fail(h, SRNL_E_INVAL, "route must be 0..3");
+  cudaError_t e = srnl::launch_gather(h->geom, route, x, xr, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "gather launch");
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_enable_stage_timing(srnl_scan* h, int n) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (n < 0 || n > 1024) return fail(h, SRNL_E_INVAL, "ring size must be in [0, 1024]");
+  for (cudaEvent_t ev : h->ev) cudaEventDestroy(ev);
+  h->ev.clear();
+  h->ring = 0;
+  h->recorded = 0;
+  if (n == 0) return SRNL_OK;
+  h->ev.assign((size_t)n * 4, nullptr);
+  for (auto& ev : h->ev) {
+    cudaError_t e = cudaEventCreate(&ev);
+    if (e != cudaSuccess) {
+      for (cudaEvent_t x : h->ev)
+        if (x != nullptr) cudaEventDestroy(x);
+      h->ev.clear();
+      return cuda_fail(h, e, "cudaEventCreate");
+    }
+  }
+  h->ring = n;
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_stage_times(srnl_scan* h, float* ms_out, int* count) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (ms_out == nullptr) return fail(h, SRNL_E_INVAL, "ms_out is NULL");
+  if (h->ring == 0 || h->recorded == 0) return fail(h, SRNL_E_INVAL, "stage timing is off or no forward ran");
+  const int n = h->recorded < h->ring ? h->recorded : h->ring;
+  double acc[3] = {0.0, 0.0, 0.0};
+  for (int k = 0; k < n; ++k) {
+    cudaEvent_t* ev = &h->ev[(size_t)k * 4];
+    cudaError_t e = cudaEventSynchronize(ev[3]);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventSynchronize");
+    for (int i = 0; i < 3; ++i) {
+      float ms = 0.f;
+      e = cudaEventElapsedTime(&ms, ev[i], ev[i + 1]);
+      if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventElapsedTime");
+      acc[i] += ms;
+    }
+  }
+  for (int i = 0; i < 3; ++i) ms_out[i] = (float)(acc[i] / n);
+  if (count != nullptr) *count = n;
+  h->recorded = 0;
+  return SRNL_OK;
+}
+
+size_t srnl_scan_workspace_bytes(const srnl_scan* h) { return h != nullptr ? h->ws_bytes : 0; }
+
+void srnl_scan_destroy(srnl_scan* h) {
+  if (h == nullptr) return;
+  int prev = -1;
+  if (cudaGetDevice(&prev) == cudaSuccess && prev != h->device) cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  for (cudaEvent_t ev : h->ev)
+    if (ev != nullptr) cudaEventDestroy(ev);
+  h->ev.clear();
+  free_all(h);
+  if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
+  delete h;
+}
+
+}  // extern "C"

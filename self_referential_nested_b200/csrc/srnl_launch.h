@@ -1,0 +1,41 @@
+// Internal launch interface between the C ABI (srnl_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace srnl {
+
+struct ScanGeom {
+  int B, H, W, C, heads;
+  int Lrow, Lcol;    // resolved chunk lengths (> 0)
+  float alpha, eps;
+  bool act_bf16;     // x / y element type
+  bool gen_bf16;     // generation + projection operands in bf16
+};
+
+struct ScanParamsDev {
+  const float* Wq;      // [C][C] (bf16-rounded values when gen_bf16)
+  const float* G;       // [4][heads][kGen][kD]  generating initials per route/head
+  const float* Mm;      // [4][heads][kD][kD]    content-memory initials
+  const float* scales;  // [4][C]
+};
+
+// q[B*N][C] = x W_q^T ; q is fp32 or bf16 (gen_bf16).
+cudaError_t launch_query_projection(const ScanGeom& g, const ScanParamsDev& p, const void* x,
+                                    void* q, cudaStream_t s);
+
+// Route partials yr[4][B*N][C] (fp32, already scaled by the fusion scales),
+// optional final states.
+cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
+                        float* yr, float* finals, cudaStream_t s);
+
+// y = yr[0] + yr[1] + yr[2] + yr[3] in act dtype.
+cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_t s);
+
+cudaError_t launch_route_index(int route, int H, int W, int32_t* out, cudaStream_t s);
+cudaError_t launch_gather(const ScanGeom& g, int route, const void* x, void* xr, cudaStream_t s);
+
+cudaError_t prepare_kernels();  // one-time function attributes (dynamic smem)
+
+}  // namespace srnl

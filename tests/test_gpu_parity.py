@@ -1,0 +1,262 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Tolerances (relative Frobenius error per output tensor): 1e-4 for the fp32
+path (fp32 activations and generation operands), 2e-2 whenever bf16 enters
+(bf16 activations or bf16 generation/projection operands).  Integer work
+(route maps, gathers) is compared bit for bit.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import self_referential_nested_b200 as S
+from oracle import srnl_oracle as O
+from srnl_inputs import CONFIGS, ScanConfig, bf16_bits_to_f32, bf16_round_bits, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+def tol(act, gen):
+    return TOL_F32 if (act == "f32" and gen == "f32") else TOL_BF16
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from self_referential_nested_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+
+
+def _cfg_dict(cfg, act, gen):
+    return dict(B=cfg.B, H=cfg.H, W=cfg.W, C=cfg.C, heads=cfg.heads, d=cfg.d, alpha=cfg.alpha,
+                eps=cfg.eps, chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, act_dtype=act,
+                gen_dtype=gen)
+
+
+def _x_device(x32, act):
+    if act == "bf16":
+        bits = bf16_round_bits(x32)
+        return torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).cuda()
+
+
+def gpu_forward(inp, act, gen, finals=False, params=None):
+    cfg = inp.cfg
+    h = S.srnl_scan_create(_cfg_dict(cfg, act, gen), params or inp.params())
+    try:
+        x = _x_device(inp.x32, act)
+        y = torch.empty_like(x)
+        fin = torch.full((4, cfg.B, cfg.heads, S.STATE_FLOATS_D32), float("nan"), device="cuda") if finals else None
+        S.srnl_scan_forward(h, x, y, fin)
+        torch.cuda.synchronize()
+        return y.float().cpu().numpy(), (fin.cpu().numpy() if finals else None)
+    finally:
+        h.close()
+
+
+def oracle_forward(inp, batch=None, params=None):
+    cfg = inp.cfg
+    x = inp.x32 if batch is None else inp.x32[batch]
+    return O.operator_forward(x, params or inp.params(), alpha_max=cfg.alpha, eps=cfg.eps,
+                              chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, heads=cfg.heads)[:2]
+
+
+@functools.lru_cache(maxsize=None)
+def _cached_oracle(name, batch):
+    inp = make_inputs(CONFIGS[name], seed=0)
+    out, fin = oracle_forward(inp, list(batch))
+    return out, fin
+
+
+def assert_rel(a, b, bound, what):
+    err = O.rel_fro(a, b)
+    assert err <= bound, f"{what}: relative Frobenius error {err:.3e} > {bound:.1e}"
+    return err
+
+
+# ------------------------------------------------------------ integer work
+@pytest.mark.parametrize("H,W", [(1, 1), (1, 7), (7, 1), (2, 3), (8, 8), (14, 20), (56, 56), (200, 304)])
+def test_route_index_bit_exact(H, W):
+    cfg = ScanConfig("idx", B=1, H=H, W=W, C=32, heads=1, d=32, alpha=0.9, act_dtype="f32")
+    inp = make_inputs(cfg)
+    h = S.srnl_scan_create(_cfg_dict(cfg, "f32", "f32"), inp.params())
+    try:
+        for r in range(4):
+            out = torch.full((H * W,), -1, dtype=torch.int32, device="cuda")
+            S.srnl_scan_route_index(h, r, out)
+            torch.cuda.synchronize()
+            assert np.array_equal(out.cpu().numpy().astype(np.int64), O.route_index_map(H, W, r)), r
+    finally:
+        h.close()
+
+
+@pytest.mark.parametrize("act", ["f32", "bf16"])
+@pytest.mark.parametrize("H,W", [(2, 3), (5, 7), (14, 20)])
+def test_gather_bit_exact(act, H, W):
+    cfg = ScanConfig("g", B=2, H=H, W=W, C=64, heads=2, d=32, alpha=0.9, act_dtype=act)
+    inp = make_inputs(cfg, seed=5)
+    h = S.srnl_scan_create(_cfg_dict(cfg, act, act), inp.params())
+    try:
+        x = _x_device(inp.x32, act)
+        for r in range(4):
+            xr = torch.empty_like(x)
+            S.srnl_scan_gather(h, r, x, xr)
+            torch.cuda.synchronize()
+            got = xr.float().cpu().numpy().reshape(2, H * W, 64)
+            assert np.array_equal(got, O.gather(inp.x32, r)), r
+    finally:
+        h.close()
+
+
+# ------------------------------------------------------------ the five workloads
+def test_pr1_fp32_path_outputs_and_states():
+    inp = make_inputs(CONFIGS["pr1_8x8"], seed=0)
+    y, fin = gpu_forward(inp, "f32", "f32", finals=True)
+    ref, ref_fin = oracle_forward(inp)
+    assert_rel(y, ref, TOL_F32, "pr1 y")
+    assert_rel(fin, ref_fin, TOL_F32, "pr1 final states")
+
+
+def test_pr1_bf16_path():
+    cfg = CONFIGS["pr1_8x8"].replace(act_dtype="bf16")
+    inp = make_inputs(cfg, seed=0)
+    y, fin = gpu_forward(inp, "bf16", "bf16", finals=True)
+    ref, ref_fin = oracle_forward(inp)
+    assert_rel(y, ref, TOL_BF16, "pr1 bf16 y")
+    assert_rel(fin, ref_fin, TOL_BF16, "pr1 bf16 final states")
+
+
+SAMPLED = {
+    "hier_s1_56x56": (0, 31),
+    "hier_s3_14x14": (0, 17, 63),
+    "plain_14x14": (0, 64, 127),
+    "hires_200x304": (1,),
+}
+
+
+@pytest.mark.parametrize("path", [("f32", "f32"), ("bf16", "bf16"), ("bf16", "f32")])
+@pytest.mark.parametrize("name", list(SAMPLED))
+def test_full_size_config_sampled_batch(name, path):
+    """Full-size launch (the benchmark's), compared on sampled batch items."""
+    act, gen = path
+    inp = make_inputs(CONFIGS[name], seed=0)
+    y, _ = gpu_forward(inp, act, gen)
+    batch = SAMPLED[name]
+    ref, _ = _cached_oracle(name, batch)
+    assert np.all(np.isfinite(y))
+    assert_rel(y[list(batch)], ref, tol(act, gen), f"{name} {act}/{gen}")
+
+
+# ------------------------------------------------------------ ragged and edge cases
+ACTIVE = dict(mem_scale=0.3, vec_scale=1.0)
+
+RAGGED = [
+    # (H, W, B, heads, chunk_row, chunk_col, alpha)
+    (3, 5, 2, 1, 0, 0, 0.95),
+    (5, 3, 1, 3, 0, 0, 0.9),
+    (1, 9, 2, 2, 0, 0, 0.95),
+    (9, 1, 2, 2, 0, 0, 0.95),
+    (7, 13, 2, 2, 4, 3, 0.95),      # incomplete final chunks on every route
+    (6, 6, 1, 2, 1, 1, 0.9),        # chunk 1: token-wise generation
+    (5, 7, 1, 1, 200, 200, 0.95),   # one chunk longer than the sequence
+    (12, 11, 1, 1, 100, 70, 0.9),   # chunks longer than the staged sub-block
+]
+
+
+@pytest.mark.parametrize("path", [("f32", "f32"), ("bf16", "bf16")])
+@pytest.mark.parametrize("case", RAGGED)
+@pytest.mark.parametrize("active", [False, True])
+def test_ragged_shapes_and_chunks(case, path, active):
+    H, W, B, heads, cr, cc, alpha = case
+    act, gen = path
+    cfg = ScanConfig("ragged", B=B, H=H, W=W, C=32 * heads, heads=heads, d=32, alpha=alpha,
+                     chunk_row=cr, chunk_col=cc, act_dtype=act)
+    inp = make_inputs(cfg, seed=11, **(ACTIVE if active else {}))
+    y, fin = gpu_forward(inp, act, gen, finals=True)
+    ref, ref_fin = oracle_forward(inp)
+    assert_rel(y, ref, tol(act, gen), f"ragged {case} y")
+    if np.linalg.norm(ref_fin) > 1e-30:
+        assert_rel(fin, ref_fin, tol(act, gen), f"ragged {case} states")
+
+
+@pytest.mark.parametrize("route", [0, 1, 2, 3])
+def test_each_route_chunk_by_chunk(route):
+    """One-hot fusion isolates a route; every chunk of it must match on its own
+    (so errors in later chunks cannot hide behind larger early outputs)."""
+    H, W = 6, 8
+    cfg = ScanConfig("route", B=2, H=H, W=W, C=64, heads=2, d=32, alpha=0.95, chunk_row=3,
+                     chunk_col=2, act_dtype="f32")
+    inp = make_inputs(cfg, seed=21, mem_scale=0.3, vec_scale=0.6)
+    params = inp.params()
+    params["scales"] = np.zeros_like(params["scales"])
+    params["scales"][route] = 1.0
+    y, _ = gpu_forward(inp, "f32", "f32", params=params)
+    ref, _ = oracle_forward(inp, params=params)
+    yr, rr = O.gather(y, route), O.gather(ref, route)
+    L = O.default_chunk(H, W, route, cfg.chunk_row, cfg.chunk_col)
+    peak = np.linalg.norm(rr)
+    checked = 0
+    for c0 in range(0, H * W, L):
+        ref_c = rr[:, c0:c0 + L]
+        if np.linalg.norm(ref_c) < 1e-6 * peak:
+            continue
+        assert_rel(yr[:, c0:c0 + L], ref_c, 1e-3, f"route {route} chunk at {c0}")
+        checked += 1
+    assert checked >= 3
+
+
+def test_forward_host_matches_device_path():
+    cfg = CONFIGS["hier_s3_14x14"].replace(B=4)
+    inp = make_inputs(cfg, seed=0)
+    h = S.srnl_scan_create(_cfg_dict(cfg, "bf16", "bf16"), inp.params())
+    try:
+        x = _x_device(inp.x32, "bf16")
+        y = torch.empty_like(x)
+        S.srnl_scan_forward(h, x, y)
+        torch.cuda.synchronize()
+        xh = x.cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        S.srnl_scan_forward_host(h, xh, yh)
+        assert torch.equal(yh, y.cpu())
+    finally:
+        h.close()
+
+
+def test_repeated_calls_are_bitwise_identical():
+    inp = make_inputs(CONFIGS["hier_s1_56x56"].replace(B=2), seed=0)
+    h = S.srnl_scan_create(_cfg_dict(inp.cfg, "bf16", "bf16"), inp.params())
+    try:
+        x = _x_device(inp.x32, "bf16")
+        y1, y2 = torch.empty_like(x), torch.empty_like(x)
+        S.srnl_scan_forward(h, x, y1)
+        S.srnl_scan_forward(h, x, y2)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2)
+    finally:
+        h.close()
+
+
+def test_argument_errors_are_reported():
+    inp = make_inputs(CONFIGS["pr1_8x8"], seed=0)
+    h = S.srnl_scan_create(_cfg_dict(inp.cfg, "f32", "f32"), inp.params())
+    try:
+        buf = torch.zeros(2 * inp.x32.size + 16, device="cuda")
+        x = buf[: inp.x32.size]
+        with pytest.raises(S.SrnlError) as e:
+            S.srnl_scan_forward(h, x.data_ptr() + 4, buf[inp.x32.size + 8:].data_ptr())
+        assert e.value.status == S.SRNL_E_INVAL and "aligned" in str(e.value)
+        with pytest.raises(S.SrnlError) as e:
+            S.srnl_scan_forward(h, x, buf[16:])
+        assert e.value.status == S.SRNL_E_INVAL and "overlap" in str(e.value)
+        with pytest.raises(S.SrnlError) as e:
+            S.srnl_scan_route_index(h, 4, x)
+        assert e.value.status == S.SRNL_E_INVAL
+    finally:
+        h.close()
