@@ -129,6 +129,33 @@ SRNL_API srnl_status srnl_scan_forward(srnl_scan* h, const void* x, void* y,
 SRNL_API srnl_status srnl_scan_forward_host(srnl_scan* h, const void* x_host, void* y_host,
                                    void* stream);
 
+/* Allocation-free forward (the pages have no counterpart: this is an
+ * interface for callers, not part of the method).  It is for callers that
+ * must not call cudaMalloc: code hosted by a framework that owns all device
+ * memory through its own pool, where a raw allocation bypasses its accounting,
+ * and latency-critical loops where an allocation may synchronise the device.
+ * No handle is created and nothing is allocated or freed; the scratch (packed
+ * parameters, projected queries, route partials) is a file-scope device array
+ * of SRNL_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds
+ * until the process exits.
+ *   cfg    : same rules as srnl_scan_create.
+ *   params : DEVICE pointers on the current device, same layouts as
+ *            srnl_scan_params; W_q 16-byte aligned.
+ *   x, y   : DEVICE pointers as in srnl_scan_forward.
+ * A workload needing more than SRNL_NOALLOC_SCRATCH_BYTES of scratch
+ * (about 18 bytes per activation element on the bf16 path, 20 on fp32, plus
+ * the parameters) is rejected with SRNL_E_INVAL and a message giving both
+ * sizes.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array and it keeps the last
+ * call's contents (nothing in it needs to start at zero); calls that overlap
+ * on the GPU race.  Errors are reported through srnl_scan_last_error(NULL).
+ * Asynchronous on `stream`. */
+#define SRNL_NOALLOC_SCRATCH_BYTES (32u << 20)
+SRNL_API srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
+                                               const srnl_scan_params* params,
+                                               const void* x, void* y, void* stream);
+
 /* Test hook: the device computes the route map the scan kernels use and
  * writes out[t] = raster index of the t-th token of `route`, t < H*W, into the
  * DEVICE int32 buffer `out`.  Asynchronous. */

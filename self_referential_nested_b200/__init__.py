@@ -23,7 +23,10 @@ SRNL_OK, SRNL_E_INVAL, SRNL_E_UNSUPPORTED, SRNL_E_CUDA, SRNL_E_NOMEM, SRNL_E_TIM
 SRNL_F32, SRNL_BF16 = 0, 1
 STATE_FLOATS_D32 = 3 * 32 * 32 + 2 * 32
 
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
 EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
+            "srnl_scan_forward_noalloc",
             "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
             "srnl_scan_stage_times", "srnl_scan_workspace_bytes",
             "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy")
@@ -63,6 +66,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_scan_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(_Config), ctypes.POINTER(_Params)]
     lib.srnl_scan_forward.argtypes = [vp, vp, vp, vp, vp]
     lib.srnl_scan_forward_host.argtypes = [vp, vp, vp, vp]
+    lib.srnl_scan_forward_noalloc.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(_Params), vp, vp, vp]
     lib.srnl_scan_route_index.argtypes = [vp, i, vp, vp]
     lib.srnl_scan_gather.argtypes = [vp, i, vp, vp, vp]
     lib.srnl_scan_enable_stage_timing.argtypes = [vp, i]
@@ -75,7 +79,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_status_string.restype = ctypes.c_char_p
     lib.srnl_scan_destroy.argtypes = [vp]
     lib.srnl_scan_destroy.restype = None
-    for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
+    for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
                  "srnl_scan_stage_times"):
         getattr(lib, name).restype = ctypes.c_int
@@ -137,19 +141,22 @@ class SrnlScan:
         return int(load_library().srnl_scan_workspace_bytes(self.handle))
 
 
+def _config_struct(cfg: Dict) -> _Config:
+    def dt(v):
+        return {"f32": SRNL_F32, "bf16": SRNL_BF16}.get(v, v)
+
+    return _Config(B=cfg["B"], H=cfg["H"], W=cfg["W"], C=cfg["C"], heads=cfg["heads"], d=cfg["d"],
+                   alpha=cfg["alpha"], eps=cfg.get("eps", 1e-6), chunk_row=cfg.get("chunk_row", 0),
+                   chunk_col=cfg.get("chunk_col", 0), act_dtype=dt(cfg["act_dtype"]),
+                   gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])))
+
+
 def srnl_scan_create(cfg: Dict, params: Dict[str, np.ndarray]) -> SrnlScan:
     """cfg keys: B, H, W, C, heads, d, alpha, eps, chunk_row, chunk_col,
     act_dtype, gen_dtype ("f32"/"bf16" or SRNL_F32/SRNL_BF16).  params: float32
     host arrays W_q, scales, M_mem0, M_k0, M_v0, m_eta0, m_alpha0."""
     lib = load_library()
-
-    def dt(v):
-        return {"f32": SRNL_F32, "bf16": SRNL_BF16}.get(v, v)
-
-    c = _Config(B=cfg["B"], H=cfg["H"], W=cfg["W"], C=cfg["C"], heads=cfg["heads"], d=cfg["d"],
-                alpha=cfg["alpha"], eps=cfg.get("eps", 1e-6), chunk_row=cfg.get("chunk_row", 0),
-                chunk_col=cfg.get("chunk_col", 0), act_dtype=dt(cfg["act_dtype"]),
-                gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])))
+    c = _config_struct(cfg)
     keep = {k: np.ascontiguousarray(params[k], dtype=np.float32)
             for k in ("W_q", "scales", "M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")}
     p = _Params(**{k: v.ctypes.data for k, v in keep.items()})
@@ -168,6 +175,24 @@ def srnl_scan_forward(h: SrnlScan, x, y, final_states=None, stream=None) -> None
 def srnl_scan_forward_host(h: SrnlScan, x_host, y_host, stream=None) -> None:
     st = load_library().srnl_scan_forward_host(h.handle, _ptr(x_host), _ptr(y_host), _stream(stream))
     h._check(st, "srnl_scan_forward_host")
+
+
+def srnl_scan_forward_noalloc(cfg: Dict, params_dev: Dict, x, y, stream=None) -> None:
+    """Allocation-free forward: no handle, no device allocation.
+
+    For callers that must not call cudaMalloc (a host framework that owns all
+    device memory through its own pool; latency-critical loops).  params_dev:
+    the seven parameter arrays as DEVICE buffers (torch CUDA tensors or raw
+    addresses) in the srnl_scan_params layouts.  Scratch is a fixed
+    NOALLOC_SCRATCH_BYTES device array inside the library, shared by all calls.
+    """
+    lib = load_library()
+    c = _config_struct(cfg)
+    p = _Params(**{k: _ptr(params_dev[k]) for k in ("W_q", "scales", "M_mem0", "M_k0", "M_v0",
+                                                     "m_eta0", "m_alpha0")})
+    st = lib.srnl_scan_forward_noalloc(ctypes.byref(c), ctypes.byref(p), _ptr(x), _ptr(y), _stream(stream))
+    if st != SRNL_OK:
+        raise SrnlError(st, "srnl_scan_forward_noalloc", lib.srnl_scan_last_error(None).decode())
 
 
 def srnl_scan_route_index(h: SrnlScan, route: int, out, stream=None) -> None:

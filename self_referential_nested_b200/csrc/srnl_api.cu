@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "srnl_common.cuh"
+#include "srnl_internal.h"
 #include "srnl_launch.h"
 #include "srnl_scan.h"
 
@@ -95,6 +96,11 @@ srnl_status validate_config(const srnl_scan_config* c) {
 }
 
 }  // namespace
+
+namespace srnl {
+srnl_status validate_scan_config(const srnl_scan_config* cfg) { return validate_config(cfg); }
+void set_thread_error(const std::string& msg) { g_create_error = msg; }
+}  // namespace srnl
 
 extern "C" {
 

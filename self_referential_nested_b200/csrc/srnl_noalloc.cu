@@ -1,0 +1,174 @@
+// srnl_scan_forward_noalloc: the forward pass without any device allocation.
+//
+// For callers that must not call cudaMalloc: code hosted by a framework that
+// owns all device memory through its own pool (a raw cudaMalloc bypasses its
+// accounting and can fail or fragment the pool), and latency-critical loops
+// where cudaMalloc may synchronise the device and take unbounded time.
+//
+// The scratch the forward needs (repacked parameters, the projected queries
+// and the four scaled route partials) lives in one file-scope __device__ array
+// of kNoallocScratchBytes.  Every GPU that loads this library holds that array
+// until the process exits.  In host code the array's name is only a host-side
+// stand-in, so its device address is looked up with cudaGetSymbolAddress once
+// per device, on the first call made with that device current, and cached.
+//
+// All calls share the array and it keeps the last call's contents.  Nothing in
+// it has to start at zero: every byte a call reads is written earlier in the
+// same call (pack, projection, scan in that order on the caller's stream).
+// Calls that overlap on the GPU (for example on two streams) race on the array.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+#include <string>
+
+#include "srnl_common.cuh"
+#include "srnl_internal.h"
+#include "srnl_launch.h"
+#include "srnl_scan.h"
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = SRNL_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array for the current device (set up once per device).
+srnl_status scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    srnl::set_thread_error(std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+    return SRNL_E_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    srnl::set_thread_error("device ordinal out of range for the no-allocation scratch table");
+    return SRNL_E_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      srnl::set_thread_error(std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(e));
+      return SRNL_E_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return SRNL_OK;
+}
+
+size_t round_up(size_t n) { return (n + 255) & ~size_t(255); }
+
+// W_q copy (bf16-rounded on the bf16 path) and G = [M_k0; M_v0; m_eta0; m_alpha0]
+// per (route, head), the layouts the scan kernels read.
+__global__ void noalloc_pack_kernel(const float* __restrict__ Wq_src, float* __restrict__ Wq_dst,
+                                    int64_t n_wq, bool round_bf16_wq, const float* __restrict__ Mk,
+                                    const float* __restrict__ Mv, const float* __restrict__ me,
+                                    const float* __restrict__ ma, float* __restrict__ G,
+                                    int64_t n_g) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n_wq) {
+    const float w = Wq_src[i];
+    Wq_dst[i] = round_bf16_wq ? srnl::round_bf16(w) : w;
+  }
+  if (i < n_g) {
+    constexpr int per = srnl::kGen * srnl::kD;
+    const int64_t rh = i / per;
+    const int rem = (int)(i - rh * per);
+    const int m = rem / srnl::kD, j = rem % srnl::kD;
+    float v;
+    if (m < srnl::kD) v = Mk[(rh * srnl::kD + m) * srnl::kD + j];
+    else if (m < 2 * srnl::kD) v = Mv[(rh * srnl::kD + (m - srnl::kD)) * srnl::kD + j];
+    else if (m == 2 * srnl::kD) v = me[rh * srnl::kD + j];
+    else v = ma[rh * srnl::kD + j];
+    G[i] = v;
+  }
+}
+
+}  // namespace
+
+extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
+                                                 const srnl_scan_params* p, const void* x,
+                                                 void* y, void* stream) {
+  srnl::set_thread_error("");
+  if (cfg == nullptr || p == nullptr) {
+    srnl::set_thread_error("cfg or params is NULL");
+    return SRNL_E_INVAL;
+  }
+  if (p->W_q == nullptr || p->scales == nullptr || p->M_mem0 == nullptr || p->M_k0 == nullptr ||
+      p->M_v0 == nullptr || p->m_eta0 == nullptr || p->m_alpha0 == nullptr) {
+    srnl::set_thread_error("a parameter pointer is NULL");
+    return SRNL_E_INVAL;
+  }
+  srnl_status st = srnl::validate_scan_config(cfg);
+  if (st != SRNL_OK) return st;
+  if (x == nullptr || y == nullptr) {
+    srnl::set_thread_error("x or y is NULL");
+    return SRNL_E_INVAL;
+  }
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u) ||
+      (reinterpret_cast<uintptr_t>(p->W_q) & 15u)) {
+    srnl::set_thread_error("x, y and W_q must be 16-byte aligned");
+    return SRNL_E_INVAL;
+  }
+  const bool act_bf16 = cfg->act_dtype == SRNL_BF16, gen_bf16 = cfg->gen_dtype == SRNL_BF16;
+  const size_t tokens = (size_t)cfg->B * cfg->H * cfg->W;
+  const size_t act_bytes = tokens * cfg->C * (act_bf16 ? 2 : 4);
+  {
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+    if (xa < ya + act_bytes && ya < xa + act_bytes) {
+      srnl::set_thread_error("x and y overlap");
+      return SRNL_E_INVAL;
+    }
+  }
+  const size_t n_wq = (size_t)cfg->C * cfg->C;
+  const size_t n_g = (size_t)4 * cfg->heads * srnl::kGen * srnl::kD;
+  const size_t wq_b = round_up(n_wq * 4), g_b = round_up(n_g * 4);
+  const size_t q_b = round_up(tokens * cfg->C * (gen_bf16 ? 2 : 4));
+  const size_t yr_b = round_up(4 * tokens * cfg->C * sizeof(float));
+  const size_t need = wq_b + g_b + q_b + yr_b;
+  if (need > kNoallocScratchBytes) {
+    srnl::set_thread_error("workload needs " + std::to_string(need) +
+                           " bytes of scratch; the no-allocation forward holds " +
+                           std::to_string(kNoallocScratchBytes));
+    return SRNL_E_INVAL;
+  }
+  void* base = nullptr;
+  st = scratch_address(&base);
+  if (st != SRNL_OK) return st;
+  unsigned char* s8 = static_cast<unsigned char*>(base);
+  float* Wq = reinterpret_cast<float*>(s8);
+  float* G = reinterpret_cast<float*>(s8 + wq_b);
+  void* q = s8 + wq_b + g_b;
+  float* yr = reinterpret_cast<float*>(s8 + wq_b + g_b + q_b);
+
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const size_t n_pack = n_wq > n_g ? n_wq : n_g;
+  noalloc_pack_kernel<<<(unsigned)((n_pack + 255) / 256), 256, 0, cs>>>(
+      p->W_q, Wq, (int64_t)n_wq, gen_bf16, p->M_k0, p->M_v0, p->m_eta0, p->m_alpha0, G, (int64_t)n_g);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = srnl::prepare_kernels();
+
+  srnl::ScanGeom g{};
+  g.B = cfg->B; g.H = cfg->H; g.W = cfg->W; g.C = cfg->C; g.heads = cfg->heads;
+  g.Lrow = cfg->chunk_row > 0 ? cfg->chunk_row : cfg->W;
+  g.Lcol = cfg->chunk_col > 0 ? cfg->chunk_col : cfg->H;
+  g.alpha = cfg->alpha; g.eps = cfg->eps;
+  g.act_bf16 = act_bf16; g.gen_bf16 = gen_bf16;
+  const srnl::ScanParamsDev dp{Wq, G, p->M_mem0, p->scales};
+  if (e == cudaSuccess) e = srnl::launch_query_projection(g, dp, x, q, cs);
+  if (e == cudaSuccess) e = srnl::launch_scan(g, dp, x, q, yr, nullptr, cs);
+  if (e == cudaSuccess) e = srnl::launch_fuse(g, yr, y, cs);
+  if (e != cudaSuccess) {
+    srnl::set_thread_error(std::string("no-allocation forward launch: ") + cudaGetErrorString(e));
+    return SRNL_E_CUDA;
+  }
+  return SRNL_OK;
+}
