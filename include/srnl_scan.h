@@ -40,15 +40,19 @@
  * raster order and fused: y[p][c] = sum_r scales[r][c] * y_r[p][c] (r = 0..3).
  *
  * Precision.  Memory states and all recurrence arithmetic are fp32.
- * gen_dtype = SRNL_BF16 rounds the generation operands (x, and the boundary
- * states of the four generating memories) and the query-projection operands
- * (x, W_q, and the stored q) to bfloat16, with fp32 accumulation.
+ * gen_dtype = SRNL_BF16 computes the boundary generation as a bf16 tensor-core
+ * contraction with fp32 accumulation: the four generating memories at a chunk
+ * boundary are G Q_b (G their initial states, Q_b the product of the
+ * transitions so far), and each token's k~, v, a, beta = G (Q_b x); G and
+ * Q_b x are rounded to bfloat16.  It also rounds the query-projection operands
+ * (x, W_q) and the stored q to bfloat16.
  *
  * Errors.  Every entry point returns an srnl_status and never aborts.  On
  * failure the outputs are unspecified and srnl_scan_last_error() describes
  * the cause.  Kernels are asynchronous on the given stream: a CUDA error
  * raised by a kernel surfaces from a later call or a stream synchronisation.
- * No kernel of this library waits on another kernel, rank or flag.
+ * No kernel of this library waits on another kernel, rank or flag; the scan
+ * kernel's only waits are bounded polls on its own tensor-core completions.
  *
  * Threads.  A handle may be used from one host thread at a time; forward
  * calls on one handle must not overlap on the device (they share the
@@ -78,7 +82,7 @@ typedef enum {
   SRNL_E_UNSUPPORTED = -2, /* valid but not built (e.g. head dim other than 32) */
   SRNL_E_CUDA = -3,        /* a CUDA runtime call failed */
   SRNL_E_NOMEM = -4,       /* device or pinned allocation failed */
-  SRNL_E_TIMEOUT = -5      /* reserved: no kernel in this library waits */
+  SRNL_E_TIMEOUT = -5      /* a bounded in-kernel wait gave up (see srnl_scan_device_status) */
 } srnl_status;
 
 typedef enum { SRNL_F32 = 0, SRNL_BF16 = 1 } srnl_dtype;
@@ -177,6 +181,12 @@ SRNL_API srnl_status srnl_scan_gather(const srnl_scan* h, int route, const void*
  * window.  Returns SRNL_E_INVAL if timing is off or no forward ran. */
 SRNL_API srnl_status srnl_scan_enable_stage_timing(srnl_scan* h, int n);
 SRNL_API srnl_status srnl_scan_stage_times(srnl_scan* h, float* ms_out, int* count);
+
+/* Device status of the handle's kernels: synchronously reads the status word
+ * the scan kernel sets when one of its bounded waits (for its own tensor-core
+ * work) gives up.  Returns SRNL_OK, or SRNL_E_TIMEOUT once that has happened
+ * (outputs of that forward are then unspecified). */
+SRNL_API srnl_status srnl_scan_device_status(srnl_scan* h);
 
 /* Bytes of device workspace the handle holds (packed params excluded). */
 SRNL_API size_t srnl_scan_workspace_bytes(const srnl_scan* h);

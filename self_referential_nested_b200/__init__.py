@@ -28,7 +28,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_scan_forward_noalloc",
             "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
-            "srnl_scan_stage_times", "srnl_scan_workspace_bytes",
+            "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_scan_workspace_bytes",
             "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy")
 
 
@@ -71,6 +71,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_scan_gather.argtypes = [vp, i, vp, vp, vp]
     lib.srnl_scan_enable_stage_timing.argtypes = [vp, i]
     lib.srnl_scan_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
+    lib.srnl_scan_device_status.argtypes = [vp]
     lib.srnl_scan_workspace_bytes.argtypes = [vp]
     lib.srnl_scan_workspace_bytes.restype = ctypes.c_size_t
     lib.srnl_scan_last_error.argtypes = [vp]
@@ -81,7 +82,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_scan_destroy.restype = None
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
-                 "srnl_scan_stage_times"):
+                 "srnl_scan_stage_times", "srnl_scan_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -217,6 +218,11 @@ def srnl_scan_stage_times(h: SrnlScan):
     n = ctypes.c_int(0)
     h._check(load_library().srnl_scan_stage_times(h.handle, out, ctypes.byref(n)), "srnl_scan_stage_times")
     return tuple(float(v) for v in out), int(n.value)
+
+
+def srnl_scan_device_status(h: SrnlScan) -> None:
+    """Raise SrnlError if a bounded in-kernel wait of this handle ever gave up."""
+    h._check(load_library().srnl_scan_device_status(h.handle), "srnl_scan_device_status")
 
 
 def srnl_scan_destroy(h: SrnlScan) -> None:

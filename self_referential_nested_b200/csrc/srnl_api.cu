@@ -29,6 +29,7 @@ struct srnl_scan {
   float* yr = nullptr;      // [4][B*N][C] fp32 route partials
   void* x_stage = nullptr;  // staging for srnl_scan_forward_host
   void* y_stage = nullptr;
+  int* dev_err = nullptr;   // device status word written by the scan kernel
   size_t ws_bytes = 0;
   // optional stage timing: a ring of event sets, 4 events per forward
   std::vector<cudaEvent_t> ev;
@@ -62,12 +63,13 @@ size_t act_bytes(const srnl_scan_config& c) {
 }
 
 void free_all(srnl_scan* h) {
-  void* ptrs[] = {h->Wq, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage};
+  void* ptrs[] = {h->Wq, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->Wq = h->G = h->Mm = h->scales = nullptr;
   h->q = h->x_stage = h->y_stage = nullptr;
   h->yr = nullptr;
+  h->dev_err = nullptr;
 }
 
 srnl_status validate_config(const srnl_scan_config* c) {
@@ -172,7 +174,8 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
       {(void**)&h->Wq, Wq.size() * sizeof(float)}, {(void**)&h->G, G.size() * sizeof(float)},
       {(void**)&h->Mm, n_mm * sizeof(float)},      {(void**)&h->scales, n_sc * sizeof(float)},
       {&h->q, q_bytes},                            {(void**)&h->yr, yr_bytes},
-      {&h->x_stage, stage_bytes},                  {&h->y_stage, stage_bytes}};
+      {&h->x_stage, stage_bytes},                  {&h->y_stage, stage_bytes},
+      {(void**)&h->dev_err, sizeof(int)}};
   for (auto& a : allocs) {
     e = cudaMalloc(a.p, a.n);
     if (e != cudaSuccess) {
@@ -188,6 +191,8 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
     e = cudaMemcpy(cp.dst, cp.src, cp.n, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemcpy (params)"); free_all(h); delete h; return st; }
   }
+  e = cudaMemset(h->dev_err, 0, sizeof(int));
+  if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemset (status)"); free_all(h); delete h; return st; }
   e = srnl::prepare_kernels();
   if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "kernel attributes"); free_all(h); delete h; return st; }
   *out = h;
@@ -202,7 +207,7 @@ static srnl_status run_forward(srnl_scan* h, const void* x, void* y, float* fina
   e = srnl::launch_query_projection(h->geom, p, x, h->q, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
-  e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, finals, s);
+  e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, finals, h->dev_err, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "scan launch");
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   e = srnl::launch_fuse(h->geom, h->yr, y, s);
@@ -324,6 +329,16 @@ srnl_status srnl_scan_stage_times(srnl_scan* h, float* ms_out, int* count) {
   for (int i = 0; i < 3; ++i) ms_out[i] = (float)(acc[i] / n);
   if (count != nullptr) *count = n;
   h->recorded = 0;
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_device_status(srnl_scan* h) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  int v = 0;
+  cudaError_t e = cudaMemcpy(&v, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "status read");
+  if (v != 0) return fail(h, static_cast<srnl_status>(v), "a bounded in-kernel wait gave up");
   return SRNL_OK;
 }
 

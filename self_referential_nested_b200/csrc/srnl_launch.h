@@ -27,8 +27,9 @@ cudaError_t launch_query_projection(const ScanGeom& g, const ScanParamsDev& p, c
 
 // Route partials yr[4][B*N][C] (fp32, already scaled by the fusion scales),
 // optional final states.
+// `err` (device int) receives SRNL_E_TIMEOUT if a bounded in-kernel wait gives up.
 cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
-                        float* yr, float* finals, cudaStream_t s);
+                        float* yr, float* finals, int* err, cudaStream_t s);
 
 // y = yr[0] + yr[1] + yr[2] + yr[3] in act dtype.
 cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_t s);
@@ -36,6 +37,7 @@ cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_
 cudaError_t launch_route_index(int route, int H, int W, int32_t* out, cudaStream_t s);
 cudaError_t launch_gather(const ScanGeom& g, int route, const void* x, void* xr, cudaStream_t s);
 
-cudaError_t prepare_kernels();  // one-time function attributes (dynamic smem)
+cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)
+cudaError_t prepare_scan_kernels();
 
 }  // namespace srnl

@@ -133,7 +133,8 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   const size_t wq_b = round_up(n_wq * 4), g_b = round_up(n_g * 4);
   const size_t q_b = round_up(tokens * cfg->C * (gen_bf16 ? 2 : 4));
   const size_t yr_b = round_up(4 * tokens * cfg->C * sizeof(float));
-  const size_t need = wq_b + g_b + q_b + yr_b;
+  const size_t err_b = 256;  // device status word of the scan kernel
+  const size_t need = err_b + wq_b + g_b + q_b + yr_b;
   if (need > kNoallocScratchBytes) {
     srnl::set_thread_error("workload needs " + std::to_string(need) +
                            " bytes of scratch; the no-allocation forward holds " +
@@ -144,6 +145,8 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   st = scratch_address(&base);
   if (st != SRNL_OK) return st;
   unsigned char* s8 = static_cast<unsigned char*>(base);
+  int* dev_err = reinterpret_cast<int*>(s8);
+  s8 += err_b;
   float* Wq = reinterpret_cast<float*>(s8);
   float* G = reinterpret_cast<float*>(s8 + wq_b);
   void* q = s8 + wq_b + g_b;
@@ -164,7 +167,7 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   g.act_bf16 = act_bf16; g.gen_bf16 = gen_bf16;
   const srnl::ScanParamsDev dp{Wq, G, p->M_mem0, p->scales};
   if (e == cudaSuccess) e = srnl::launch_query_projection(g, dp, x, q, cs);
-  if (e == cudaSuccess) e = srnl::launch_scan(g, dp, x, q, yr, nullptr, cs);
+  if (e == cudaSuccess) e = srnl::launch_scan(g, dp, x, q, yr, nullptr, dev_err, cs);
   if (e == cudaSuccess) e = srnl::launch_fuse(g, yr, y, cs);
   if (e != cudaSuccess) {
     srnl::set_thread_error(std::string("no-allocation forward launch: ") + cudaGetErrorString(e));
