@@ -14,27 +14,24 @@
 // sequence carries only Q:
 //   boundary generation  w_t = Q_b x_t,  [k~ v a beta]_t = G w_t
 //                        (G = [M_k0; M_v0; m_eta0; m_alpha0], 66 x 32)
-//   token-order write    row <- alpha_t row - eta_t (row . u_t) k_t  (per row of Q)
+//   token-order write    row <- alpha_t row - eta_t s_t k_t,  s_t = row . u_t
 //   readout              y_t = M_mem0 z_t,  z_t = Q_t q_t
-// Inside a block of 4 tokens the write is applied in closed form: with
-// A_t = alpha_1..alpha_t (block-relative),
-//   s_t = row_{t-1} . u_t = A_{t-1} (row_0 . u_t) - sum_{j<t} (A_{t-1}/A_j) eta_j (k_j . u_t) s_j
-//   z_t = row_t . q_t     = A_t (row_0 . q_t)     - sum_{j<=t} (A_t/A_j) eta_j (k_j . q_t) s_j
-//   row_4 = A_4 row_0 - sum_j (A_4/A_j) eta_j s_j k_j
-// which is the token-order recurrence reorganised (same terms, exact).
+// The write keeps two tokens of lookahead: with c1_t = k_t . u_{t+1} and
+// c2_t = k_t . u_{t+2} (shared by all rows),
+//   s_{t+2} = alpha_{t+1} (alpha_t (row_{t-1} . u_{t+2}) - eta_t c2_t s_t) - eta_{t+1} c1_{t+1} s_{t+1}
+// so each row's dot-product reduction has two tokens of slack before it is used.
 //
 // One CTA owns one (route, batch, head) sequence; 192 threads:
-//   warps 0-1  rows of Q: each lane holds 8 columns of two rows (rows rp and
-//              rp + 16), runs the block recursion and writes z_t (bf16 hi/lo)
-//   warps 2-3  one thread per token (TMEM lanes 64..127): gates from the
-//              generation MMA, the block tables, and the readout y from TMEM
-//   warps 4-5  asynchronous copies of the next stage's x and q
-//   all        boundary products w_t (SIMT)
-// Tensor cores (tcgen05, fp32 accumulate in TMEM):
-//   generation  [k~ v a beta] = w G^T     A = w (bf16), B = G (bf16), N = 80
-//               (bf16 path; the fp32 path runs this product on the SIMT pipes)
-//   readout     y = z M_mem0^T            3-term bf16 split of z and M_mem0
-//               (z_hi M_hi + z_hi M_lo + z_lo M_hi), about fp32 accuracy
+//   warps 0-3  rows of Q: four lanes per row, 8 columns per lane; the token
+//              loop above; z_t (bf16 hi/lo) into the readout operand tile
+//   warps 4-5  one thread per token (TMEM lanes 0..63): boundary products and
+//              generation drained from TMEM, gates, lookahead coefficients,
+//              readout y from TMEM, and asynchronous copies of the next stage
+// Tensor cores (tcgen05, fp32 accumulate in TMEM), bf16 path:
+//   boundary products  w = x Q_b^T     A = x (bf16), B = Q_b as bf16 hi + lo
+//   generation         [k~ v a beta] = w G^T    A = w (bf16), B = G (bf16)
+//   readout            y = z M_mem0^T  z and M_mem0 as bf16 hi + lo, three products
+// The fp32 path computes w and the generation on the SIMT pipes in fp32.
 // Tokens are staged kStage at a time; a chunk longer than kStage spans several
 // stages that all generate from the chunk's boundary Q_b.
 #include <cuda_bf16.h>
@@ -50,44 +47,45 @@ namespace srnl {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kCopyThreads = 64;  // warps 4-5
-constexpr int kStage = 64;       // tokens staged per pass
-constexpr int kGroup = 4;        // tokens per block of the row update
-constexpr int kPad = 36;         // padded fp32 row stride for per-token rows written row-wise
-constexpr int kGenStride = 68;   // padded stride of the SIMT generation rows (66 outputs)
-constexpr int kNgen = 80;        // generation MMA N: 66 outputs padded to a multiple of 16
-constexpr int kNy = 32;          // readout MMA N
-constexpr int kMmma = 128;       // MMA M; tokens occupy rows 64..127 (TMEM lanes of warps 2-3)
-constexpr int kTok0 = 64;        // first MMA row / TMEM lane holding a token
+constexpr int kRowWarps = 4;
+constexpr int kTokThreads = 64;   // warps 4-5
+constexpr int kStage = 64;        // tokens staged per pass
+constexpr int kPad = 36;          // padded fp32 row stride for per-token rows written row-wise
+constexpr int kGenStride = 68;    // padded stride of the SIMT generation rows (66 outputs)
+constexpr int kNgen = 80;         // generation MMA N: 66 outputs padded to a multiple of 16
+constexpr int kMmma = 128;        // MMA M; tokens occupy rows 0..63 (TMEM lanes of warps 4-5)
 constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kColGen = 0;  // TMEM columns of the generation accumulator
-constexpr uint32_t kColY = 96;   // TMEM columns of the readout accumulator
+constexpr uint32_t kColGen = 0;   // TMEM columns of the boundary-product / generation accumulator
+constexpr uint32_t kColY = 96;    // TMEM columns of the readout accumulator
 constexpr long long kWaitLimit = 1ll << 20;  // mbarrier polls before giving up
 
 struct alignas(128) Smem {
   union {
-    struct {                                      // bf16 path (tensor-core generation)
-      alignas(128) unsigned char a[kMmma * 64];   // w_t in bf16 (row 64 + t), K-major, no swizzle
-      alignas(128) unsigned char b[kNgen * 64];   // G in bf16
+    struct {                                      // bf16 path (tensor cores)
+      alignas(128) unsigned char xa[2][kMmma * 64];  // x in bf16, UMMA K-major tiles, double buffer
+      alignas(128) unsigned char wa[kMmma * 64];  // w in bf16 (generation A operand)
+      alignas(128) unsigned char gb[kNgen * 64];  // G in bf16 (generation B operand)
+      alignas(128) unsigned char qbh[kD * 64];    // Q_b bf16 high part (boundary-product B operand)
+      alignas(128) unsigned char qbl[kD * 64];    // Q_b bf16 low part
     } tc;
-    struct {                                      // fp32 path (SIMT generation)
+    struct {                                      // fp32 path (SIMT)
+      alignas(16) float x[2][kStage][kD];         // x head slices (source dtype), double buffer
       alignas(16) float w[kStage][kPad];          // w_t = Q_b x_t
       alignas(16) float gen[kStage][kGenStride];  // [k~ v a beta]
+      alignas(16) float qb[kD][kPad];             // Q_b
     } simt;
-    alignas(16) float qfin[kD][kD + 1];           // final-state staging (after the scan)
   } g;
-  alignas(128) unsigned char zh[kMmma * 64];      // z_t bf16 high part (row 64 + t), K = row of Q
+  alignas(128) unsigned char zh[kMmma * 64];      // z_t bf16 high part (row t), K = row of Q
   alignas(128) unsigned char zl[kMmma * 64];      // z_t bf16 low part
-  alignas(128) unsigned char mh[kNy * 64];        // M_mem0 bf16 high part (row = output channel)
-  alignas(128) unsigned char ml[kNy * 64];        // M_mem0 bf16 low part
-  alignas(16) float qb[kD][kPad];                 // boundary product Q_b of the current chunk
-  alignas(16) float x[2][kStage][kD];             // x head slices, route order, source dtype
-  alignas(16) float q[2][kStage][kD];             // q head slices, route order, source dtype
+  alignas(128) unsigned char mh[kD * 64];         // M_mem0 bf16 high part (row = output channel)
+  alignas(128) unsigned char ml[kD * 64];         // M_mem0 bf16 low part
+  alignas(16) float q[2][kStage][kD];             // q head slices (source dtype), double buffer
   alignas(16) float k[kStage][kPad];              // normalised keys
-  alignas(16) float u[kStage][kPad];              // u = (1 + alpha) k - v
-  alignas(16) float2 ae[kStage];                  // (alpha_t, eta_t)
-  alignas(16) float tbl[kStage / kGroup][32];     // per block: A_prev[4] A[4] W[4] P[6] N[10] A_G
+  alignas(16) float u[kStage + 2][kPad];          // u = (1 + alpha) k - v (two padding rows)
+  alignas(16) float4 ae[kStage + 2];              // (alpha, eta, eta c1, eta c2)
+  alignas(16) float qfin[kD][kD + 1];             // final-state staging
   alignas(16) float scale[kD];                    // fusion scales of this head's channels
+  alignas(8) unsigned long long mbar_w;           // boundary-product MMA completion
   alignas(8) unsigned long long mbar_g;           // generation MMA completion
   alignas(8) unsigned long long mbar_y;           // readout MMA completion
   uint32_t tmem_base;
@@ -121,7 +119,7 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
 }
 
 // Byte offset of element (row, k) of a [rows x 32] bf16 K-major operand tile.
-__device__ __forceinline__ uint32_t umma_off(int row, int k) {
+__host__ __device__ __forceinline__ uint32_t umma_off(int row, int k) {
   return (uint32_t)((row >> 3) * 512 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
 }
 
@@ -167,6 +165,10 @@ __device__ __forceinline__ void mbar_wait(unsigned long long* bar, uint32_t phas
     }
   }
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tok_bar() {  // named barrier of the two token warps
+  asm volatile("bar.sync 1, %0;" ::"n"(kTokThreads) : "memory");
 }
 
 __device__ __forceinline__ void store_bf16(unsigned char* tile, int row, int k, float v) {
@@ -220,6 +222,12 @@ __device__ __forceinline__ float dot32(const float (&a)[kD], const float* b) {
     acc2 = __ffma2_rn(f2(a[i + 2], a[i + 3]), f2(v.z, v.w), acc2);
   }
   return (acc.x + acc.y) + (acc2.x + acc2.y);
+}
+
+__device__ __forceinline__ float quad_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  return v;
 }
 
 // Gates of one token from its generated row (k~[32], v[32], a, beta): kt becomes the
@@ -300,27 +308,55 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
 
-// Warps 4-5: asynchronous copy of a stage's x and q head slices (source dtype).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Token warps: copy of a stage's q head slices (source dtype) and x head slices:
+// on the bf16 path x goes straight into its UMMA operand tile (bf16; fp32
+// activations are rounded), on the fp32 path into plain rows.
+template <bool kTC>
 __device__ __forceinline__ void prefetch_stage(Smem& sm, int buf, const StageInfo& si, const Args& a,
-                                               int r, int64_t tok0, int ch0, int hc) {
-  const int xe = a.act_bf16 ? 2 : 4, qe = a.q_bf16 ? 2 : 4;
-  const int xparts = kD * xe / 16, qparts = kD * qe / 16;  // 16-byte pieces per token slice
-  for (int idx = hc; idx < si.T * xparts; idx += kCopyThreads) {
-    const int tt = idx / xparts, part = idx - tt * xparts;
-    const int p = route_pos(r, si.t0 + tt, a.H, a.W);
-    const char* src = reinterpret_cast<const char*>(a.x) + ((tok0 + p) * a.C + ch0) * xe + part * 16;
-    cp_async16(reinterpret_cast<char*>(sm.x[buf][tt]) + part * 16, src);
-  }
-  for (int idx = hc; idx < si.T * qparts; idx += kCopyThreads) {
+                                               int r, int64_t tok0, int ch0, int ht) {
+  const int qe = a.q_bf16 ? 2 : 4;
+  const int qparts = kD * qe / 16;
+  for (int idx = ht; idx < si.T * qparts; idx += kTokThreads) {
     const int tt = idx / qparts, part = idx - tt * qparts;
     const int p = route_pos(r, si.t0 + tt, a.H, a.W);
     const char* src = reinterpret_cast<const char*>(a.q) + ((tok0 + p) * a.C + ch0) * qe + part * 16;
     cp_async16(reinterpret_cast<char*>(sm.q[buf][tt]) + part * 16, src);
   }
+  if (kTC && a.act_bf16) {  // 16 B = 8 bf16 channels = one core-matrix row
+    for (int idx = ht; idx < si.T * 4; idx += kTokThreads) {
+      const int tt = idx >> 2, part = idx & 3;
+      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
+      const char* src = reinterpret_cast<const char*>(a.x) + ((tok0 + p) * a.C + ch0) * 2 + part * 16;
+      cp_async16(sm.g.tc.xa[buf] + umma_off(tt, part * 8), src);
+    }
+  } else if (kTC) {  // fp32 activations, rounded to bf16 for the tensor cores
+    for (int idx = ht; idx < si.T * 4; idx += kTokThreads) {
+      const int tt = idx >> 2, part = idx & 3;
+      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
+      const float* src = reinterpret_cast<const float*>(a.x) + (tok0 + p) * a.C + ch0 + part * 8;
+      const float4 v0 = *reinterpret_cast<const float4*>(src);
+      const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(v0.x, v0.y), b1 = __floats2bfloat162_rn(v0.z, v0.w);
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(v1.x, v1.y), b3 = __floats2bfloat162_rn(v1.z, v1.w);
+      uint4 raw;
+      raw.x = *reinterpret_cast<uint32_t*>(&b0); raw.y = *reinterpret_cast<uint32_t*>(&b1);
+      raw.z = *reinterpret_cast<uint32_t*>(&b2); raw.w = *reinterpret_cast<uint32_t*>(&b3);
+      *reinterpret_cast<uint4*>(sm.g.tc.xa[buf] + umma_off(tt, part * 8)) = raw;
+    }
+  } else {
+    const int xe = a.act_bf16 ? 2 : 4;
+    const int xparts = kD * xe / 16;
+    for (int idx = ht; idx < si.T * xparts; idx += kTokThreads) {
+      const int tt = idx / xparts, part = idx - tt * xparts;
+      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
+      const char* src = reinterpret_cast<const char*>(a.x) + ((tok0 + p) * a.C + ch0) * xe + part * 16;
+      cp_async16(reinterpret_cast<char*>(sm.g.simt.x[buf][tt]) + part * 16, src);
+    }
+  }
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 #define SRNL_LD16(dst, addr)                                                                          \
   asm volatile(                                                                                       \
@@ -332,16 +368,18 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
         "=f"((dst)[15])                                                                               \
       : "r"(addr))
 
-// Warps 2-3: y_t = (readout accumulator row) scaled, stored at the token's raster slot.
-__device__ __forceinline__ void readout_from_tmem(Smem& sm, uint32_t tmem, const StageInfo& si,
-                                                  const Args& a, int r, int64_t tok0, int ch0, int gw,
-                                                  int gt) {
-  float y[kD];
-  const uint32_t ta = tmem + ((uint32_t)(kTok0 + 32 * gw) << 16) + kColY;
-  SRNL_LD16(y, ta);
-  SRNL_LD16(y + 16, ta + 16);
+__device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+// Token warps: y_t = (readout accumulator row) scaled, stored at the token's raster slot.
+__device__ __forceinline__ void readout_from_tmem(Smem& sm, uint32_t tmem_lane, const StageInfo& si,
+                                                  const Args& a, int r, int64_t tok0, int ch0, int gt) {
+  float y[kD];
+  SRNL_LD16(y, tmem_lane + kColY);
+  SRNL_LD16(y + 16, tmem_lane + kColY + 16);
+  tmem_wait_ld();
   if (gt < si.T) {
     const int p = route_pos(r, si.t0 + gt, a.H, a.W);
     float* dst = a.yr + ((int64_t)r * a.B * a.H * a.W + tok0 + p) * a.C + ch0;
@@ -360,14 +398,10 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const bool is_row = warp < 2;                  // warps 0-1: rows of Q
-  const bool is_gate = warp == 2 || warp == 3;   // warps 2-3: tokens (TMEM lanes 64..127)
-  const bool is_copy = warp >= 4;                // warps 4-5: prefetch
-  const int cq = lane & 3, cb = cq * 8;          // row lanes: column block
-  const int ra = (lane >> 2) + 8 * (warp & 1);   // row lanes: rows ra and ra + 16
-  const int rb = ra + 16;
-  const int gw = warp - 2, gt = tid - 64;        // token lanes: token gt of the stage
-  const int hc = tid - 128;
+  const bool is_row = warp < kRowWarps;          // warps 0-3: rows of Q
+  const bool is_tok = !is_row;                   // warps 4-5: tokens (TMEM lanes 0..63)
+  const int row = (tid >> 2) & 31, cq = tid & 3, cb = cq * 8;  // row lanes
+  const int gt = tid - kRowWarps * 32;           // token lanes: token gt of the stage
 
   const int seq = blockIdx.x;  // ((r * B + b) * heads + h)
   const int h = seq % a.heads;
@@ -383,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
   // ---- one-time set-up
   if (tid == 0) {
     sm.wait_failed = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_w)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_g)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_y)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -393,110 +428,142 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  if (kTC) {  // B operand of the generation MMA: G in bf16 (rows 66..79 zero)
+  for (int i = tid; i < kD * kD; i += kThreads) {
+    const int o = i / kD, kk = i % kD;
+    store_split(sm.mh, sm.ml, o, kk, Msrc[i]);  // readout B operand
+    if (kTC) store_split(sm.g.tc.qbh, sm.g.tc.qbl, o, kk, o == kk ? 1.f : 0.f);  // Q_b = I
+    else sm.g.simt.qb[o][kk] = (o == kk) ? 1.f : 0.f;
+  }
+  if (kTC) {  // generation B operand: G in bf16 (rows 66..79 zero)
     for (int i = tid; i < kNgen * kD; i += kThreads) {
       const int n = i / kD, kk = i % kD;
-      store_bf16(sm.g.tc.b, n, kk, n < kGen ? Gsrc[n * kD + kk] : 0.f);
+      store_bf16(sm.g.tc.gb, n, kk, n < kGen ? Gsrc[n * kD + kk] : 0.f);
     }
   }
-  for (int i = tid; i < kD * kD; i += kThreads) {  // readout B operand: M_mem0 hi/lo; Q_b = I
-    const int o = i / kD, kk = i % kD;
-    store_split(sm.mh, sm.ml, o, kk, Msrc[i]);
-    sm.qb[o][kk] = (o == kk) ? 1.f : 0.f;
-  }
   if (tid < kD) sm.scale[tid] = a.scales[r * a.C + ch0 + tid];
+  if (tid < 2) {  // the lookahead reads two rows past the stage: keep them inert
+    sm.ae[kStage + tid] = make_float4(1.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kD; ++i) sm.u[kStage + tid][i] = 0.f;
+  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
-  // row state: 8 columns of rows ra and rb (identity at the start)
-  float2 qa[4], qz[4];
+  // row state: this lane's 8 columns of row `row` (identity at the start)
+  float2 qr[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    qa[j] = f2((cb + 2 * j == ra) ? 1.f : 0.f, (cb + 2 * j + 1 == ra) ? 1.f : 0.f);
-    qz[j] = f2((cb + 2 * j == rb) ? 1.f : 0.f, (cb + 2 * j + 1 == rb) ? 1.f : 0.f);
-  }
+  for (int j = 0; j < 4; ++j)
+    qr[j] = f2((cb + 2 * j == row) ? 1.f : 0.f, (cb + 2 * j + 1 == row) ? 1.f : 0.f);
 
   const int nst = num_stages(N, L);
-  if (is_copy && nst > 0) {
-    prefetch_stage(sm, 0, stage_info(0, N, L), a, r, tok0, ch0, hc);
+  if (is_tok && nst > 0) {
+    prefetch_stage<kTC>(sm, 0, stage_info(0, N, L), a, r, tok0, ch0, gt);
     cp_async_wait_all();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t idesc_gen = idesc_bf16(kNgen), idesc_y = idesc_bf16(kNy);
+  const uint32_t tmem_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's TMEM lanes
+  const uint32_t idesc_w = idesc_bf16(kD), idesc_gen = idesc_bf16(kNgen), idesc_y = idesc_bf16(kD);
 
-  uint32_t phase_g = 0, phase_y = 0;
+  uint32_t phase_w = 0, phase_g = 0, phase_y = 0;
   bool y_pending = false;  // a readout MMA was issued and not yet consumed
   for (int st = 0; st < nst; ++st) {
     const int cur = st & 1;
     const StageInfo si = stage_info(st, N, L);
     const int T = si.T;
-    const int Tp = (T + kGroup - 1) & ~(kGroup - 1);
-    // ---- P1: boundary products w_t = Q_b x_t (all threads: lane = row, warp = token group)
-    {
-      float2 qv[16];
-#pragma unroll
-      for (int j = 0; j < 16; j += 2) {
-        const float4 v = *reinterpret_cast<const float4*>(&sm.qb[lane][2 * j]);
-        qv[j] = f2(v.x, v.y);
-        qv[j + 1] = f2(v.z, v.w);
-      }
-#pragma unroll 1
-      for (int tt = warp; tt < T; tt += kThreads / 32) {
-        float2 acc = f2(0.f, 0.f), acc2 = f2(0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float2 xv[4];
-          load8(sm.x[cur][tt], 8 * j, a.act_bf16, xv);
-          acc = __ffma2_rn(qv[4 * j], xv[0], acc);
-          acc2 = __ffma2_rn(qv[4 * j + 1], xv[1], acc2);
-          acc = __ffma2_rn(qv[4 * j + 2], xv[2], acc);
-          acc2 = __ffma2_rn(qv[4 * j + 3], xv[3], acc2);
+    // ---- generation: w = x Q_b^T, [k~ v a beta] = w G^T, gates, lookahead coefficients
+    if (kTC) {
+      if (is_tok && T > 0) {
+        if (gt == 0) {
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const uint32_t xa = smem_u32(sm.g.tc.xa[cur]);
+          mma_k32(tmem + kColGen, xa, smem_u32(sm.g.tc.qbh), idesc_w, false);
+          mma_k32(tmem + kColGen, xa, smem_u32(sm.g.tc.qbl), idesc_w, true);
+          mma_commit(&sm.mbar_w);
         }
-        const float w = (acc.x + acc.y) + (acc2.x + acc2.y);
-        if (kTC)
-          store_bf16(sm.g.tc.a, kTok0 + tt, lane, w);
-        else
-          sm.g.simt.w[tt][lane] = w;
-      }
-      if (kTC) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    __syncthreads();
-    // ---- P2: generation, gates and block tables (token lanes)
-    if (!kTC) {
-      // SIMT generation: thread (m = tid & 63, token group tid >> 6), m < 32 -> k~, else v
-      const int m = tid & 63;
-      float grow[kD];
+        mbar_wait(&sm.mbar_w, phase_w, &sm.wait_failed);
+        float wv[kD];
+        SRNL_LD16(wv, tmem_lane + kColGen);
+        SRNL_LD16(wv + 16, tmem_lane + kColGen + 16);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < kD; j += 4) {
-        const float4 g4 = __ldg(reinterpret_cast<const float4*>(Gsrc + m * kD + j));
-        grow[j] = g4.x; grow[j + 1] = g4.y; grow[j + 2] = g4.z; grow[j + 3] = g4.w;
-      }
-#pragma unroll 1
-      for (int tt = tid >> 6; tt < T; tt += kThreads / 64) sm.g.simt.gen[tt][m] = dot32(grow, sm.g.simt.w[tt]);
-      __syncthreads();
-    } else if (tid == 64 && T > 0) {
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      mma_k32(tmem + kColGen, smem_u32(sm.g.tc.a), smem_u32(sm.g.tc.b), idesc_gen, false);
-      mma_commit(&sm.mbar_g);
-    }
-    if (is_gate && T > 0) {
-      float kt[kD], vv[kD];
-      float ga = 0.f, gb = 0.f;
-      if (kTC) {
+        for (int c = 0; c < kD; c += 8) {  // one 16-byte core-matrix row per 8 columns
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(wv[c], wv[c + 1]);
+          __nv_bfloat162 b1 = __floats2bfloat162_rn(wv[c + 2], wv[c + 3]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(wv[c + 4], wv[c + 5]);
+          __nv_bfloat162 b3 = __floats2bfloat162_rn(wv[c + 6], wv[c + 7]);
+          uint4 raw;
+          raw.x = *reinterpret_cast<uint32_t*>(&b0); raw.y = *reinterpret_cast<uint32_t*>(&b1);
+          raw.z = *reinterpret_cast<uint32_t*>(&b2); raw.w = *reinterpret_cast<uint32_t*>(&b3);
+          *reinterpret_cast<uint4*>(sm.g.tc.wa + umma_off(gt, c)) = raw;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tok_bar();
+        if (gt == 0) {
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          mma_k32(tmem + kColGen, smem_u32(sm.g.tc.wa), smem_u32(sm.g.tc.gb), idesc_gen, false);
+          mma_commit(&sm.mbar_g);
+        }
         mbar_wait(&sm.mbar_g, phase_g, &sm.wait_failed);
-        const uint32_t ta = tmem + ((uint32_t)(kTok0 + 32 * gw) << 16) + kColGen;
-        SRNL_LD16(kt, ta);
-        SRNL_LD16(kt + 16, ta + 16);
-        SRNL_LD16(vv, ta + 32);
-        SRNL_LD16(vv + 16, ta + 48);
+        float kt[kD], vv[kD], ga, gb;
+        SRNL_LD16(kt, tmem_lane + kColGen);
+        SRNL_LD16(kt + 16, tmem_lane + kColGen + 16);
+        SRNL_LD16(vv, tmem_lane + kColGen + 32);
+        SRNL_LD16(vv + 16, tmem_lane + kColGen + 48);
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
                      : "=f"(ga), "=f"(gb)
-                     : "r"(ta + 64u));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      } else if (gt < T) {
+                     : "r"(tmem_lane + kColGen + 64u));
+        tmem_wait_ld();
+        if (gt < T) {
+          float al, eta;
+          gates_row(kt, vv, ga, gb, a.alpha, a.eps, al, eta);
+          store_row(sm.k[gt], kt);
+          store_row(sm.u[gt], vv);
+          sm.ae[gt] = make_float4(al, eta, 0.f, 0.f);
+        }
+      }
+    } else {
+      // SIMT: boundary products (all threads: lane = row, warp = token group), then generation
+      {
+        float2 qv[16];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          const float4 v = *reinterpret_cast<const float4*>(&sm.g.simt.qb[lane][2 * j]);
+          qv[j] = f2(v.x, v.y);
+          qv[j + 1] = f2(v.z, v.w);
+        }
+#pragma unroll 1
+        for (int tt = warp; tt < T; tt += kThreads / 32) {
+          float2 acc = f2(0.f, 0.f), acc2 = f2(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float2 xv[4];
+            load8(sm.g.simt.x[cur][tt], 8 * j, a.act_bf16, xv);
+            acc = __ffma2_rn(qv[4 * j], xv[0], acc);
+            acc2 = __ffma2_rn(qv[4 * j + 1], xv[1], acc2);
+            acc = __ffma2_rn(qv[4 * j + 2], xv[2], acc);
+            acc2 = __ffma2_rn(qv[4 * j + 3], xv[3], acc2);
+          }
+          sm.g.simt.w[tt][lane] = (acc.x + acc.y) + (acc2.x + acc2.y);
+        }
+      }
+      __syncthreads();
+      {
+        const int m = tid & 63;  // m < 32 -> k~, else v
+        float grow[kD];
+#pragma unroll
+        for (int j = 0; j < kD; j += 4) {
+          const float4 g4 = __ldg(reinterpret_cast<const float4*>(Gsrc + m * kD + j));
+          grow[j] = g4.x; grow[j + 1] = g4.y; grow[j + 2] = g4.z; grow[j + 3] = g4.w;
+        }
+#pragma unroll 1
+        for (int tt = tid >> 6; tt < T; tt += kThreads / 64) sm.g.simt.gen[tt][m] = dot32(grow, sm.g.simt.w[tt]);
+      }
+      __syncthreads();
+      if (is_tok && gt < T) {
+        float kt[kD], vv[kD], ga = 0.f, gb = 0.f;
         const float* wt = sm.g.simt.w[gt];
 #pragma unroll
         for (int i = 0; i < kD; ++i) {
@@ -505,184 +572,116 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
           ga = fmaf(Gsrc[2 * kD * kD + i], wt[i], ga);
           gb = fmaf(Gsrc[2 * kD * kD + kD + i], wt[i], gb);
         }
-      }
-      float al = 1.f, eta = 0.f;
-      if (gt < T) {
+        float al, eta;
         gates_row(kt, vv, ga, gb, a.alpha, a.eps, al, eta);
-      } else {  // pad to whole blocks: alpha = 1, eta = 0, k = u = 0 (inert tokens)
-#pragma unroll
-        for (int i = 0; i < kD; ++i) kt[i] = vv[i] = 0.f;
-      }
-      if (gt < Tp) {
         store_row(sm.k[gt], kt);
         store_row(sm.u[gt], vv);
-        sm.ae[gt] = make_float2(al, eta);
-      }
-      __syncwarp();
-      // tables of this token's block: P(t, j) = (A_{t-1}/A_j) eta_j (k_j . u_t),
-      // N(t, j) = (A_t/A_j) eta_j (k_j . q_t), W_j = (A_G/A_j) eta_j, A_{t-1}, A_t, A_G
-      if (gt < Tp) {
-        const int g0 = gt & ~(kGroup - 1), i = gt & (kGroup - 1);
-        float alb[kGroup], etb[kGroup];
-#pragma unroll
-        for (int m = 0; m < kGroup; ++m) {
-          const float2 v = sm.ae[g0 + m];
-          alb[m] = v.x;
-          etb[m] = v.y;
-        }
-        auto decay = [&](int j, int t) {  // prod_{m = j+1 .. t} alpha_m
-          float d = 1.f;
-#pragma unroll
-          for (int m = 0; m < kGroup; ++m)
-            if (m > j && m <= t) d *= alb[m];
-          return d;
-        };
-        float qt[kD];
-        if (gt < T) {
-#pragma unroll
-          for (int c = 0; c < kD; c += 8) {
-            float2 qv2[4];
-            load8(sm.q[cur][gt], c, a.q_bf16, qv2);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              qt[c + 2 * e] = qv2[e].x;
-              qt[c + 2 * e + 1] = qv2[e].y;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kD; ++c) qt[c] = 0.f;
-        }
-        float* tb = sm.tbl[g0 / kGroup];
-        tb[i] = decay(-1, i - 1);
-        tb[4 + i] = decay(-1, i);
-        tb[8 + i] = decay(i, kGroup - 1) * etb[i];
-        if (i == 0) tb[28] = decay(-1, kGroup - 1);
-#pragma unroll
-        for (int j = 0; j < kGroup; ++j) {
-          if (j > i) break;
-          const float* kj = sm.k[g0 + j];
-          if (j < i) tb[12 + i * (i - 1) / 2 + j] = decay(j, i - 1) * etb[j] * dot32(vv, kj);
-          tb[18 + i * (i + 1) / 2 + j] = decay(j, i) * etb[j] * dot32(qt, kj);
-        }
+        sm.ae[gt] = make_float4(al, eta, 0.f, 0.f);
       }
     }
-    if (kTC) phase_g ^= (T > 0) ? 1u : 0u;
+    if (is_tok && T > 0) {
+      tok_bar();
+      // lookahead coefficients eta_t (k_t . u_{t+1}) and eta_t (k_t . u_{t+2}); padding rows
+      if (gt < T) {
+        float kt[kD];
+#pragma unroll
+        for (int i = 0; i < kD; i += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(&sm.k[gt][i]);
+          kt[i] = v.x; kt[i + 1] = v.y; kt[i + 2] = v.z; kt[i + 3] = v.w;
+        }
+        const float eta = sm.ae[gt].y;
+        const float c1 = (gt + 1 < T) ? dot32(kt, sm.u[gt + 1]) : 0.f;
+        const float c2 = (gt + 2 < T) ? dot32(kt, sm.u[gt + 2]) : 0.f;
+        sm.ae[gt].z = eta * c1;
+        sm.ae[gt].w = eta * c2;
+      } else if (gt < T + 2) {
+        sm.ae[gt] = make_float4(1.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kD; ++i) sm.u[gt][i] = 0.f;
+      }
+    }
+    if (kTC && T > 0) {
+      phase_w ^= 1u;
+      phase_g ^= 1u;
+    }
     __syncthreads();
-    // ---- P4: rows | readout of the previous stage | prefetch of the next stage
+    // ---- token-order write (row warps) | readout + prefetch (token warps)
     if (is_row) {
       if (y_pending) mbar_wait(&sm.mbar_y, phase_y, &sm.wait_failed);  // z tiles free again
-      const int ng = Tp / kGroup;
+      if (T > 0) {
+        float2 uv[4];
+        load8f(sm.u[0] + cb, uv);
+        float s0 = quad_sum(dot8v(qr, uv));
+        load8f(sm.u[1] + cb, uv);
+        const float4 ae0 = sm.ae[0];
+        float s1 = fmaf(ae0.x, quad_sum(dot8v(qr, uv)), -ae0.z * s0);
+        float2 kc[4], qc[4], un[4];
+        load8f(sm.k[0] + cb, kc);
+        load8(sm.q[cur][0], cb, a.q_bf16, qc);
+        load8f(sm.u[2] + cb, un);
+        float4 ae_c = ae0;
 #pragma unroll 1
-      for (int gi = 0; gi < ng; ++gi) {
-        const int t0 = gi * kGroup;
-        // partial dots over this lane's 8 columns: b (row . u), e (row . q), rows ra and rb
-        float pb[2][kGroup], pe[2][kGroup];
+        for (int tt = 0; tt < T; ++tt) {
+          const float4 ae_n = sm.ae[tt + 1];
+          float2 kn[4], qn[4], un2[4];
+          load8f(sm.k[tt + 1 < kStage ? tt + 1 : tt] + cb, kn);  // rows past T are unused
+          load8(sm.q[cur][tt + 1 < kStage ? tt + 1 : tt], cb, a.q_bf16, qn);
+          load8f(sm.u[tt + 3 < kStage + 2 ? tt + 3 : kStage + 1] + cb, un2);
+          const float pp = dot8v(qr, un);              // row_{t-1} . u_{t+2}
+          const float cs = ae_c.y * s0;
+          const float2 al2 = f2(ae_c.x, ae_c.x), ncs = f2(-cs, -cs);
+          qr[0] = __ffma2_rn(ncs, kc[0], __fmul2_rn(al2, qr[0]));
+          qr[1] = __ffma2_rn(ncs, kc[1], __fmul2_rn(al2, qr[1]));
+          qr[2] = __ffma2_rn(ncs, kc[2], __fmul2_rn(al2, qr[2]));
+          qr[3] = __ffma2_rn(ncs, kc[3], __fmul2_rn(al2, qr[3]));
+          const float zt = quad_sum(dot8v(qr, qc));
+          if (cq == 0) store_split(sm.zh, sm.zl, tt, row, zt);
+          // s_{t+2} = alpha_{t+1} (alpha_t P - eta_t c2_t s_t) - eta_{t+1} c1_{t+1} s_{t+1}
+          const float s2 = fmaf(ae_n.x, fmaf(ae_c.x, quad_sum(pp), -ae_c.w * s0), -ae_n.z * s1);
+          s0 = s1;
+          s1 = s2;
+          ae_c = ae_n;
 #pragma unroll
-        for (int j = 0; j < kGroup; ++j) {
-          float2 v[4];
-          load8f(sm.u[t0 + j] + cb, v);
-          pb[0][j] = dot8v(qa, v);
-          pb[1][j] = dot8v(qz, v);
-          load8(sm.q[cur][t0 + j], cb, a.q_bf16, v);
-          pe[0][j] = dot8v(qa, v);
-          pe[1][j] = dot8v(qz, v);
-        }
-        // interleaved reductions over the 4 lanes of a row
-#pragma unroll
-        for (int o = 1; o <= 2; o <<= 1) {
-          float tb_[2][kGroup], te_[2][kGroup];
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-            for (int j = 0; j < kGroup; ++j) {
-              tb_[rr][j] = __shfl_xor_sync(0xffffffffu, pb[rr][j], o);
-              te_[rr][j] = __shfl_xor_sync(0xffffffffu, pe[rr][j], o);
-            }
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-            for (int j = 0; j < kGroup; ++j) {
-              pb[rr][j] += tb_[rr][j];
-              pe[rr][j] += te_[rr][j];
-            }
-        }
-        const float* tb = sm.tbl[gi];
-        const float4 Ap = *reinterpret_cast<const float4*>(tb);
-        const float4 Aa = *reinterpret_cast<const float4*>(tb + 4);
-        const float4 Wv = *reinterpret_cast<const float4*>(tb + 8);
-        const float4 P0 = *reinterpret_cast<const float4*>(tb + 12);   // P10 P20 P21 P30
-        const float4 P1 = *reinterpret_cast<const float4*>(tb + 16);   // P31 P32 N00 N10
-        const float4 N0 = *reinterpret_cast<const float4*>(tb + 20);   // N11 N20 N21 N22
-        const float4 N1 = *reinterpret_cast<const float4*>(tb + 24);   // N30 N31 N32 N33
-        const float AG = tb[28];
-        float sv[2][kGroup];
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const float* bp = pb[rr];
-          const float* ep = pe[rr];
-          // s_t = A_{t-1} b_t - sum_{j<t} P(t,j) s_j
-          const float s0 = Ap.x * bp[0];
-          const float s1 = fmaf(-P0.x, s0, Ap.y * bp[1]);
-          const float s2 = fmaf(-P0.z, s1, fmaf(-P0.y, s0, Ap.z * bp[2]));
-          const float s3 = fmaf(-P1.y, s2, fmaf(-P1.x, s1, fmaf(-P0.w, s0, Ap.w * bp[3])));
-          // z_t = A_t e_t - sum_{j<=t} N(t,j) s_j; lane cq handles token t0 + cq
-          float zs;
-          if (cq == 0) zs = fmaf(-P1.z, s0, Aa.x * ep[0]);
-          else if (cq == 1) zs = fmaf(-N0.x, s1, fmaf(-P1.w, s0, Aa.y * ep[1]));
-          else if (cq == 2) zs = fmaf(-N0.w, s2, fmaf(-N0.z, s1, fmaf(-N0.y, s0, Aa.z * ep[2])));
-          else zs = fmaf(-N1.w, s3, fmaf(-N1.z, s2, fmaf(-N1.y, s1, fmaf(-N1.x, s0, Aa.w * ep[3]))));
-          if (t0 + cq < T) store_split(sm.zh, sm.zl, kTok0 + t0 + cq, rr ? rb : ra, zs);
-          sv[rr][0] = s0; sv[rr][1] = s1; sv[rr][2] = s2; sv[rr][3] = s3;
-        }
-        // row <- A_G row - sum_j W_j s_j k_j (both rows, one key vector at a time)
-        {
-          const float2 ag = f2(AG, AG);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            qa[e] = __fmul2_rn(ag, qa[e]);
-            qz[e] = __fmul2_rn(ag, qz[e]);
-          }
-          const float wv[kGroup] = {Wv.x, Wv.y, Wv.z, Wv.w};
-#pragma unroll
-          for (int j = 0; j < kGroup; ++j) {
-            float2 kv[4];
-            load8f(sm.k[t0 + j] + cb, kv);
-            const float ca = -wv[j] * sv[0][j], cz = -wv[j] * sv[1][j];
-            const float2 na = f2(ca, ca), nz = f2(cz, cz);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              qa[e] = __ffma2_rn(na, kv[e], qa[e]);
-              qz[e] = __ffma2_rn(nz, kv[e], qz[e]);
-            }
+          for (int j = 0; j < 4; ++j) {
+            kc[j] = kn[j];
+            qc[j] = qn[j];
+            un[j] = un2[j];
           }
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       const StageInfo nx = stage_info(st + 1, N, L);
       if (st + 1 < nst && nx.chunk_start) {  // next stage opens a chunk: publish Q_b
-        *reinterpret_cast<float4*>(&sm.qb[ra][cb]) = make_float4(qa[0].x, qa[0].y, qa[1].x, qa[1].y);
-        *reinterpret_cast<float4*>(&sm.qb[ra][cb + 4]) = make_float4(qa[2].x, qa[2].y, qa[3].x, qa[3].y);
-        *reinterpret_cast<float4*>(&sm.qb[rb][cb]) = make_float4(qz[0].x, qz[0].y, qz[1].x, qz[1].y);
-        *reinterpret_cast<float4*>(&sm.qb[rb][cb + 4]) = make_float4(qz[2].x, qz[2].y, qz[3].x, qz[3].y);
-      }
-    } else if (is_gate) {
-      if (y_pending) {  // readout of the previous stage
-        mbar_wait(&sm.mbar_y, phase_y, &sm.wait_failed);
-        readout_from_tmem(sm, tmem, stage_info(st - 1, N, L), a, r, tok0, ch0, gw, gt);
+        if (kTC) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            store_split(sm.g.tc.qbh, sm.g.tc.qbl, row, cb + 2 * j, qr[j].x);
+            store_split(sm.g.tc.qbh, sm.g.tc.qbl, row, cb + 2 * j + 1, qr[j].y);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        } else {
+          *reinterpret_cast<float4*>(&sm.g.simt.qb[row][cb]) = make_float4(qr[0].x, qr[0].y, qr[1].x, qr[1].y);
+          *reinterpret_cast<float4*>(&sm.g.simt.qb[row][cb + 4]) = make_float4(qr[2].x, qr[2].y, qr[3].x, qr[3].y);
+        }
       }
     } else {
-      if (st + 1 < nst) prefetch_stage(sm, cur ^ 1, stage_info(st + 1, N, L), a, r, tok0, ch0, hc);
+      if (y_pending) {  // readout of the previous stage
+        mbar_wait(&sm.mbar_y, phase_y, &sm.wait_failed);
+        readout_from_tmem(sm, tmem_lane, stage_info(st - 1, N, L), a, r, tok0, ch0, gt);
+      }
+      if (st + 1 < nst) prefetch_stage<kTC>(sm, cur ^ 1, stage_info(st + 1, N, L), a, r, tok0, ch0, gt);
       cp_async_wait_all();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (y_pending) {
       phase_y ^= 1u;
       y_pending = false;
     }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     // ---- readout MMA of this stage: y = z M_mem0^T (3-term bf16 split)
     if (T > 0) {
-      if (tid == 64) {
+      if (tid == kRowWarps * 32) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t zh = smem_u32(sm.zh), zl = smem_u32(sm.zl);
         const uint32_t mh = smem_u32(sm.mh), ml = smem_u32(sm.ml);
@@ -694,9 +693,9 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
       y_pending = true;
     }
   }
-  if (y_pending && is_gate) {
+  if (y_pending && is_tok) {
     mbar_wait(&sm.mbar_y, phase_y, &sm.wait_failed);
-    readout_from_tmem(sm, tmem, stage_info(nst - 1, N, L), a, r, tok0, ch0, gw, gt);
+    readout_from_tmem(sm, tmem_lane, stage_info(nst - 1, N, L), a, r, tok0, ch0, gt);
   }
 
   __syncthreads();
@@ -707,10 +706,8 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
     if (is_row) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        sm.g.qfin[ra][cb + 2 * j] = qa[j].x;
-        sm.g.qfin[ra][cb + 2 * j + 1] = qa[j].y;
-        sm.g.qfin[rb][cb + 2 * j] = qz[j].x;
-        sm.g.qfin[rb][cb + 2 * j + 1] = qz[j].y;
+        sm.qfin[row][cb + 2 * j] = qr[j].x;
+        sm.qfin[row][cb + 2 * j + 1] = qr[j].y;
       }
     }
     __syncthreads();
@@ -718,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
     for (int mm = warp; mm < kMemRows; mm += kThreads / 32) {
       const float* src = (mm < kD) ? (Msrc + mm * kD) : (Gsrc + (mm - kD) * kD);
       float acc = 0.f;
-      for (int i = 0; i < kD; ++i) acc = fmaf(src[i], sm.g.qfin[i][lane], acc);
+      for (int i = 0; i < kD; ++i) acc = fmaf(src[i], sm.qfin[i][lane], acc);
       dst[mm * kD + lane] = acc;
     }
   }
