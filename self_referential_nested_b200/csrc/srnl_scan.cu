@@ -613,23 +613,14 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
         load8f(sm.u[0] + cb, uv);
         float s0 = quad_sum(dot8v(qr, uv));
         load8f(sm.u[1] + cb, uv);
-        const float4 ae0 = sm.ae[0];
-        float s1 = fmaf(ae0.x, quad_sum(dot8v(qr, uv)), -ae0.z * s0);
-        float2 kc[4], qc[4], un[4];
-        load8f(sm.k[0] + cb, kc);
-        load8(sm.q[cur][0], cb, a.q_bf16, qc);
-        load8f(sm.u[2] + cb, un);
-        float4 ae_c = ae0;
-#pragma unroll 1
-        for (int tt = 0; tt < T; ++tt) {
-          const float4 ae_n = sm.ae[tt + 1];
-          float2 kn[4], qn[4], un2[4];
-          load8f(sm.k[tt + 1 < kStage ? tt + 1 : tt] + cb, kn);  // rows past T are unused
-          load8(sm.q[cur][tt + 1 < kStage ? tt + 1 : tt], cb, a.q_bf16, qn);
-          load8f(sm.u[tt + 3 < kStage + 2 ? tt + 3 : kStage + 1] + cb, un2);
-          const float pp = dot8v(qr, un);              // row_{t-1} . u_{t+2}
-          const float cs = ae_c.y * s0;
-          const float2 al2 = f2(ae_c.x, ae_c.x), ncs = f2(-cs, -cs);
+        float4 ae_c = sm.ae[0];
+        float s1 = fmaf(ae_c.x, quad_sum(dot8v(qr, uv)), -ae_c.z * s0);
+        // one token of the write; operands of token tt (k, q, u_{tt+2}) in registers
+        auto step = [&](int tt, const float2 (&kc)[4], const float2 (&qc)[4], const float2 (&un)[4],
+                        const float4& ae_t, const float4& ae_n) {
+          const float pp = dot8v(qr, un);  // row_{t-1} . u_{t+2}
+          const float cs = ae_t.y * s0;
+          const float2 al2 = f2(ae_t.x, ae_t.x), ncs = f2(-cs, -cs);
           qr[0] = __ffma2_rn(ncs, kc[0], __fmul2_rn(al2, qr[0]));
           qr[1] = __ffma2_rn(ncs, kc[1], __fmul2_rn(al2, qr[1]));
           qr[2] = __ffma2_rn(ncs, kc[2], __fmul2_rn(al2, qr[2]));
@@ -637,16 +628,30 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
           const float zt = quad_sum(dot8v(qr, qc));
           if (cq == 0) store_split(sm.zh, sm.zl, tt, row, zt);
           // s_{t+2} = alpha_{t+1} (alpha_t P - eta_t c2_t s_t) - eta_{t+1} c1_{t+1} s_{t+1}
-          const float s2 = fmaf(ae_n.x, fmaf(ae_c.x, quad_sum(pp), -ae_c.w * s0), -ae_n.z * s1);
+          const float s2 = fmaf(ae_n.x, fmaf(ae_t.x, quad_sum(pp), -ae_t.w * s0), -ae_n.z * s1);
           s0 = s1;
           s1 = s2;
-          ae_c = ae_n;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            kc[j] = kn[j];
-            qc[j] = qn[j];
-            un[j] = un2[j];
-          }
+        };
+        float2 ka[4], qa_[4], ua[4], kb[4], qb_[4], ub[4];
+        load8f(sm.k[0] + cb, ka);
+        load8(sm.q[cur][0], cb, kTC, qa_);
+        load8f(sm.u[2] + cb, ua);
+#pragma unroll 1
+        for (int tt = 0; tt < T; tt += 2) {
+          // tokens tt (operands a) and tt + 1 (operands b); rows past T are inert or unused
+          const int t1 = tt + 1 < kStage ? tt + 1 : tt;
+          const float4 ae_1 = sm.ae[tt + 1];
+          load8f(sm.k[t1] + cb, kb);
+          load8(sm.q[cur][t1], cb, kTC, qb_);
+          load8f(sm.u[tt + 3] + cb, ub);
+          step(tt, ka, qa_, ua, ae_c, ae_1);
+          if (tt + 1 >= T) break;
+          const int t2 = tt + 2 < kStage ? tt + 2 : tt;
+          ae_c = sm.ae[tt + 2];
+          load8f(sm.k[t2] + cb, ka);
+          load8(sm.q[cur][t2], cb, kTC, qa_);
+          load8f(sm.u[tt + 4 < kStage + 2 ? tt + 4 : kStage + 1] + cb, ua);
+          step(tt + 1, kb, qb_, ub, ae_1, ae_c);
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
