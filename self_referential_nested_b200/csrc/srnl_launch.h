@@ -37,7 +37,12 @@ cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_
 cudaError_t launch_route_index(int route, int H, int W, int32_t* out, cudaStream_t s);
 cudaError_t launch_gather(const ScanGeom& g, int route, const void* x, void* xr, cudaStream_t s);
 
+// The chunkwise tensor-core scan (bf16 generation); launch_scan dispatches to it.
+cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
+                                  float* yr, float* finals, int* err, cudaStream_t s);
+
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)
 cudaError_t prepare_scan_kernels();
+cudaError_t prepare_scan_chunkwise_kernel();
 
 }  // namespace srnl

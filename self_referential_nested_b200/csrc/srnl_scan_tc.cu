@@ -1,0 +1,695 @@
+// SRNL four-direction chunked scan, bf16-generation path (sm_100a): the token-order
+// write in chunkwise form on the tensor cores.
+//
+// Method sources (web pages on VisionHOPE; no page prints an equation):
+//   "VisionHOPE: Visual Backbones as Self-Modifying Learning Systems" (summary
+//   of arXiv 2609.33325) - write-rule, stability and 2D-maps paragraphs;
+//   "VisionHOPE Model Overview: Architecture, Benchmarks, and Practical
+//   Limits" - "Four-Directional Scanning and Spatial Chunking"; "VisionHOPE"
+//   README - "SRNL and VisionHOPE operator".
+//
+// Single-product form: every write right-multiplies all memories by
+// T_t = alpha_t I - eta_t u_t k_t^T (u_t = (1 + alpha_t) k_t - v_t), so a sequence
+// carries one d x d product Q, generation reads w_t = Q_b x_t (Q_b: Q at the chunk
+// boundary) and the readout is y_t = M_mem0 Q_t q_t.
+//
+// Chunkwise write.  Inside a stage (up to 64 tokens of one chunk) all gates are
+// known before the first write, because generation only reads the boundary state.
+// For one row rho of Q (rho_s: the row at stage start) and the base-2 prefix
+// Lambda_t = sum_{m <= t} log2 alpha_m (Lambda_{-1} = 0), g(j, t) = 2^(Lambda_t - Lambda_j):
+//   rho_t = 2^Lambda_t rho_s - sum_{j <= t} g(j, t) eta_j s_j k_j,   s_t = rho_{t-1} . u_t
+// hence the s_t of every row solve one unit lower-triangular system that all rows share,
+//   s_t + sum_{j < t} A[t][j] s_j = 2^Lambda_{t-1} (rho_s . u_t),  A[t][j] = g(j, t-1) eta_j (u_t . k_j),
+// and the readout and the stage-end rows are products:
+//   z_t   = 2^Lambda_t (rho_s . q_t) - sum_{j <= t} g(j, t) eta_j (q_t . k_j) s_j
+//   rho_e = 2^Lambda_{T-1} rho_s - sum_j g(j, T-1) eta_j s_j k_j.
+// Only ratios g <= 1 of the retention products appear, so nothing overflows when a
+// retention gate is tiny.
+//
+// One CTA owns one (route, batch, head) sequence; 192 threads:
+//   warps 0-1  solve warps: A and the right-hand sides from TMEM lanes 0..63, then the
+//              forward substitution (two rows x 16 tokens per thread); warp 0 also
+//              forms the stage-end Q
+//   warps 2-3  readout warps: the readout coefficients from TMEM lanes 64..127, then
+//              z_t and the readout MMA of the previous stage
+//   warps 4-5  token warps: boundary products and generation, gates, the retention
+//              prefix, the copies of the next stage, and y_t from TMEM
+// Tensor-core products per stage (tcgen05, M = 128, fp32 accumulate in TMEM; an fp32
+// operand is split into bf16 hi + lo and a product of two such takes three MMAs):
+//   W    [x] Q_b^T                      N = 32   w_t = Q_b x_t
+//   Gen  [w] G^T                        N = 80   [k~ v a beta]_t
+//   M1   [u; q] [k; Q_s]^T              N = 96   u.k, Q_s u, q.k, Q_s q
+//   Z    [Kd^T; -; Mz^T] (-S)^T         N = 32   stage-end correction and z_t - 2^Lambda_t Q_s q_t
+//   Y    [z] M_mem0^T                   N = 32   y_t
+// TMEM holds two 128-column halves; consecutive stages alternate, so the readout of
+// one stage overlaps the generation of the next.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "srnl_common.cuh"
+#include "srnl_launch.h"
+#include "srnl_scan.h"
+#include "srnl_umma.cuh"
+
+namespace srnl {
+namespace {
+
+constexpr int kThreadsTc = 192;
+constexpr int kTile = kUmmaM * 64;      // 128 rows x 32 bf16: one K = 32 operand tile
+constexpr int kB1Rows = 96;             // M1 B operand: 64 keys + 32 rows of Q_s
+constexpr uint32_t kTmemColsTc = 256;   // two halves of 128 columns
+constexpr uint32_t kColM1 = 0;          // W, Gen, M1 and Y accumulate from column 0 of a half
+constexpr uint32_t kColZ0 = 64;         // M1 columns 64..95: Q_s u_t / Q_s q_t
+constexpr uint32_t kColZ = 96;          // Z accumulator
+
+struct alignas(128) TcSmem {
+  // x tile (rows 0..63 tokens, 64..127 zero); after the W product it holds w in bf16
+  alignas(128) unsigned char xa[kTile];
+  // M1 A operand: rows 0..63 u_t, rows 64..127 q_t (bf16, exact: its low part stays zero)
+  alignas(128) unsigned char a1h[kTile];
+  alignas(128) unsigned char a1l[kTile];
+  // M1 B operand: rows 0..63 k_j, rows 64..95 Q_s (row r, K = column)
+  alignas(128) unsigned char b1h[kB1Rows * 64];
+  alignas(128) unsigned char b1l[kB1Rows * 64];
+  // Z A operand, K halves j < 32 and j >= 32: rows 0..31 Kd^T, rows 32..63 free,
+  // rows 64..127 Mz^T.  Rows 32..63 hold the right-hand sides b^T during the solve.
+  alignas(128) unsigned char zah[2][kTile];
+  alignas(128) unsigned char zal[2][kTile];
+  // Z B operand: -S (row r, K = token j)
+  alignas(128) unsigned char zbh[2][kD * 64];
+  alignas(128) unsigned char zbl[2][kD * 64];
+  // Y A operand: z_t rows 0..63; the MMA's rows 64..127 read the next 4 KB (unused lanes)
+  alignas(128) unsigned char yah[64 * 64];
+  alignas(128) unsigned char yal[64 * 64];
+  alignas(128) unsigned char mh[kD * 64];      // M_mem0 hi (row = output channel)
+  alignas(128) unsigned char ml[kD * 64];      // M_mem0 lo
+  alignas(128) unsigned char gb[80 * 64];      // G in bf16 (rows 66..79 zero)
+  alignas(128) unsigned char qbh[kD * 64];     // Q_b hi (W product B operand)
+  alignas(128) unsigned char qbl[kD * 64];     // Q_b lo
+  alignas(16) float qsT[kD][kD + 1];            // Q_s transposed, fp32 (column c in row c)
+  alignas(16) float lam[kStage];                // Lambda_t (log2 retention prefix)
+  alignas(16) float eta[kStage];
+  alignas(16) float scale[kD];
+  float wsum;                                   // prefix of the first token warp
+  alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y;
+  uint32_t tmem_base;
+  int wait_failed;
+};
+static_assert(sizeof(TcSmem) <= 113 * 1024, "two CTAs per SM");
+static_assert(offsetof(TcSmem, yal) + 2 * 64 * 64 <= sizeof(TcSmem), "Y operand rows 64..127 stay in bounds");
+static_assert(offsetof(TcSmem, a1l) == offsetof(TcSmem, a1h) + kTile, "A pieces");
+static_assert(offsetof(TcSmem, b1h) == offsetof(TcSmem, a1h) + 2 * kTile, "A pieces");
+static_assert(offsetof(TcSmem, b1l) == offsetof(TcSmem, b1h) + kB1Rows * 64, "A pieces");
+static_assert(offsetof(TcSmem, zal) == offsetof(TcSmem, zah) + 2 * kTile, "b pieces");
+
+struct TcArgs {
+  const void* x;
+  const __nv_bfloat16* q;
+  float* yr;
+  float* finals;
+  int* err;
+  const float* G;
+  const float* Mm;
+  const float* scales;
+  int B, H, W, C, heads, Lrow, Lcol;
+  float alpha, eps;
+  bool act_bf16;
+};
+
+// -A[t][j] for j in [16p, 16p + 16) lives in the first 4 KB of a1h, a1l, b1h, b1l
+// (p = 0..3): the u and k rows of M1, dead between M1 and the next stage's gates.
+__device__ __forceinline__ float* neg_a_row(TcSmem& sm, int j) {
+  const int p = j >> 4;
+  unsigned char* base = p < 2 ? sm.a1h + p * kTile : sm.b1h + (p - 2) * (kB1Rows * 64);
+  return reinterpret_cast<float*>(base) + (j & 15) * kStage;
+}
+
+// b^T[r][t] (right-hand sides) in rows 32..63 of the four Z A sub-tiles.
+__device__ __forceinline__ float* rhs_row(TcSmem& sm, int r) {
+  return reinterpret_cast<float*>(&sm.zah[0][0] + (r >> 3) * kTile + 2048) + (r & 7) * kStage;
+}
+
+// 8 fp32 values -> bf16 hi and lo, each one 16-byte core-matrix row.
+__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 bh = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    const float2 fh = __bfloat1622float2(bh);
+    const __nv_bfloat162 bl = __floats2bfloat162_rn(v[2 * i] - fh.x, v[2 * i + 1] - fh.y);
+    h[i] = *reinterpret_cast<const uint32_t*>(&bh);
+    l[i] = *reinterpret_cast<const uint32_t*>(&bl);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Row `row` (32 fp32 values) of a K = 32 operand tile, as bf16 hi and lo.
+__device__ __forceinline__ void store_row_split(unsigned char* th, unsigned char* tl, int row, const float* v) {
+#pragma unroll
+  for (int c = 0; c < kD; c += 8) {
+    uint4 hi, lo;
+    split8(v + c, hi, lo);
+    *reinterpret_cast<uint4*>(th + umma_off(row, c)) = hi;
+    *reinterpret_cast<uint4*>(tl + umma_off(row, c)) = lo;
+  }
+}
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Number of stages that hold tokens: only the last chunk can be short.
+__device__ __forceinline__ int live_stages(int N, int L) {
+  const int per = (L + kStage - 1) / kStage;
+  const int chunks = (N + L - 1) / L;
+  const int last = N - (chunks - 1) * L;
+  return (chunks - 1) * per + (last + kStage - 1) / kStage;
+}
+
+// Token warps: asynchronous copies of a stage's x head slices (into the x tile; fp32
+// activations are rounded to bf16) and q head slices (into rows 64.. of the M1 A tile).
+__device__ __forceinline__ void tc_prefetch(TcSmem& sm, const StageInfo& si, const TcArgs& a, int r,
+                                            int64_t tok0, int ch0, int ht) {
+  for (int idx = ht; idx < si.T * 4; idx += 64) {
+    const int tt = idx >> 2, part = idx & 3;
+    const int p = route_pos(r, si.t0 + tt, a.H, a.W);
+    const __nv_bfloat16* src = a.q + (tok0 + p) * a.C + ch0 + part * 8;
+    cp_async16(sm.a1h + umma_off(64 + tt, part * 8), src);
+  }
+  if (a.act_bf16) {
+    for (int idx = ht; idx < si.T * 4; idx += 64) {
+      const int tt = idx >> 2, part = idx & 3;
+      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
+      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.x) + (tok0 + p) * a.C + ch0 + part * 8;
+      cp_async16(sm.xa + umma_off(tt, part * 8), src);
+    }
+  } else {
+    for (int idx = ht; idx < si.T * 4; idx += 64) {
+      const int tt = idx >> 2, part = idx & 3;
+      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
+      const float* src = reinterpret_cast<const float*>(a.x) + (tok0 + p) * a.C + ch0 + part * 8;
+      const float4 v0 = *reinterpret_cast<const float4*>(src);
+      const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+      const __nv_bfloat162 b0 = __floats2bfloat162_rn(v0.x, v0.y), b1 = __floats2bfloat162_rn(v0.z, v0.w);
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(v1.x, v1.y), b3 = __floats2bfloat162_rn(v1.z, v1.w);
+      uint4 raw;
+      raw.x = *reinterpret_cast<const uint32_t*>(&b0); raw.y = *reinterpret_cast<const uint32_t*>(&b1);
+      raw.z = *reinterpret_cast<const uint32_t*>(&b2); raw.w = *reinterpret_cast<const uint32_t*>(&b3);
+      *reinterpret_cast<uint4*>(sm.xa + umma_off(tt, part * 8)) = raw;
+    }
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(const TcArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const bool is_s = warp < 2;                  // solve warps (TMEM lanes 0..63)
+  const bool is_r = warp == 2 || warp == 3;    // readout warps (TMEM lanes 64..127)
+  const bool is_k = warp >= 4;                 // token warps (TMEM lanes 0..63)
+
+  const int seq = blockIdx.x;  // ((r * B + b) * heads + h)
+  const int h = seq % a.heads;
+  const int b = (seq / a.heads) % a.B;
+  const int r = seq / (a.heads * a.B);
+  const int N = a.H * a.W;
+  const int L = (r < 2) ? a.Lrow : a.Lcol;
+  const int64_t tok0 = (int64_t)b * N;
+  const int ch0 = h * kD;
+  const float* Gsrc = a.G + (int64_t)(r * a.heads + h) * kGen * kD;
+  const float* Msrc = a.Mm + (int64_t)(r * a.heads + h) * kD * kD;
+
+  // ---- set-up: zero the operand tiles, constants, Q_s = Q_b = I
+  {
+    uint4* z = reinterpret_cast<uint4*>(&sm);
+    const int n16 = (int)(offsetof(TcSmem, qsT) / 16);
+    for (int i = tid; i < n16; i += kThreadsTc) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (tid == 0) {
+    sm.wait_failed = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_w)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_g)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_1)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_z)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_y)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm.tmem_base)),
+                 "r"(kTmemColsTc));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  __syncthreads();
+  for (int i = tid; i < kD * kD; i += kThreadsTc) {
+    const int o = i / kD, kk = i % kD;
+    store_split(sm.mh, sm.ml, o, kk, Msrc[i]);
+    const float e = (o == kk) ? 1.f : 0.f;
+    store_split(sm.qbh, sm.qbl, o, kk, e);
+    store_split(sm.b1h, sm.b1l, 64 + o, kk, e);
+    sm.qsT[o][kk] = e;
+  }
+  for (int i = tid; i < 80 * kD; i += kThreadsTc) {
+    const int n = i / kD, kk = i % kD;
+    store_bf16(sm.gb, n, kk, n < kGen ? Gsrc[n * kD + kk] : 0.f);
+  }
+  if (tid < kD) sm.scale[tid] = a.scales[r * a.C + ch0 + tid];
+
+  const int nst = live_stages(N, L);
+  if (is_k && nst > 0) {
+    tc_prefetch(sm, stage_info(0, N, L), a, r, tok0, ch0, tid - 128);
+    cp_async_wait_all();
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t tmem_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+  const uint32_t idesc32 = idesc_bf16(32), idesc80 = idesc_bf16(80), idesc96 = idesc_bf16(96);
+
+  // readout warps: the stage whose z / y is still to be produced
+  bool pend = false;
+  StageInfo pst{0, 0, 0};
+  uint32_t phb = 0;
+  float ct_pend = 0.f;
+
+  for (int ne = 0; ne < nst; ++ne) {
+    const StageInfo si = stage_info(ne, N, L);
+    const int T = si.T;
+    const uint32_t hb = (uint32_t)(ne & 1) * 128u;
+    const uint32_t par = (uint32_t)(ne & 1);
+
+    // ---- (A) generation (token warps) | z and Y product of the previous stage (readout warps)
+    if (is_k) {
+      const int gt = tid - 128;
+      if (gt == 0) {
+        tc_fence_after();
+        mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), smem_u32(sm.qbh), idesc32, false);
+        mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), smem_u32(sm.qbl), idesc32, true);
+        mma_commit(&sm.mbar_w);
+      }
+      mbar_wait(&sm.mbar_w, par, &sm.wait_failed);
+      {
+        float wv[kD];
+        SRNL_LD16(wv, tmem_lane + hb + kColM1);
+        SRNL_LD16(wv + 16, tmem_lane + hb + kColM1 + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kD; c += 8) {
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(wv[c], wv[c + 1]);
+          const __nv_bfloat162 b1 = __floats2bfloat162_rn(wv[c + 2], wv[c + 3]);
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(wv[c + 4], wv[c + 5]);
+          const __nv_bfloat162 b3 = __floats2bfloat162_rn(wv[c + 6], wv[c + 7]);
+          uint4 raw;
+          raw.x = *reinterpret_cast<const uint32_t*>(&b0); raw.y = *reinterpret_cast<const uint32_t*>(&b1);
+          raw.z = *reinterpret_cast<const uint32_t*>(&b2); raw.w = *reinterpret_cast<const uint32_t*>(&b3);
+          *reinterpret_cast<uint4*>(sm.xa + umma_off(gt, c)) = raw;
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      tok_bar();
+      if (gt == 0) {
+        tc_fence_after();
+        mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), smem_u32(sm.gb), idesc80, false);
+        mma_commit(&sm.mbar_g);
+      }
+      mbar_wait(&sm.mbar_g, par, &sm.wait_failed);
+      float kt[kD], vv[kD], ga, gbeta;
+      SRNL_LD16(kt, tmem_lane + hb + kColM1);
+      SRNL_LD16(kt + 16, tmem_lane + hb + kColM1 + 16);
+      SRNL_LD16(vv, tmem_lane + hb + kColM1 + 32);
+      SRNL_LD16(vv + 16, tmem_lane + hb + kColM1 + 48);
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
+                   : "=f"(ga), "=f"(gbeta)
+                   : "r"(tmem_lane + hb + kColM1 + 64u));
+      tmem_wait_ld();
+      float l2a = 0.f, et = 0.f;
+      if (gt < T) {
+        float al;
+        gates_row(kt, vv, ga, gbeta, a.alpha, a.eps, al, et);
+        l2a = fmaxf(log2f(al), -126.f);  // a retention that underflows acts as 2^-126
+      } else {
+#pragma unroll
+        for (int i = 0; i < kD; ++i) { kt[i] = 0.f; vv[i] = 0.f; }
+      }
+      store_row_split(sm.a1h, sm.a1l, gt, vv);  // u_t
+      store_row_split(sm.b1h, sm.b1l, gt, kt);  // k_t
+      sm.eta[gt] = et;
+      // inclusive prefix of log2 alpha over the stage
+      float pre = l2a;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += v;
+      }
+      if (gt == 31) sm.wsum = pre;
+      tok_bar();
+      if (gt >= 32) pre += sm.wsum;
+      sm.lam[gt] = pre;
+      tok_bar();
+      // Kd^T[c][j] = g(j, T-1) eta_j k_j[c]: column j = gt of rows 0..31 of Z A
+      const float gk = (gt < T) ? exp2f(sm.lam[T - 1] - pre) * et : 0.f;
+      unsigned char* zh = sm.zah[gt >> 5];
+      unsigned char* zl = sm.zal[gt >> 5];
+#pragma unroll
+      for (int c = 0; c < kD; ++c) store_split(zh, zl, c, gt & 31, gk * kt[c]);
+      fence_async_smem();
+    } else if (is_r && pend) {
+      const int t = tid - 64;
+      mbar_wait(&sm.mbar_z, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
+      float z0[kD], zm[kD];
+      SRNL_LD16(z0, tmem_lane + phb + kColZ0);
+      SRNL_LD16(z0 + 16, tmem_lane + phb + kColZ0 + 16);
+      SRNL_LD16(zm, tmem_lane + phb + kColZ);
+      SRNL_LD16(zm + 16, tmem_lane + phb + kColZ + 16);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < kD; ++i) z0[i] = fmaf(ct_pend, z0[i], zm[i]);
+      store_row_split(sm.yah, sm.yal, t, z0);
+      fence_async_smem();
+      tc_fence_before();
+      named_bar(4, 64);
+      if (t == 0) {
+        tc_fence_after();
+        mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.mh), idesc32, false);
+        mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.ml), idesc32, true);
+        mma_k32(tmem + phb + kColM1, smem_u32(sm.yal), smem_u32(sm.mh), idesc32, true);
+        mma_commit(&sm.mbar_y);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    // ---- (C) M1 = [u; q] [k; Q_s]^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ah = smem_u32(sm.a1h), al = smem_u32(sm.a1l);
+      const uint32_t bh = smem_u32(sm.b1h), bl = smem_u32(sm.b1l);
+      mma_k32(tmem + hb + kColM1, ah, bh, idesc96, false);
+      mma_k32(tmem + hb + kColM1, ah, bl, idesc96, true);
+      mma_k32(tmem + hb + kColM1, al, bh, idesc96, true);
+      mma_commit(&sm.mbar_1);
+    }
+    // ---- (D) solve | readout coefficients | copies of the next stage and y of the previous one
+    if (is_s) {
+      mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
+      {
+        const int t = tid;  // TMEM lane = token
+        const bool live = t < T;
+        const float lp = (t > 0 && live) ? sm.lam[t - 1] : 0.f;  // Lambda_{t-1}
+        float g[16];
+#pragma unroll 1
+        for (int jb = 0; jb < kStage; jb += 16) {
+          SRNL_LD16(g, tmem_lane + hb + kColM1 + jb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
+            const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
+            const float lv[4] = {lj.x, lj.y, lj.z, lj.w}, ev[4] = {ej.x, ej.y, ej.z, ej.w};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const int j = jb + i + m;
+              const float v = (live && j < t) ? -exp2f(lp - lv[m]) * ev[m] * g[i + m] : 0.f;
+              neg_a_row(sm, j)[t] = v;
+            }
+          }
+        }
+        SRNL_LD16(g, tmem_lane + hb + kColZ0);
+        tmem_wait_ld();
+        const float cp = live ? exp2f(lp) : 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rhs_row(sm, i)[t] = cp * g[i];
+        SRNL_LD16(g, tmem_lane + hb + kColZ0 + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rhs_row(sm, 16 + i)[t] = cp * g[i];
+      }
+      tc_fence_before();
+      named_bar(2, 64);
+      // forward substitution: rows rp and rp + 16, tokens [16 qb, 16 qb + 16)
+      const int rp = 8 * warp + (lane & 7), qb = lane >> 3;
+      float2 s0[8], s1[8];
+      {
+        const float* b0 = rhs_row(sm, rp) + 16 * qb;
+        const float* b1 = rhs_row(sm, rp + 16) + 16 * qb;
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          const float4 v0 = *reinterpret_cast<const float4*>(b0 + 2 * i);
+          const float4 v1 = *reinterpret_cast<const float4*>(b1 + 2 * i);
+          s0[i] = f2(v0.x, v0.y); s0[i + 1] = f2(v0.z, v0.w);
+          s1[i] = f2(v1.x, v1.y); s1[i + 1] = f2(v1.z, v1.w);
+        }
+      }
+      const int nblk = (T + 15) >> 4;
+#pragma unroll 1
+      for (int qt = 0; qt < nblk; ++qt) {
+        const int src = (qt << 3) | (lane & 7);
+        const float* abase = neg_a_row(sm, 16 * qt) + 16 * qb;
+#pragma unroll
+        for (int tl = 0; tl < 16; ++tl) {
+          const float* ar = abase + tl * kStage;
+          const float4 a0 = *reinterpret_cast<const float4*>(ar);
+          const float4 a1 = *reinterpret_cast<const float4*>(ar + 4);
+          const float4 a2 = *reinterpret_cast<const float4*>(ar + 8);
+          const float4 a3 = *reinterpret_cast<const float4*>(ar + 12);
+          const float v0 = (tl & 1) ? s0[tl >> 1].y : s0[tl >> 1].x;
+          const float v1 = (tl & 1) ? s1[tl >> 1].y : s1[tl >> 1].x;
+          const float st0 = __shfl_sync(0xffffffffu, v0, src);
+          const float st1 = __shfl_sync(0xffffffffu, v1, src);
+          const float2 x0 = f2(st0, st0), x1 = f2(st1, st1);
+          const float2 av[8] = {f2(a0.x, a0.y), f2(a0.z, a0.w), f2(a1.x, a1.y), f2(a1.z, a1.w),
+                                f2(a2.x, a2.y), f2(a2.z, a2.w), f2(a3.x, a3.y), f2(a3.z, a3.w)};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            s0[i] = __ffma2_rn(av[i], x0, s0[i]);
+            s1[i] = __ffma2_rn(av[i], x1, s1[i]);
+          }
+        }
+      }
+      // -S into the Z B operand (row r, K = token)
+      {
+        unsigned char* th = sm.zbh[qb >> 1];
+        unsigned char* tl = sm.zbl[qb >> 1];
+        const int k0 = 16 * (qb & 1);
+        float v[8];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint4 hi, lo;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) { v[2 * i] = -s0[4 * half + i].x; v[2 * i + 1] = -s0[4 * half + i].y; }
+          split8(v, hi, lo);
+          *reinterpret_cast<uint4*>(th + umma_off(rp, k0 + 8 * half)) = hi;
+          *reinterpret_cast<uint4*>(tl + umma_off(rp, k0 + 8 * half)) = lo;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) { v[2 * i] = -s1[4 * half + i].x; v[2 * i + 1] = -s1[4 * half + i].y; }
+          split8(v, hi, lo);
+          *reinterpret_cast<uint4*>(th + umma_off(rp + 16, k0 + 8 * half)) = hi;
+          *reinterpret_cast<uint4*>(tl + umma_off(rp + 16, k0 + 8 * half)) = lo;
+        }
+      }
+      fence_async_smem();
+    } else if (is_r) {
+      mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
+      const int t = tid - 64;
+      const bool live = t < T;
+      const float lt = live ? sm.lam[t] : 0.f;
+      float g[16];
+#pragma unroll 1
+      for (int jb = 0; jb < kStage; jb += 16) {
+        SRNL_LD16(g, tmem_lane + hb + kColM1 + jb);
+        tmem_wait_ld();
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
+          const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
+          const float lv[4] = {lj.x, lj.y, lj.z, lj.w}, ev[4] = {ej.x, ej.y, ej.z, ej.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int j = jb + i + m;
+            v[i + m] = (live && j <= t) ? exp2f(lt - lv[m]) * ev[m] * g[i + m] : 0.f;
+          }
+        }
+        unsigned char* th = sm.zah[jb >> 5];
+        unsigned char* tl = sm.zal[jb >> 5];
+#pragma unroll
+        for (int c = 0; c < 16; c += 8) {
+          uint4 hi, lo;
+          split8(v + c, hi, lo);
+          *reinterpret_cast<uint4*>(th + umma_off(64 + t, (jb & 31) + c)) = hi;
+          *reinterpret_cast<uint4*>(tl + umma_off(64 + t, (jb & 31) + c)) = lo;
+        }
+      }
+      fence_async_smem();
+      ct_pend = live ? exp2f(lt) : 0.f;
+    } else {
+      const int gt = tid - 128;
+      mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
+      if (ne + 1 < nst) tc_prefetch(sm, stage_info(ne + 1, N, L), a, r, tok0, ch0, gt);
+      if (pend) {  // y of the previous stage: the Y product was issued in (A)
+        mbar_wait(&sm.mbar_y, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
+        float y[kD];
+        SRNL_LD16(y, tmem_lane + phb + kColM1);
+        SRNL_LD16(y + 16, tmem_lane + phb + kColM1 + 16);
+        tmem_wait_ld();
+        if (gt < pst.T) {
+          const int p = route_pos(r, pst.t0 + gt, a.H, a.W);
+          float* dst = a.yr + ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0;
+#pragma unroll
+          for (int i = 0; i < kD; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(sm.scale[i] * y[i], sm.scale[i + 1] * y[i + 1], sm.scale[i + 2] * y[i + 2],
+                            sm.scale[i + 3] * y[i + 3]);
+        }
+      }
+      cp_async_wait_all();
+      fence_async_smem();
+    }
+    // ---- (E) Z = [Kd^T; -; Mz^T] (-S)^T
+    if (!is_k) {
+      tc_fence_before();
+      named_bar(3, 128);
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t ah = smem_u32(sm.zah[kk]), al = smem_u32(sm.zal[kk]);
+          const uint32_t bh = smem_u32(sm.zbh[kk]), bl = smem_u32(sm.zbl[kk]);
+          mma_k32(tmem + hb + kColZ, ah, bh, idesc32, kk > 0);
+          mma_k32(tmem + hb + kColZ, ah, bl, idesc32, true);
+          mma_k32(tmem + hb + kColZ, al, bh, idesc32, true);
+        }
+        mma_commit(&sm.mbar_z);
+      }
+    }
+    // ---- (F) stage-end Q (warp 0: lane = column c)
+    if (warp == 0) {
+      mbar_wait(&sm.mbar_z, par, &sm.wait_failed);
+      float qc[kD];
+      SRNL_LD16(qc, tmem_lane + hb + kColZ);
+      SRNL_LD16(qc + 16, tmem_lane + hb + kColZ + 16);
+      tmem_wait_ld();
+      const float cT = exp2f(sm.lam[T - 1]);
+      float* col = sm.qsT[lane];
+#pragma unroll
+      for (int i = 0; i < kD; ++i) col[i] = fmaf(cT, col[i], qc[i]);
+      __syncwarp();
+      // lane = row r of Q_s: operand rows (hi/lo) of M1 and, at a chunk boundary, of W
+      float row[kD];
+#pragma unroll
+      for (int c = 0; c < kD; ++c) row[c] = sm.qsT[c][lane];
+      store_row_split(sm.b1h, sm.b1l, 64 + lane, row);
+      if (ne + 1 < nst && stage_info(ne + 1, N, L).chunk_start) store_row_split(sm.qbh, sm.qbl, lane, row);
+      fence_async_smem();
+    }
+    pend = true;
+    pst = si;
+    phb = hb;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  // ---- the last stage's z, Y product and y
+  if (is_r && pend) {
+    const int t = tid - 64;
+    mbar_wait(&sm.mbar_z, (uint32_t)((nst - 1) & 1), &sm.wait_failed);
+    float z0[kD], zm[kD];
+    SRNL_LD16(z0, tmem_lane + phb + kColZ0);
+    SRNL_LD16(z0 + 16, tmem_lane + phb + kColZ0 + 16);
+    SRNL_LD16(zm, tmem_lane + phb + kColZ);
+    SRNL_LD16(zm + 16, tmem_lane + phb + kColZ + 16);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < kD; ++i) z0[i] = fmaf(ct_pend, z0[i], zm[i]);
+    store_row_split(sm.yah, sm.yal, t, z0);
+    fence_async_smem();
+    tc_fence_before();
+    named_bar(4, 64);
+    if (t == 0) {
+      tc_fence_after();
+      mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.mh), idesc32, false);
+      mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.ml), idesc32, true);
+      mma_k32(tmem + phb + kColM1, smem_u32(sm.yal), smem_u32(sm.mh), idesc32, true);
+      mma_commit(&sm.mbar_y);
+    }
+  }
+  if (is_k && pend) {
+    const int gt = tid - 128;
+    mbar_wait(&sm.mbar_y, (uint32_t)((nst - 1) & 1), &sm.wait_failed);
+    float y[kD];
+    SRNL_LD16(y, tmem_lane + phb + kColM1);
+    SRNL_LD16(y + 16, tmem_lane + phb + kColM1 + 16);
+    tmem_wait_ld();
+    if (gt < pst.T) {
+      const int p = route_pos(r, pst.t0 + gt, a.H, a.W);
+      float* dst = a.yr + ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0;
+#pragma unroll
+      for (int i = 0; i < kD; i += 4)
+        *reinterpret_cast<float4*>(dst + i) = make_float4(sm.scale[i] * y[i], sm.scale[i + 1] * y[i + 1],
+                                                          sm.scale[i + 2] * y[i + 2], sm.scale[i + 3] * y[i + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (sm.wait_failed && tid == 0) atomicExch(a.err, SRNL_E_TIMEOUT);
+
+  if (a.finals != nullptr) {
+    // memories after the last token: [M_mem0; G] Q  (Q[i][c] = qsT[c][i])
+    float* dst = a.finals + (int64_t)seq * kStateFloats;
+    for (int mm = warp; mm < kMemRows; mm += kThreadsTc / 32) {
+      const float* src = (mm < kD) ? (Msrc + mm * kD) : (Gsrc + (mm - kD) * kD);
+      float acc = 0.f;
+      for (int i = 0; i < kD; ++i) acc = fmaf(src[i], sm.qsT[lane][i], acc);
+      dst[mm * kD + lane] = acc;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemColsTc));
+  }
+}
+
+}  // namespace
+
+cudaError_t prepare_scan_chunkwise_kernel() {
+  return cudaFuncSetAttribute(srnl_scan_chunkwise_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)sizeof(TcSmem));
+}
+
+cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
+                                  float* yr, float* finals, int* err, cudaStream_t s) {
+  TcArgs a;
+  a.x = x; a.q = static_cast<const __nv_bfloat16*>(q); a.yr = yr; a.finals = finals; a.err = err;
+  a.G = p.G; a.Mm = p.Mm; a.scales = p.scales;
+  a.B = g.B; a.H = g.H; a.W = g.W; a.C = g.C; a.heads = g.heads;
+  a.Lrow = g.Lrow; a.Lcol = g.Lcol; a.alpha = g.alpha; a.eps = g.eps;
+  a.act_bf16 = g.act_bf16;
+  const unsigned nseq = 4u * (unsigned)g.B * (unsigned)g.heads;
+  srnl_scan_chunkwise_kernel<<<nseq, kThreadsTc, sizeof(TcSmem), s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace srnl
