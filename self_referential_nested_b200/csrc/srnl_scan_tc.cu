@@ -157,6 +157,14 @@ __device__ __forceinline__ void store_row_split(unsigned char* th, unsigned char
   }
 }
 
+// 2^x on the MUFU (ex2.approx.ftz): the retention ratios g(j, t) <= 1 need no more, and a
+// ratio below 2^-126 is a decay to zero.
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -369,7 +377,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       sm.lam[gt] = pre;
       tok_bar();
       // Kd^T[c][j] = g(j, T-1) eta_j k_j[c]: column j = gt of rows 0..31 of Z A
-      const float gk = (gt < T) ? exp2f(sm.lam[T - 1] - pre) * et : 0.f;
+      const float gk = (gt < T) ? exp2_fast(sm.lam[T - 1] - pre) * et : 0.f;
       unsigned char* zh = sm.zah[gt >> 5];
       unsigned char* zl = sm.zal[gt >> 5];
 #pragma unroll
@@ -416,96 +424,102 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       {
         const int t = tid;  // TMEM lane = token
         const bool live = t < T;
+        float g[kStage], bv[kD];
+        SRNL_LD16(g, tmem_lane + hb + kColM1);
+        SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + 16);
+        SRNL_LD16(g + 32, tmem_lane + hb + kColM1 + 32);
+        SRNL_LD16(g + 48, tmem_lane + hb + kColM1 + 48);
+        SRNL_LD16(bv, tmem_lane + hb + kColZ0);
+        SRNL_LD16(bv + 16, tmem_lane + hb + kColZ0 + 16);
+        tmem_wait_ld();
         const float lp = (t > 0 && live) ? sm.lam[t - 1] : 0.f;  // Lambda_{t-1}
-        float g[16];
-#pragma unroll 1
+#pragma unroll
         for (int jb = 0; jb < kStage; jb += 16) {
-          SRNL_LD16(g, tmem_lane + hb + kColM1 + jb);
-          tmem_wait_ld();
+          // the block's Lambda_j and eta_j first: the stores below may alias them
+          float lv[16], ev[16], v[16];
 #pragma unroll
           for (int i = 0; i < 16; i += 4) {
             const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
             const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
-            const float lv[4] = {lj.x, lj.y, lj.z, lj.w}, ev[4] = {ej.x, ej.y, ej.z, ej.w};
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const int j = jb + i + m;
-              const float v = (live && j < t) ? -exp2f(lp - lv[m]) * ev[m] * g[i + m] : 0.f;
-              neg_a_row(sm, j)[t] = v;
-            }
+            lv[i] = lj.x; lv[i + 1] = lj.y; lv[i + 2] = lj.z; lv[i + 3] = lj.w;
+            ev[i] = ej.x; ev[i + 1] = ej.y; ev[i + 2] = ej.z; ev[i + 3] = ej.w;
           }
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            v[i] = (live && jb + i < t) ? -exp2_fast(lp - lv[i]) * ev[i] * g[jb + i] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) neg_a_row(sm, jb + i)[t] = v[i];
         }
-        SRNL_LD16(g, tmem_lane + hb + kColZ0);
-        tmem_wait_ld();
-        const float cp = live ? exp2f(lp) : 0.f;
+        const float cp = live ? exp2_fast(lp) : 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) rhs_row(sm, i)[t] = cp * g[i];
-        SRNL_LD16(g, tmem_lane + hb + kColZ0 + 16);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) rhs_row(sm, 16 + i)[t] = cp * g[i];
+        for (int i = 0; i < kD; ++i) rhs_row(sm, i)[t] = cp * bv[i];
       }
       tc_fence_before();
       named_bar(2, 64);
-      // forward substitution: rows rp and rp + 16, tokens [16 qb, 16 qb + 16)
-      const int rp = 8 * warp + (lane & 7), qb = lane >> 3;
-      float2 s0[8], s1[8];
-      {
-        const float* b0 = rhs_row(sm, rp) + 16 * qb;
-        const float* b1 = rhs_row(sm, rp + 16) + 16 * qb;
+      // Forward substitution.  Thread: rows rg + 8 m (m = 0..3, rg = 4 warp + (lane & 3)),
+      // tokens [8 kb, 8 kb + 8) (kb = lane >> 2).  Step t: the owner lanes of token t
+      // (kb == t / 8) broadcast the final s_t of each row; every lane subtracts
+      // A[t'][t] s_t from its tokens t' (A is zero for t' <= t).
+      const int rg = 4 * warp + (lane & 3), kb = lane >> 2;
+      float sv[4][8];
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-          const float4 v0 = *reinterpret_cast<const float4*>(b0 + 2 * i);
-          const float4 v1 = *reinterpret_cast<const float4*>(b1 + 2 * i);
-          s0[i] = f2(v0.x, v0.y); s0[i + 1] = f2(v0.z, v0.w);
-          s1[i] = f2(v1.x, v1.y); s1[i + 1] = f2(v1.z, v1.w);
-        }
+      for (int m = 0; m < 4; ++m) {
+        const float* src = rhs_row(sm, rg + 8 * m) + 8 * kb;
+        const float4 v0 = *reinterpret_cast<const float4*>(src);
+        const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+        sv[m][0] = v0.x; sv[m][1] = v0.y; sv[m][2] = v0.z; sv[m][3] = v0.w;
+        sv[m][4] = v1.x; sv[m][5] = v1.y; sv[m][6] = v1.z; sv[m][7] = v1.w;
       }
-      const int nblk = (T + 15) >> 4;
+      const int nblk = (T + 7) >> 3;
 #pragma unroll 1
-      for (int qt = 0; qt < nblk; ++qt) {
-        const int src = (qt << 3) | (lane & 7);
-        const float* abase = neg_a_row(sm, 16 * qt) + 16 * qb;
+      for (int bt = 0; bt < nblk; ++bt) {
+        const int src = (bt << 2) | (lane & 3);
+        const float* abase = neg_a_row(sm, 8 * bt) + 8 * kb;
 #pragma unroll
-        for (int tl = 0; tl < 16; ++tl) {
+        for (int tl = 0; tl < 8; ++tl) {
           const float* ar = abase + tl * kStage;
           const float4 a0 = *reinterpret_cast<const float4*>(ar);
           const float4 a1 = *reinterpret_cast<const float4*>(ar + 4);
-          const float4 a2 = *reinterpret_cast<const float4*>(ar + 8);
-          const float4 a3 = *reinterpret_cast<const float4*>(ar + 12);
-          const float v0 = (tl & 1) ? s0[tl >> 1].y : s0[tl >> 1].x;
-          const float v1 = (tl & 1) ? s1[tl >> 1].y : s1[tl >> 1].x;
-          const float st0 = __shfl_sync(0xffffffffu, v0, src);
-          const float st1 = __shfl_sync(0xffffffffu, v1, src);
-          const float2 x0 = f2(st0, st0), x1 = f2(st1, st1);
-          const float2 av[8] = {f2(a0.x, a0.y), f2(a0.z, a0.w), f2(a1.x, a1.y), f2(a1.z, a1.w),
-                                f2(a2.x, a2.y), f2(a2.z, a2.w), f2(a3.x, a3.y), f2(a3.z, a3.w)};
+          const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+          float st[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            s0[i] = __ffma2_rn(av[i], x0, s0[i]);
-            s1[i] = __ffma2_rn(av[i], x1, s1[i]);
+          for (int m = 0; m < 4; ++m) st[m] = __shfl_sync(0xffffffffu, sv[m][tl], src);
+          // the owner's next token first: it feeds the next shuffle
+          if (tl < 7) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) sv[m][tl + 1] = fmaf(av[tl + 1], st[m], sv[m][tl + 1]);
+          }
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              if (i + 1 == tl + 1) {
+                sv[m][i] = fmaf(av[i], st[m], sv[m][i]);
+              } else if (i == tl + 1) {
+                sv[m][i + 1] = fmaf(av[i + 1], st[m], sv[m][i + 1]);
+              } else {
+                const float2 r2 = __ffma2_rn(f2(av[i], av[i + 1]), f2(st[m], st[m]), f2(sv[m][i], sv[m][i + 1]));
+                sv[m][i] = r2.x;
+                sv[m][i + 1] = r2.y;
+              }
+            }
           }
         }
       }
-      // -S into the Z B operand (row r, K = token)
+      // -S into the Z B operand (row r, K = token): one core-matrix row per (row, hi/lo)
       {
-        unsigned char* th = sm.zbh[qb >> 1];
-        unsigned char* tl = sm.zbl[qb >> 1];
-        const int k0 = 16 * (qb & 1);
-        float v[8];
+        unsigned char* th = sm.zbh[kb >> 2];
+        unsigned char* tl = sm.zbl[kb >> 2];
+        const int k0 = 8 * (kb & 3);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int m = 0; m < 4; ++m) {
+          float v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = -sv[m][i];
           uint4 hi, lo;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) { v[2 * i] = -s0[4 * half + i].x; v[2 * i + 1] = -s0[4 * half + i].y; }
           split8(v, hi, lo);
-          *reinterpret_cast<uint4*>(th + umma_off(rp, k0 + 8 * half)) = hi;
-          *reinterpret_cast<uint4*>(tl + umma_off(rp, k0 + 8 * half)) = lo;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) { v[2 * i] = -s1[4 * half + i].x; v[2 * i + 1] = -s1[4 * half + i].y; }
-          split8(v, hi, lo);
-          *reinterpret_cast<uint4*>(th + umma_off(rp + 16, k0 + 8 * half)) = hi;
-          *reinterpret_cast<uint4*>(tl + umma_off(rp + 16, k0 + 8 * half)) = lo;
+          *reinterpret_cast<uint4*>(th + umma_off(rg + 8 * m, k0)) = hi;
+          *reinterpret_cast<uint4*>(tl + umma_off(rg + 8 * m, k0)) = lo;
         }
       }
       fence_async_smem();
@@ -514,23 +528,25 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       const int t = tid - 64;
       const bool live = t < T;
       const float lt = live ? sm.lam[t] : 0.f;
-      float g[16];
-#pragma unroll 1
+      float g[kStage];
+      SRNL_LD16(g, tmem_lane + hb + kColM1);
+      SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + 16);
+      SRNL_LD16(g + 32, tmem_lane + hb + kColM1 + 32);
+      SRNL_LD16(g + 48, tmem_lane + hb + kColM1 + 48);
+      tmem_wait_ld();
+#pragma unroll
       for (int jb = 0; jb < kStage; jb += 16) {
-        SRNL_LD16(g, tmem_lane + hb + kColM1 + jb);
-        tmem_wait_ld();
-        float v[16];
+        float lv[16], ev[16], v[16];
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
           const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
           const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
-          const float lv[4] = {lj.x, lj.y, lj.z, lj.w}, ev[4] = {ej.x, ej.y, ej.z, ej.w};
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int j = jb + i + m;
-            v[i + m] = (live && j <= t) ? exp2f(lt - lv[m]) * ev[m] * g[i + m] : 0.f;
-          }
+          lv[i] = lj.x; lv[i + 1] = lj.y; lv[i + 2] = lj.z; lv[i + 3] = lj.w;
+          ev[i] = ej.x; ev[i + 1] = ej.y; ev[i + 2] = ej.z; ev[i + 3] = ej.w;
         }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] = (live && jb + i <= t) ? exp2_fast(lt - lv[i]) * ev[i] * g[jb + i] : 0.f;
         unsigned char* th = sm.zah[jb >> 5];
         unsigned char* tl = sm.zal[jb >> 5];
 #pragma unroll
@@ -542,7 +558,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         }
       }
       fence_async_smem();
-      ct_pend = live ? exp2f(lt) : 0.f;
+      ct_pend = live ? exp2_fast(lt) : 0.f;
     } else {
       const int gt = tid - 128;
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
@@ -590,7 +606,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       SRNL_LD16(qc, tmem_lane + hb + kColZ);
       SRNL_LD16(qc + 16, tmem_lane + hb + kColZ + 16);
       tmem_wait_ld();
-      const float cT = exp2f(sm.lam[T - 1]);
+      const float cT = exp2_fast(sm.lam[T - 1]);
       float* col = sm.qsT[lane];
 #pragma unroll
       for (int i = 0; i < kD; ++i) col[i] = fmaf(cT, col[i], qc[i]);

@@ -152,7 +152,7 @@ __device__ __forceinline__ void gates_row(float (&kt)[kD], float (&vv)[kD], floa
     n2 = fmaf(kt[i + 2], kt[i + 2], n2);
     n3 = fmaf(kt[i + 3], kt[i + 3], n3);
   }
-  const float inv = 1.f / sqrtf(((n0 + n1) + (n2 + n3)) + eps);
+  const float inv = rsqrtf(((n0 + n1) + (n2 + n3)) + eps);
   float k0 = 0.f, k1 = 0.f, d0 = 0.f, d1 = 0.f;
 #pragma unroll
   for (int i = 0; i < kD; i += 2) {
@@ -166,20 +166,15 @@ __device__ __forceinline__ void gates_row(float (&kt)[kD], float (&vv)[kD], floa
     d1 = fmaf(db, db, d1);
   }
   const float kn2 = k0 + k1;
-  const float gain = sqrtf(d0 + d1) * sqrtf(kn2);
-  float sg;
-  if (beta >= 0.f) {
-    sg = 1.f / (1.f + expf(-beta));
-  } else {
-    const float e = expf(beta);
-    sg = e / (1.f + e);
-  }
+  const float gain = sqrtf((d0 + d1) * kn2);
+  const float eb = __expf(-fabsf(beta));  // sigmoid without overflow
+  const float sg = (beta >= 0.f) ? __fdividef(1.f, 1.f + eb) : __fdividef(eb, 1.f + eb);
   al = fminf(sg, alpha_max);
-  const float eta0 = fmaxf(a, 0.f) + log1pf(expf(-fabsf(a)));
-  const float zc = eta0 * gain / (1.f - al);
-  const float phi = (zc < 1e-4f) ? (1.f - zc * zc * (1.f / 3.f)) : tanhf(zc) / zc;
+  const float eta0 = fmaxf(a, 0.f) + log1pf(__expf(-fabsf(a)));
+  const float zc = __fdividef(eta0 * gain, 1.f - al);
+  const float phi = (zc < 1e-4f) ? (1.f - zc * zc * (1.f / 3.f)) : __fdividef(tanhf(zc), zc);
   eta = eta0 * phi;
-  if (eta * kn2 > 2.f) eta = 2.f / kn2;
+  if (eta * kn2 > 2.f) eta = __fdividef(2.f, kn2);
 #pragma unroll
   for (int i = 0; i < kD; ++i) vv[i] = (1.f + al) * kt[i] - vv[i];
 }
