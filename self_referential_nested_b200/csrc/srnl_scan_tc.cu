@@ -27,11 +27,11 @@
 // retention gate is tiny.
 //
 // One CTA owns one (route, batch, head) sequence; 192 threads:
-//   warps 0-1  solve warps: A and the right-hand sides from TMEM lanes 0..63, then the
-//              forward substitution (two rows x 16 tokens per thread); warp 0 also
-//              forms the stage-end Q
-//   warps 2-3  readout warps: the readout coefficients from TMEM lanes 64..127, then
+//   warps 0-1  solve warps: A and the right-hand sides from TMEM lanes 0..63; warp 0
+//              also forms the stage-end Q
+//   warps 2-3  readout warps: the readout coefficients from TMEM lanes 64..127, and
 //              z_t and the readout MMA of the previous stage
+//   warps 0-3  the forward substitution (four rows x four tokens per thread)
 //   warps 4-5  token warps: boundary products and generation, gates, the retention
 //              prefix, the copies of the next stage, and y_t from TMEM
 // Tensor-core products per stage (tcgen05, M = 128, fp32 accumulate in TMEM; an fp32
@@ -454,75 +454,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
 #pragma unroll
         for (int i = 0; i < kD; ++i) rhs_row(sm, i)[t] = cp * bv[i];
       }
-      tc_fence_before();
-      named_bar(2, 64);
-      // Forward substitution.  Thread: rows rg + 8 m (m = 0..3, rg = 4 warp + (lane & 3)),
-      // tokens [8 kb, 8 kb + 8) (kb = lane >> 2).  Step t: the owner lanes of token t
-      // (kb == t / 8) broadcast the final s_t of each row; every lane subtracts
-      // A[t'][t] s_t from its tokens t' (A is zero for t' <= t).
-      const int rg = 4 * warp + (lane & 3), kb = lane >> 2;
-      float sv[4][8];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float* src = rhs_row(sm, rg + 8 * m) + 8 * kb;
-        const float4 v0 = *reinterpret_cast<const float4*>(src);
-        const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
-        sv[m][0] = v0.x; sv[m][1] = v0.y; sv[m][2] = v0.z; sv[m][3] = v0.w;
-        sv[m][4] = v1.x; sv[m][5] = v1.y; sv[m][6] = v1.z; sv[m][7] = v1.w;
-      }
-      const int nblk = (T + 7) >> 3;
-#pragma unroll 1
-      for (int bt = 0; bt < nblk; ++bt) {
-        const int src = (bt << 2) | (lane & 3);
-        const float* abase = neg_a_row(sm, 8 * bt) + 8 * kb;
-#pragma unroll
-        for (int tl = 0; tl < 8; ++tl) {
-          const float* ar = abase + tl * kStage;
-          const float4 a0 = *reinterpret_cast<const float4*>(ar);
-          const float4 a1 = *reinterpret_cast<const float4*>(ar + 4);
-          const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-          float st[4];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) st[m] = __shfl_sync(0xffffffffu, sv[m][tl], src);
-          // the owner's next token first: it feeds the next shuffle
-          if (tl < 7) {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) sv[m][tl + 1] = fmaf(av[tl + 1], st[m], sv[m][tl + 1]);
-          }
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-              if (i + 1 == tl + 1) {
-                sv[m][i] = fmaf(av[i], st[m], sv[m][i]);
-              } else if (i == tl + 1) {
-                sv[m][i + 1] = fmaf(av[i + 1], st[m], sv[m][i + 1]);
-              } else {
-                const float2 r2 = __ffma2_rn(f2(av[i], av[i + 1]), f2(st[m], st[m]), f2(sv[m][i], sv[m][i + 1]));
-                sv[m][i] = r2.x;
-                sv[m][i + 1] = r2.y;
-              }
-            }
-          }
-        }
-      }
-      // -S into the Z B operand (row r, K = token): one core-matrix row per (row, hi/lo)
-      {
-        unsigned char* th = sm.zbh[kb >> 2];
-        unsigned char* tl = sm.zbl[kb >> 2];
-        const int k0 = 8 * (kb & 3);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          float v[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = -sv[m][i];
-          uint4 hi, lo;
-          split8(v, hi, lo);
-          *reinterpret_cast<uint4*>(th + umma_off(rg + 8 * m, k0)) = hi;
-          *reinterpret_cast<uint4*>(tl + umma_off(rg + 8 * m, k0)) = lo;
-        }
-      }
-      fence_async_smem();
     } else if (is_r) {
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
       const int t = tid - 64;
@@ -580,6 +511,73 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         }
       }
       cp_async_wait_all();
+      fence_async_smem();
+    }
+    // ---- forward substitution (warps 0-3).  Thread: rows rg + 8 m (m = 0..3, rg = 2 warp +
+    // (lane & 1)), tokens [4 kq, 4 kq + 4) (kq = lane >> 1).  Two tokens per broadcast: the
+    // owner lanes of tokens t, t + 1 (kq == t / 4) finish s_{t+1} = b_{t+1} - A[t+1][t] s_t
+    // from their registers, then every lane subtracts A[t'][t] s_t + A[t'][t+1] s_{t+1}
+    // from its tokens t' (A is zero for t' <= t, so finished tokens stay as they are).
+    if (!is_k) {
+      named_bar(5, 128);  // A, the right-hand sides and Mz^T are complete
+      const int rg = 2 * warp + (lane & 1), kq = lane >> 1;
+      float sv[4][4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float4 v = *reinterpret_cast<const float4*>(rhs_row(sm, rg + 8 * m) + 4 * kq);
+        sv[m][0] = v.x; sv[m][1] = v.y; sv[m][2] = v.z; sv[m][3] = v.w;
+      }
+      const int nb4 = (T + 3) >> 2;
+#pragma unroll 1
+      for (int bt = 0; bt < nb4; ++bt) {
+        const int src = (bt << 1) | (lane & 1);
+        const float* abase = neg_a_row(sm, 4 * bt) + 4 * kq;
+#pragma unroll
+        for (int tl = 0; tl < 4; tl += 2) {
+          const float4 p0 = *reinterpret_cast<const float4*>(abase + tl * kStage);
+          const float4 p1 = *reinterpret_cast<const float4*>(abase + (tl + 1) * kStage);
+          const float a0[4] = {p0.x, p0.y, p0.z, p0.w}, a1[4] = {p1.x, p1.y, p1.z, p1.w};
+          float xs[4], ys[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float xo = sv[m][tl];
+            const float yo = fmaf(a0[tl + 1], xo, sv[m][tl + 1]);
+            xs[m] = __shfl_sync(0xffffffffu, xo, src);
+            ys[m] = __shfl_sync(0xffffffffu, yo, src);
+          }
+          // the pair of tokens t + 2, t + 3 first: it feeds the next broadcast
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int i = ((tl + 2) & 3) ^ (2 * q);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const float2 r2 = __ffma2_rn(f2(a1[i], a1[i + 1]), f2(ys[m], ys[m]),
+                                           __ffma2_rn(f2(a0[i], a0[i + 1]), f2(xs[m], xs[m]), f2(sv[m][i], sv[m][i + 1])));
+              sv[m][i] = r2.x;
+              sv[m][i + 1] = r2.y;
+            }
+          }
+        }
+      }
+      // -S into the Z B operand (row r, K = token): half a core-matrix row per (row, hi/lo)
+      {
+        unsigned char* th = sm.zbh[kq >> 3];
+        unsigned char* tl = sm.zbl[kq >> 3];
+        const int k0 = (4 * kq) & 31;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const __nv_bfloat162 h0 = __floats2bfloat162_rn(-sv[m][0], -sv[m][1]);
+          const __nv_bfloat162 h1 = __floats2bfloat162_rn(-sv[m][2], -sv[m][3]);
+          const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+          const __nv_bfloat162 l0 = __floats2bfloat162_rn(-sv[m][0] - f0.x, -sv[m][1] - f0.y);
+          const __nv_bfloat162 l1 = __floats2bfloat162_rn(-sv[m][2] - f1.x, -sv[m][3] - f1.y);
+          uint2 hv, lv;
+          hv.x = *reinterpret_cast<const uint32_t*>(&h0); hv.y = *reinterpret_cast<const uint32_t*>(&h1);
+          lv.x = *reinterpret_cast<const uint32_t*>(&l0); lv.y = *reinterpret_cast<const uint32_t*>(&l1);
+          *reinterpret_cast<uint2*>(th + umma_off(rg + 8 * m, k0)) = hv;
+          *reinterpret_cast<uint2*>(tl + umma_off(rg + 8 * m, k0)) = lv;
+        }
+      }
       fence_async_smem();
     }
     // ---- (E) Z = [Kd^T; -; Mz^T] (-S)^T
