@@ -1,4 +1,5 @@
-// SRNL four-direction chunked scan: the sequence kernel (sm_100a).
+// SRNL four-direction chunked scan, fp32-generation path (sm_100a): the token-order
+// write one token at a time.
 //
 // Method sources (web pages on VisionHOPE; no page prints an equation):
 //   "VisionHOPE: Visual Backbones as Self-Modifying Learning Systems" (summary
@@ -21,17 +22,19 @@
 //   s_{t+2} = alpha_{t+1} (alpha_t (row_{t-1} . u_{t+2}) - eta_t c2_t s_t) - eta_{t+1} c1_{t+1} s_{t+1}
 // so each row's dot-product reduction has two tokens of slack before it is used.
 //
+// This kernel serves the fp32 generation path: boundary products and generation run
+// on the SIMT pipes in fp32, and every step of the write is an fp32 FMA, so its
+// results follow the sequential recurrence to fp32 rounding.  (The bf16 generation
+// path runs the chunkwise kernel in srnl_scan_tc.cu.)
+//
 // One CTA owns one (route, batch, head) sequence; 192 threads:
 //   warps 0-3  rows of Q: four lanes per row, 8 columns per lane; the token
 //              loop above; z_t (bf16 hi/lo) into the readout operand tile
-//   warps 4-5  one thread per token (TMEM lanes 0..63): boundary products and
-//              generation drained from TMEM, gates, lookahead coefficients,
-//              readout y from TMEM, and asynchronous copies of the next stage
-// Tensor cores (tcgen05, fp32 accumulate in TMEM), bf16 path:
-//   boundary products  w = x Q_b^T     A = x (bf16), B = Q_b as bf16 hi + lo
-//   generation         [k~ v a beta] = w G^T    A = w (bf16), B = G (bf16)
-//   readout            y = z M_mem0^T  z and M_mem0 as bf16 hi + lo, three products
-// The fp32 path computes w and the generation on the SIMT pipes in fp32.
+//   warps 4-5  one thread per token (TMEM lanes 0..63): gates, lookahead
+//              coefficients, readout y from TMEM, and asynchronous copies of the
+//              next stage
+// The readout y = z M_mem0^T runs on the tensor cores (tcgen05, z and M_mem0 as bf16
+// hi + lo, three products, fp32 accumulate in TMEM).
 // Tokens are staged kStage at a time; a chunk longer than kStage spans several
 // stages that all generate from the chunk's boundary Q_b.
 #include <cuda_bf16.h>
@@ -52,40 +55,27 @@ constexpr int kRowWarps = 4;
 constexpr int kTokThreads = 64;   // warps 4-5
 constexpr int kPad = 36;          // padded fp32 row stride for per-token rows written row-wise
 constexpr int kGenStride = 68;    // padded stride of the SIMT generation rows (66 outputs)
-constexpr int kNgen = 80;         // generation MMA N: 66 outputs padded to a multiple of 16
 constexpr int kMmma = kUmmaM;     // MMA M; tokens occupy rows 0..63 (TMEM lanes of warps 4-5)
-constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kColGen = 0;   // TMEM columns of the boundary-product / generation accumulator
-constexpr uint32_t kColY = 96;    // TMEM columns of the readout accumulator
+constexpr uint32_t kTmemCols = 32;
+constexpr uint32_t kColY = 0;     // TMEM columns of the readout accumulator
 
 struct alignas(128) Smem {
-  union {
-    struct {                                      // bf16 path (tensor cores)
-      alignas(128) unsigned char xa[2][kMmma * 64];  // x in bf16, UMMA K-major tiles, double buffer
-      alignas(128) unsigned char wa[kMmma * 64];  // w in bf16 (generation A operand)
-      alignas(128) unsigned char gb[kNgen * 64];  // G in bf16 (generation B operand)
-      alignas(128) unsigned char qbh[kD * 64];    // Q_b bf16 high part (boundary-product B operand)
-      alignas(128) unsigned char qbl[kD * 64];    // Q_b bf16 low part
-    } tc;
-    struct {                                      // fp32 path (SIMT)
-      alignas(16) float x[2][kStage][kD];         // x head slices (source dtype), double buffer
-      alignas(16) float w[kStage][kPad];          // w_t = Q_b x_t
-      alignas(16) float gen[kStage][kGenStride];  // [k~ v a beta]
-      alignas(16) float qb[kD][kPad];             // Q_b
-    } simt;
-  } g;
+  struct {
+    alignas(16) float x[2][kStage][kD];           // x head slices (source dtype), double buffer
+    alignas(16) float w[kStage][kPad];            // w_t = Q_b x_t
+    alignas(16) float gen[kStage][kGenStride];    // [k~ v a beta]
+    alignas(16) float qb[kD][kPad];               // Q_b
+  } simt;
   alignas(128) unsigned char zh[kMmma * 64];      // z_t bf16 high part (row t), K = row of Q
   alignas(128) unsigned char zl[kMmma * 64];      // z_t bf16 low part
   alignas(128) unsigned char mh[kD * 64];         // M_mem0 bf16 high part (row = output channel)
   alignas(128) unsigned char ml[kD * 64];         // M_mem0 bf16 low part
-  alignas(16) float q[2][kStage][kD];             // q head slices (source dtype), double buffer
+  alignas(16) float q[2][kStage][kD];             // q head slices (fp32), double buffer
   alignas(16) float k[kStage][kPad];              // normalised keys
   alignas(16) float u[kStage + 2][kPad];          // u = (1 + alpha) k - v (two padding rows)
   alignas(16) float4 ae[kStage + 2];              // (alpha, eta, eta c1, eta c2)
   alignas(16) float qfin[kD][kD + 1];             // final-state staging
   alignas(16) float scale[kD];                    // fusion scales of this head's channels
-  alignas(8) unsigned long long mbar_w;           // boundary-product MMA completion
-  alignas(8) unsigned long long mbar_g;           // generation MMA completion
   alignas(8) unsigned long long mbar_y;           // readout MMA completion
   uint32_t tmem_base;
   int wait_failed;
@@ -103,53 +93,25 @@ struct Args {
   const float* scales;
   int B, H, W, C, heads, Lrow, Lcol;
   float alpha, eps;
-  bool act_bf16, q_bf16;
+  bool act_bf16;  // q is fp32 on this path
 };
 
-// Token warps: copy of a stage's q head slices (source dtype) and x head slices:
-// on the bf16 path x goes straight into its UMMA operand tile (bf16; fp32
-// activations are rounded), on the fp32 path into plain rows.
-template <bool kTC>
+// Token warps: asynchronous copies of a stage's q (fp32) and x (source dtype) head slices.
 __device__ __forceinline__ void prefetch_stage(Smem& sm, int buf, const StageInfo& si, const Args& a,
                                                int r, int64_t tok0, int ch0, int ht) {
-  const int qe = a.q_bf16 ? 2 : 4;
-  const int qparts = kD * qe / 16;
-  for (int idx = ht; idx < si.T * qparts; idx += kTokThreads) {
-    const int tt = idx / qparts, part = idx - tt * qparts;
+  for (int idx = ht; idx < si.T * 8; idx += kTokThreads) {
+    const int tt = idx >> 3, part = idx & 7;
     const int p = route_pos(r, si.t0 + tt, a.H, a.W);
-    const char* src = reinterpret_cast<const char*>(a.q) + ((tok0 + p) * a.C + ch0) * qe + part * 16;
+    const char* src = reinterpret_cast<const char*>(a.q) + ((tok0 + p) * a.C + ch0) * 4 + part * 16;
     cp_async16(reinterpret_cast<char*>(sm.q[buf][tt]) + part * 16, src);
   }
-  if (kTC && a.act_bf16) {  // 16 B = 8 bf16 channels = one core-matrix row
-    for (int idx = ht; idx < si.T * 4; idx += kTokThreads) {
-      const int tt = idx >> 2, part = idx & 3;
-      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
-      const char* src = reinterpret_cast<const char*>(a.x) + ((tok0 + p) * a.C + ch0) * 2 + part * 16;
-      cp_async16(sm.g.tc.xa[buf] + umma_off(tt, part * 8), src);
-    }
-  } else if (kTC) {  // fp32 activations, rounded to bf16 for the tensor cores
-    for (int idx = ht; idx < si.T * 4; idx += kTokThreads) {
-      const int tt = idx >> 2, part = idx & 3;
-      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
-      const float* src = reinterpret_cast<const float*>(a.x) + (tok0 + p) * a.C + ch0 + part * 8;
-      const float4 v0 = *reinterpret_cast<const float4*>(src);
-      const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
-      __nv_bfloat162 b0 = __floats2bfloat162_rn(v0.x, v0.y), b1 = __floats2bfloat162_rn(v0.z, v0.w);
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(v1.x, v1.y), b3 = __floats2bfloat162_rn(v1.z, v1.w);
-      uint4 raw;
-      raw.x = *reinterpret_cast<uint32_t*>(&b0); raw.y = *reinterpret_cast<uint32_t*>(&b1);
-      raw.z = *reinterpret_cast<uint32_t*>(&b2); raw.w = *reinterpret_cast<uint32_t*>(&b3);
-      *reinterpret_cast<uint4*>(sm.g.tc.xa[buf] + umma_off(tt, part * 8)) = raw;
-    }
-  } else {
-    const int xe = a.act_bf16 ? 2 : 4;
-    const int xparts = kD * xe / 16;
-    for (int idx = ht; idx < si.T * xparts; idx += kTokThreads) {
-      const int tt = idx / xparts, part = idx - tt * xparts;
-      const int p = route_pos(r, si.t0 + tt, a.H, a.W);
-      const char* src = reinterpret_cast<const char*>(a.x) + ((tok0 + p) * a.C + ch0) * xe + part * 16;
-      cp_async16(reinterpret_cast<char*>(sm.g.simt.x[buf][tt]) + part * 16, src);
-    }
+  const int xe = a.act_bf16 ? 2 : 4;
+  const int xparts = kD * xe / 16;
+  for (int idx = ht; idx < si.T * xparts; idx += kTokThreads) {
+    const int tt = idx / xparts, part = idx - tt * xparts;
+    const int p = route_pos(r, si.t0 + tt, a.H, a.W);
+    const char* src = reinterpret_cast<const char*>(a.x) + ((tok0 + p) * a.C + ch0) * xe + part * 16;
+    cp_async16(reinterpret_cast<char*>(sm.simt.x[buf][tt]) + part * 16, src);
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -172,8 +134,7 @@ __device__ __forceinline__ void readout_from_tmem(Smem& sm, uint32_t tmem_lane, 
   }
 }
 
-template <bool kTC>
-__global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
+__global__ void __launch_bounds__(kThreads, 2) srnl_scan_sequential_kernel(const Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
 
@@ -198,8 +159,6 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
   // ---- one-time set-up
   if (tid == 0) {
     sm.wait_failed = 0;
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_w)));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_g)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_y)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -212,14 +171,7 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
   for (int i = tid; i < kD * kD; i += kThreads) {
     const int o = i / kD, kk = i % kD;
     store_split(sm.mh, sm.ml, o, kk, Msrc[i]);  // readout B operand
-    if (kTC) store_split(sm.g.tc.qbh, sm.g.tc.qbl, o, kk, o == kk ? 1.f : 0.f);  // Q_b = I
-    else sm.g.simt.qb[o][kk] = (o == kk) ? 1.f : 0.f;
-  }
-  if (kTC) {  // generation B operand: G in bf16 (rows 66..79 zero)
-    for (int i = tid; i < kNgen * kD; i += kThreads) {
-      const int n = i / kD, kk = i % kD;
-      store_bf16(sm.g.tc.gb, n, kk, n < kGen ? Gsrc[n * kD + kk] : 0.f);
-    }
+    sm.simt.qb[o][kk] = (o == kk) ? 1.f : 0.f;  // Q_b = I
   }
   if (tid < kD) sm.scale[tid] = a.scales[r * a.C + ch0 + tid];
   if (tid < 2) {  // the lookahead reads two rows past the stage: keep them inert
@@ -237,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
 
   const int nst = num_stages(N, L);
   if (is_tok && nst > 0) {
-    prefetch_stage<kTC>(sm, 0, stage_info(0, N, L), a, r, tok0, ch0, gt);
+    prefetch_stage(sm, 0, stage_info(0, N, L), a, r, tok0, ch0, gt);
     cp_async_wait_all();
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -246,72 +198,22 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = sm.tmem_base;
   const uint32_t tmem_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's TMEM lanes
-  const uint32_t idesc_w = idesc_bf16(kD), idesc_gen = idesc_bf16(kNgen), idesc_y = idesc_bf16(kD);
+  const uint32_t idesc_y = idesc_bf16(kD);
 
-  uint32_t phase_w = 0, phase_g = 0, phase_y = 0;
+  uint32_t phase_y = 0;
   bool y_pending = false;  // a readout MMA was issued and not yet consumed
   for (int st = 0; st < nst; ++st) {
     const int cur = st & 1;
     const StageInfo si = stage_info(st, N, L);
     const int T = si.T;
     // ---- generation: w = x Q_b^T, [k~ v a beta] = w G^T, gates, lookahead coefficients
-    if (kTC) {
-      if (is_tok && T > 0) {
-        if (gt == 0) {
-          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          const uint32_t xa = smem_u32(sm.g.tc.xa[cur]);
-          mma_k32(tmem + kColGen, xa, smem_u32(sm.g.tc.qbh), idesc_w, false);
-          mma_k32(tmem + kColGen, xa, smem_u32(sm.g.tc.qbl), idesc_w, true);
-          mma_commit(&sm.mbar_w);
-        }
-        mbar_wait(&sm.mbar_w, phase_w, &sm.wait_failed);
-        float wv[kD];
-        SRNL_LD16(wv, tmem_lane + kColGen);
-        SRNL_LD16(wv + 16, tmem_lane + kColGen + 16);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < kD; c += 8) {  // one 16-byte core-matrix row per 8 columns
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(wv[c], wv[c + 1]);
-          __nv_bfloat162 b1 = __floats2bfloat162_rn(wv[c + 2], wv[c + 3]);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(wv[c + 4], wv[c + 5]);
-          __nv_bfloat162 b3 = __floats2bfloat162_rn(wv[c + 6], wv[c + 7]);
-          uint4 raw;
-          raw.x = *reinterpret_cast<uint32_t*>(&b0); raw.y = *reinterpret_cast<uint32_t*>(&b1);
-          raw.z = *reinterpret_cast<uint32_t*>(&b2); raw.w = *reinterpret_cast<uint32_t*>(&b3);
-          *reinterpret_cast<uint4*>(sm.g.tc.wa + umma_off(gt, c)) = raw;
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        tok_bar();
-        if (gt == 0) {
-          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          mma_k32(tmem + kColGen, smem_u32(sm.g.tc.wa), smem_u32(sm.g.tc.gb), idesc_gen, false);
-          mma_commit(&sm.mbar_g);
-        }
-        mbar_wait(&sm.mbar_g, phase_g, &sm.wait_failed);
-        float kt[kD], vv[kD], ga, gb;
-        SRNL_LD16(kt, tmem_lane + kColGen);
-        SRNL_LD16(kt + 16, tmem_lane + kColGen + 16);
-        SRNL_LD16(vv, tmem_lane + kColGen + 32);
-        SRNL_LD16(vv + 16, tmem_lane + kColGen + 48);
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
-                     : "=f"(ga), "=f"(gb)
-                     : "r"(tmem_lane + kColGen + 64u));
-        tmem_wait_ld();
-        if (gt < T) {
-          float al, eta;
-          gates_row(kt, vv, ga, gb, a.alpha, a.eps, al, eta);
-          store_row(sm.k[gt], kt);
-          store_row(sm.u[gt], vv);
-          sm.ae[gt] = make_float4(al, eta, 0.f, 0.f);
-        }
-      }
-    } else {
+    {
       // SIMT: boundary products (all threads: lane = row, warp = token group), then generation
       {
         float2 qv[16];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
-          const float4 v = *reinterpret_cast<const float4*>(&sm.g.simt.qb[lane][2 * j]);
+          const float4 v = *reinterpret_cast<const float4*>(&sm.simt.qb[lane][2 * j]);
           qv[j] = f2(v.x, v.y);
           qv[j + 1] = f2(v.z, v.w);
         }
@@ -321,13 +223,13 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float2 xv[4];
-            load8(sm.g.simt.x[cur][tt], 8 * j, a.act_bf16, xv);
+            load8(sm.simt.x[cur][tt], 8 * j, a.act_bf16, xv);
             acc = __ffma2_rn(qv[4 * j], xv[0], acc);
             acc2 = __ffma2_rn(qv[4 * j + 1], xv[1], acc2);
             acc = __ffma2_rn(qv[4 * j + 2], xv[2], acc);
             acc2 = __ffma2_rn(qv[4 * j + 3], xv[3], acc2);
           }
-          sm.g.simt.w[tt][lane] = (acc.x + acc.y) + (acc2.x + acc2.y);
+          sm.simt.w[tt][lane] = (acc.x + acc.y) + (acc2.x + acc2.y);
         }
       }
       __syncthreads();
@@ -340,16 +242,16 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
           grow[j] = g4.x; grow[j + 1] = g4.y; grow[j + 2] = g4.z; grow[j + 3] = g4.w;
         }
 #pragma unroll 1
-        for (int tt = tid >> 6; tt < T; tt += kThreads / 64) sm.g.simt.gen[tt][m] = dot32(grow, sm.g.simt.w[tt]);
+        for (int tt = tid >> 6; tt < T; tt += kThreads / 64) sm.simt.gen[tt][m] = dot32(grow, sm.simt.w[tt]);
       }
       __syncthreads();
       if (is_tok && gt < T) {
         float kt[kD], vv[kD], ga = 0.f, gb = 0.f;
-        const float* wt = sm.g.simt.w[gt];
+        const float* wt = sm.simt.w[gt];
 #pragma unroll
         for (int i = 0; i < kD; ++i) {
-          kt[i] = sm.g.simt.gen[gt][i];
-          vv[i] = sm.g.simt.gen[gt][kD + i];
+          kt[i] = sm.simt.gen[gt][i];
+          vv[i] = sm.simt.gen[gt][kD + i];
           ga = fmaf(Gsrc[2 * kD * kD + i], wt[i], ga);
           gb = fmaf(Gsrc[2 * kD * kD + kD + i], wt[i], gb);
         }
@@ -381,10 +283,6 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
         for (int i = 0; i < kD; ++i) sm.u[gt][i] = 0.f;
       }
     }
-    if (kTC && T > 0) {
-      phase_w ^= 1u;
-      phase_g ^= 1u;
-    }
     __syncthreads();
     // ---- token-order write (row warps) | readout + prefetch (token warps)
     if (is_row) {
@@ -415,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
         };
         float2 ka[4], qa_[4], ua[4], kb[4], qb_[4], ub[4];
         load8f(sm.k[0] + cb, ka);
-        load8(sm.q[cur][0], cb, kTC, qa_);
+        load8f(sm.q[cur][0] + cb, qa_);
         load8f(sm.u[2] + cb, ua);
 #pragma unroll 1
         for (int tt = 0; tt < T; tt += 2) {
@@ -423,14 +321,14 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
           const int t1 = tt + 1 < kStage ? tt + 1 : tt;
           const float4 ae_1 = sm.ae[tt + 1];
           load8f(sm.k[t1] + cb, kb);
-          load8(sm.q[cur][t1], cb, kTC, qb_);
+          load8f(sm.q[cur][t1] + cb, qb_);
           load8f(sm.u[tt + 3] + cb, ub);
           step(tt, ka, qa_, ua, ae_c, ae_1);
           if (tt + 1 >= T) break;
           const int t2 = tt + 2 < kStage ? tt + 2 : tt;
           ae_c = sm.ae[tt + 2];
           load8f(sm.k[t2] + cb, ka);
-          load8(sm.q[cur][t2], cb, kTC, qa_);
+          load8f(sm.q[cur][t2] + cb, qa_);
           load8f(sm.u[tt + 4 < kStage + 2 ? tt + 4 : kStage + 1] + cb, ua);
           step(tt + 1, kb, qb_, ub, ae_1, ae_c);
         }
@@ -438,24 +336,15 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       const StageInfo nx = stage_info(st + 1, N, L);
       if (st + 1 < nst && nx.chunk_start) {  // next stage opens a chunk: publish Q_b
-        if (kTC) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            store_split(sm.g.tc.qbh, sm.g.tc.qbl, row, cb + 2 * j, qr[j].x);
-            store_split(sm.g.tc.qbh, sm.g.tc.qbl, row, cb + 2 * j + 1, qr[j].y);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        } else {
-          *reinterpret_cast<float4*>(&sm.g.simt.qb[row][cb]) = make_float4(qr[0].x, qr[0].y, qr[1].x, qr[1].y);
-          *reinterpret_cast<float4*>(&sm.g.simt.qb[row][cb + 4]) = make_float4(qr[2].x, qr[2].y, qr[3].x, qr[3].y);
-        }
+        *reinterpret_cast<float4*>(&sm.simt.qb[row][cb]) = make_float4(qr[0].x, qr[0].y, qr[1].x, qr[1].y);
+        *reinterpret_cast<float4*>(&sm.simt.qb[row][cb + 4]) = make_float4(qr[2].x, qr[2].y, qr[3].x, qr[3].y);
       }
     } else {
       if (y_pending) {  // readout of the previous stage
         mbar_wait(&sm.mbar_y, phase_y, &sm.wait_failed);
         readout_from_tmem(sm, tmem_lane, stage_info(st - 1, N, L), a, r, tok0, ch0, gt);
       }
-      if (st + 1 < nst) prefetch_stage<kTC>(sm, cur ^ 1, stage_info(st + 1, N, L), a, r, tok0, ch0, gt);
+      if (st + 1 < nst) prefetch_stage(sm, cur ^ 1, stage_info(st + 1, N, L), a, r, tok0, ch0, gt);
       cp_async_wait_all();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -516,11 +405,8 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan2_kernel(const Args a) {
 }  // namespace
 
 cudaError_t prepare_scan_kernels() {
-  cudaError_t e = cudaFuncSetAttribute(srnl_scan2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)sizeof(Smem));
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(srnl_scan2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)sizeof(Smem));
+  const cudaError_t e = cudaFuncSetAttribute(srnl_scan_sequential_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
   if (e != cudaSuccess) return e;
   return prepare_scan_chunkwise_kernel();
 }
@@ -533,12 +419,9 @@ cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x
   a.G = p.G; a.Mm = p.Mm; a.scales = p.scales;
   a.B = g.B; a.H = g.H; a.W = g.W; a.C = g.C; a.heads = g.heads;
   a.Lrow = g.Lrow; a.Lcol = g.Lcol; a.alpha = g.alpha; a.eps = g.eps;
-  a.act_bf16 = g.act_bf16; a.q_bf16 = g.gen_bf16;
+  a.act_bf16 = g.act_bf16;
   const unsigned nseq = 4u * (unsigned)g.B * (unsigned)g.heads;
-  if (g.gen_bf16)
-    srnl_scan2_kernel<true><<<nseq, kThreads, sizeof(Smem), s>>>(a);
-  else
-    srnl_scan2_kernel<false><<<nseq, kThreads, sizeof(Smem), s>>>(a);
+  srnl_scan_sequential_kernel<<<nseq, kThreads, sizeof(Smem), s>>>(a);
   return cudaGetLastError();
 }
 

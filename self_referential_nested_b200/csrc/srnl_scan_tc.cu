@@ -26,14 +26,16 @@
 // Only ratios g <= 1 of the retention products appear, so nothing overflows when a
 // retention gate is tiny.
 //
-// One CTA owns one (route, batch, head) sequence; 192 threads:
-//   warps 0-1  solve warps: A and the right-hand sides from TMEM lanes 0..63; warp 0
-//              also forms the stage-end Q
-//   warps 2-3  readout warps: the readout coefficients from TMEM lanes 64..127, and
-//              z_t and the readout MMA of the previous stage
-//   warps 0-3  the forward substitution (four rows x four tokens per thread)
-//   warps 4-5  token warps: boundary products and generation, gates, the retention
-//              prefix, the copies of the next stage, and y_t from TMEM
+// One CTA owns one (route, batch, head) sequence; 192 threads.  Warp w runs on SMSP w % 4
+// and reads TMEM lanes 32 (w % 4) .. + 31, which fixes who can drain which accumulator rows:
+//   warps 0-1  solve warps: half of -A from TMEM lanes 0..63, the forward substitution
+//              (four rows x eight tokens per thread); warp 0 also forms the stage-end Q
+//   warps 2-3  readout warps: half of the gate vector work (tokens repeated in TMEM lanes
+//              64..127), the readout coefficients from lanes 64..127 during the
+//              substitution, z_t and the Y product of the previous stage
+//   warps 4-5  token warps: boundary products and generation, the gate scalars, the
+//              retention prefix, the other half of the gate vector work, of -A and the
+//              right-hand sides, the copies of the next stage and y_t from TMEM
 // Tensor-core products per stage (tcgen05, M = 128, fp32 accumulate in TMEM; an fp32
 // operand is split into bf16 hi + lo and a product of two such takes three MMAs):
 //   W    [x] Q_b^T                      N = 32   w_t = Q_b x_t
@@ -65,7 +67,7 @@ constexpr uint32_t kColZ0 = 64;         // M1 columns 64..95: Q_s u_t / Q_s q_t
 constexpr uint32_t kColZ = 96;          // Z accumulator
 
 struct alignas(128) TcSmem {
-  // x tile (rows 0..63 tokens, 64..127 zero); after the W product it holds w in bf16
+  // x tile (token t in rows t and 64 + t); after the W product it holds w in bf16
   alignas(128) unsigned char xa[kTile];
   // M1 A operand: rows 0..63 u_t, rows 64..127 q_t (bf16, exact: its low part stays zero)
   alignas(128) unsigned char a1h[kTile];
@@ -92,6 +94,8 @@ struct alignas(128) TcSmem {
   alignas(16) float lam[kStage];                // Lambda_t (log2 retention prefix)
   alignas(16) float eta[kStage];
   alignas(16) float scale[kD];
+  alignas(16) float4 gpart[kStage];            // readout-warp halves of ||k~||^2, k~.v, ||v||^2
+  alignas(16) float4 gpar[kStage];             // gate scalars: 1/||k~||, alpha, g(t, T-1) eta, live
   float wsum;                                   // prefix of the first token warp
   alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y;
   uint32_t tmem_base;
@@ -165,6 +169,22 @@ __device__ __forceinline__ float exp2_fast(float x) {
   return y;
 }
 
+// Columns [c0, c0 + 16) of row `row` of a K = 32 operand tile, as bf16 hi and lo.
+__device__ __forceinline__ void store_half_split(unsigned char* th, unsigned char* tl, int row, int c0,
+                                                 const float* v) {
+#pragma unroll
+  for (int c = 0; c < 16; c += 8) {
+    uint4 hi, lo;
+    split8(v + c, hi, lo);
+    *reinterpret_cast<uint4*>(th + umma_off(row, c0 + c)) = hi;
+    *reinterpret_cast<uint4*>(tl + umma_off(row, c0 + c)) = lo;
+  }
+}
+
+__device__ __forceinline__ void named_bar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -189,8 +209,8 @@ __device__ __forceinline__ int live_stages(int N, int L) {
   return (chunks - 1) * per + (last + kStage - 1) / kStage;
 }
 
-// Token warps: asynchronous copies of a stage's x head slices (into the x tile; fp32
-// activations are rounded to bf16) and q head slices (into rows 64.. of the M1 A tile).
+// Token warps: asynchronous copies of a stage's x head slices (into rows t and 64 + t of the
+// x tile; fp32 activations are rounded to bf16) and q head slices (into rows 64.. of the M1 A tile).
 __device__ __forceinline__ void tc_prefetch(TcSmem& sm, const StageInfo& si, const TcArgs& a, int r,
                                             int64_t tok0, int ch0, int ht) {
   for (int idx = ht; idx < si.T * 4; idx += 64) {
@@ -205,6 +225,7 @@ __device__ __forceinline__ void tc_prefetch(TcSmem& sm, const StageInfo& si, con
       const int p = route_pos(r, si.t0 + tt, a.H, a.W);
       const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.x) + (tok0 + p) * a.C + ch0 + part * 8;
       cp_async16(sm.xa + umma_off(tt, part * 8), src);
+      cp_async16(sm.xa + umma_off(64 + tt, part * 8), src);
     }
   } else {
     for (int idx = ht; idx < si.T * 4; idx += 64) {
@@ -219,6 +240,7 @@ __device__ __forceinline__ void tc_prefetch(TcSmem& sm, const StageInfo& si, con
       raw.x = *reinterpret_cast<const uint32_t*>(&b0); raw.y = *reinterpret_cast<const uint32_t*>(&b1);
       raw.z = *reinterpret_cast<const uint32_t*>(&b2); raw.w = *reinterpret_cast<const uint32_t*>(&b3);
       *reinterpret_cast<uint4*>(sm.xa + umma_off(tt, part * 8)) = raw;
+      *reinterpret_cast<uint4*>(sm.xa + umma_off(64 + tt, part * 8)) = raw;
     }
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
@@ -294,6 +316,11 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
   const uint32_t tmem = sm.tmem_base;
   const uint32_t tmem_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   const uint32_t idesc32 = idesc_bf16(32), idesc80 = idesc_bf16(80), idesc96 = idesc_bf16(96);
+  // A chunk within one stage makes every stage open a chunk: Q_b is then Q_s, and W reads
+  // its operand from rows 64..95 of the M1 B tiles.
+  const bool qb_is_qs = L <= kStage;
+  const uint32_t wb_hi = qb_is_qs ? smem_u32(sm.b1h) + 64 * 64 : smem_u32(sm.qbh);
+  const uint32_t wb_lo = qb_is_qs ? smem_u32(sm.b1l) + 64 * 64 : smem_u32(sm.qbl);
 
   // readout warps: the stage whose z / y is still to be produced
   bool pend = false;
@@ -307,17 +334,21 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     const uint32_t hb = (uint32_t)(ne & 1) * 128u;
     const uint32_t par = (uint32_t)(ne & 1);
 
-    // ---- (A) generation (token warps) | z and Y product of the previous stage (readout warps)
-    if (is_k) {
-      const int gt = tid - 128;
-      if (gt == 0) {
-        tc_fence_after();
-        mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), smem_u32(sm.qbh), idesc32, false);
-        mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), smem_u32(sm.qbl), idesc32, true);
-        mma_commit(&sm.mbar_w);
-      }
-      mbar_wait(&sm.mbar_w, par, &sm.wait_failed);
-      {
+    // ---- (A) generation.  Token warps: boundary products, generation, the gate scalars and
+    // the retention prefix.  Readout warps: z and the Y product of the previous stage.  Both
+    // then share every token's key / value columns (the generation tile repeats the tokens in
+    // rows 64..127, so the readout warps find them in their own TMEM lanes).
+    if (is_k || is_r) {
+      const int t = is_k ? tid - 128 : tid - 64;  // token (TMEM lane t, or 64 + t)
+      const int c0 = is_k ? 0 : 16;               // this thread's half of the key and value columns
+      if (is_k) {
+        if (t == 0) {
+          tc_fence_after();
+          mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), wb_hi, idesc32, false);
+          mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), wb_lo, idesc32, true);
+          mma_commit(&sm.mbar_w);
+        }
+        mbar_wait(&sm.mbar_w, par, &sm.wait_failed);
         float wv[kD];
         SRNL_LD16(wv, tmem_lane + hb + kColM1);
         SRNL_LD16(wv + 16, tmem_lane + hb + kColM1 + 16);
@@ -331,80 +362,104 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
           uint4 raw;
           raw.x = *reinterpret_cast<const uint32_t*>(&b0); raw.y = *reinterpret_cast<const uint32_t*>(&b1);
           raw.z = *reinterpret_cast<const uint32_t*>(&b2); raw.w = *reinterpret_cast<const uint32_t*>(&b3);
-          *reinterpret_cast<uint4*>(sm.xa + umma_off(gt, c)) = raw;
+          *reinterpret_cast<uint4*>(sm.xa + umma_off(t, c)) = raw;
+          *reinterpret_cast<uint4*>(sm.xa + umma_off(64 + t, c)) = raw;
+        }
+        fence_async_smem();
+        tc_fence_before();
+        tok_bar();
+        if (t == 0) {
+          tc_fence_after();
+          mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), smem_u32(sm.gb), idesc80, false);
+          mma_commit(&sm.mbar_g);
+        }
+      } else if (pend) {  // z and the Y product of the previous stage
+        mbar_wait(&sm.mbar_z, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
+        float z0[kD], zm[kD];
+        SRNL_LD16(z0, tmem_lane + phb + kColZ0);
+        SRNL_LD16(z0 + 16, tmem_lane + phb + kColZ0 + 16);
+        SRNL_LD16(zm, tmem_lane + phb + kColZ);
+        SRNL_LD16(zm + 16, tmem_lane + phb + kColZ + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < kD; ++i) z0[i] = fmaf(ct_pend, z0[i], zm[i]);
+        store_row_split(sm.yah, sm.yal, t, z0);
+        fence_async_smem();
+        tc_fence_before();
+        named_bar(4, 64);
+        if (t == 0) {
+          tc_fence_after();
+          mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.mh), idesc32, false);
+          mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.ml), idesc32, true);
+          mma_k32(tmem + phb + kColM1, smem_u32(sm.yal), smem_u32(sm.mh), idesc32, true);
+          mma_commit(&sm.mbar_y);
         }
       }
-      fence_async_smem();
-      tc_fence_before();
-      tok_bar();
-      if (gt == 0) {
-        tc_fence_after();
-        mma_k32(tmem + hb + kColM1, smem_u32(sm.xa), smem_u32(sm.gb), idesc80, false);
-        mma_commit(&sm.mbar_g);
-      }
       mbar_wait(&sm.mbar_g, par, &sm.wait_failed);
-      float kt[kD], vv[kD], ga, gbeta;
-      SRNL_LD16(kt, tmem_lane + hb + kColM1);
-      SRNL_LD16(kt + 16, tmem_lane + hb + kColM1 + 16);
-      SRNL_LD16(vv, tmem_lane + hb + kColM1 + 32);
-      SRNL_LD16(vv + 16, tmem_lane + hb + kColM1 + 48);
-      asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
-                   : "=f"(ga), "=f"(gbeta)
-                   : "r"(tmem_lane + hb + kColM1 + 64u));
+      float kt[16], vv[16], ga = 0.f, gbeta = 0.f;
+      SRNL_LD16(kt, tmem_lane + hb + kColM1 + c0);
+      SRNL_LD16(vv, tmem_lane + hb + kColM1 + 32 + c0);
+      if (is_k)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
+                     : "=f"(ga), "=f"(gbeta)
+                     : "r"(tmem_lane + hb + kColM1 + 64u));
       tmem_wait_ld();
-      float l2a = 0.f, et = 0.f;
-      if (gt < T) {
-        float al;
-        gates_row(kt, vv, ga, gbeta, a.alpha, a.eps, al, et);
-        l2a = fmaxf(log2f(al), -126.f);  // a retention that underflows acts as 2^-126
-      } else {
+      float nk0 = 0.f, nk1 = 0.f, kv0 = 0.f, kv1 = 0.f, nv0 = 0.f, nv1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < kD; ++i) { kt[i] = 0.f; vv[i] = 0.f; }
+      for (int i = 0; i < 16; i += 2) {
+        nk0 = fmaf(kt[i], kt[i], nk0); nk1 = fmaf(kt[i + 1], kt[i + 1], nk1);
+        kv0 = fmaf(kt[i], vv[i], kv0); kv1 = fmaf(kt[i + 1], vv[i + 1], kv1);
+        nv0 = fmaf(vv[i], vv[i], nv0); nv1 = fmaf(vv[i + 1], vv[i + 1], nv1);
       }
-      store_row_split(sm.a1h, sm.a1l, gt, vv);  // u_t
-      store_row_split(sm.b1h, sm.b1l, gt, kt);  // k_t
-      sm.eta[gt] = et;
-      // inclusive prefix of log2 alpha over the stage
-      float pre = l2a;
+      if (is_r) sm.gpart[t] = make_float4(nk0 + nk1, kv0 + kv1, nv0 + nv1, 0.f);
+      named_bar(6, 128);  // warps 2-5
+      if (is_k) {
+        const float4 o = sm.gpart[t];
+        const float nk = (nk0 + nk1) + o.x, kv = (kv0 + kv1) + o.y, nv = (nv0 + nv1) + o.z;
+        const bool live = t < T;
+        float l2a = 0.f, et = 0.f, al = 1.f, inv = 0.f;
+        if (live) {
+          inv = rsqrtf(nk + a.eps);
+          // ||k||^2 and ||k - v||^2 of the stabilized key k = inv k~
+          const float kn2 = nk * inv * inv;
+          const float dk2 = fmaxf(fmaf(inv, fmaf(-2.f, kv, inv * nk), nv), 0.f);
+          gate_scalars(kn2, dk2, ga, gbeta, a.alpha, al, et);
+          l2a = fmaxf(log2f(al), -126.f);  // a retention that underflows acts as 2^-126
+        }
+        sm.eta[t] = et;
+        // inclusive prefix of log2 alpha over the stage
+        float pre = l2a;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float v = __shfl_up_sync(0xffffffffu, pre, o);
-        if (lane >= o) pre += v;
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+          const float v = __shfl_up_sync(0xffffffffu, pre, o2);
+          if (lane >= o2) pre += v;
+        }
+        if (t == 31) sm.wsum = pre;
+        tok_bar();
+        if (t >= 32) pre += sm.wsum;
+        sm.lam[t] = pre;
+        tok_bar();
+        const float gk = live ? exp2_fast(sm.lam[T - 1] - pre) * et : 0.f;
+        sm.gpar[t] = make_float4(inv, al, gk, live ? 1.f : 0.f);
       }
-      if (gt == 31) sm.wsum = pre;
-      tok_bar();
-      if (gt >= 32) pre += sm.wsum;
-      sm.lam[gt] = pre;
-      tok_bar();
-      // Kd^T[c][j] = g(j, T-1) eta_j k_j[c]: column j = gt of rows 0..31 of Z A
-      const float gk = (gt < T) ? exp2_fast(sm.lam[T - 1] - pre) * et : 0.f;
-      unsigned char* zh = sm.zah[gt >> 5];
-      unsigned char* zl = sm.zal[gt >> 5];
+      named_bar(7, 128);
+      {
+        const float4 gp = sm.gpar[t];  // (1/||k~||, alpha, g(t, T-1) eta_t, live)
+        const float up = 1.f + gp.y;
 #pragma unroll
-      for (int c = 0; c < kD; ++c) store_split(zh, zl, c, gt & 31, gk * kt[c]);
+        for (int i = 0; i < 16; ++i) {
+          kt[i] *= gp.x;                                  // k_t (zero past the stage)
+          vv[i] = gp.w != 0.f ? up * kt[i] - vv[i] : 0.f;  // u_t
+        }
+        store_half_split(sm.a1h, sm.a1l, t, c0, vv);
+        store_half_split(sm.b1h, sm.b1l, t, c0, kt);
+        // Kd^T[c][j] = g(j, T-1) eta_j k_j[c]: column j = t, rows c0..c0 + 15 of Z A
+        unsigned char* zh = sm.zah[t >> 5];
+        unsigned char* zl = sm.zal[t >> 5];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) store_split(zh, zl, c0 + c, t & 31, gp.z * kt[c]);
+      }
       fence_async_smem();
-    } else if (is_r && pend) {
-      const int t = tid - 64;
-      mbar_wait(&sm.mbar_z, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
-      float z0[kD], zm[kD];
-      SRNL_LD16(z0, tmem_lane + phb + kColZ0);
-      SRNL_LD16(z0 + 16, tmem_lane + phb + kColZ0 + 16);
-      SRNL_LD16(zm, tmem_lane + phb + kColZ);
-      SRNL_LD16(zm + 16, tmem_lane + phb + kColZ + 16);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < kD; ++i) z0[i] = fmaf(ct_pend, z0[i], zm[i]);
-      store_row_split(sm.yah, sm.yal, t, z0);
-      fence_async_smem();
-      tc_fence_before();
-      named_bar(4, 64);
-      if (t == 0) {
-        tc_fence_after();
-        mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.mh), idesc32, false);
-        mma_k32(tmem + phb + kColM1, smem_u32(sm.yah), smem_u32(sm.ml), idesc32, true);
-        mma_k32(tmem + phb + kColM1, smem_u32(sm.yal), smem_u32(sm.mh), idesc32, true);
-        mma_commit(&sm.mbar_y);
-      }
     }
     tc_fence_before();
     __syncthreads();
@@ -418,42 +473,67 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       mma_k32(tmem + hb + kColM1, al, bh, idesc96, true);
       mma_commit(&sm.mbar_1);
     }
-    // ---- (D) solve | readout coefficients | copies of the next stage and y of the previous one
-    if (is_s) {
+    // ---- (D) -A and the right-hand sides (solve and token warps) | readout coefficients
+    // (readout warps) | then the token warps copy the next stage and store y of the previous one
+    if (is_s || is_k) {
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
-      {
-        const int t = tid;  // TMEM lane = token
-        const bool live = t < T;
-        float g[kStage], bv[kD];
-        SRNL_LD16(g, tmem_lane + hb + kColM1);
-        SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + 16);
-        SRNL_LD16(g + 32, tmem_lane + hb + kColM1 + 32);
-        SRNL_LD16(g + 48, tmem_lane + hb + kColM1 + 48);
+      const int t = is_k ? tid - 128 : tid;  // TMEM lane = token
+      const bool live = t < T;
+      const int j0 = is_k ? 32 : 0;          // this thread's columns j of A: [j0, j0 + 32)
+      float g[32], bv[kD];
+      SRNL_LD16(g, tmem_lane + hb + kColM1 + j0);
+      SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + j0 + 16);
+      if (is_k) {
         SRNL_LD16(bv, tmem_lane + hb + kColZ0);
         SRNL_LD16(bv + 16, tmem_lane + hb + kColZ0 + 16);
-        tmem_wait_ld();
-        const float lp = (t > 0 && live) ? sm.lam[t - 1] : 0.f;  // Lambda_{t-1}
+      }
+      tmem_wait_ld();
+      const float lp = (t > 0 && live) ? sm.lam[t - 1] : 0.f;  // Lambda_{t-1}
 #pragma unroll
-        for (int jb = 0; jb < kStage; jb += 16) {
-          // the block's Lambda_j and eta_j first: the stores below may alias them
-          float lv[16], ev[16], v[16];
+      for (int jb = 0; jb < 32; jb += 16) {
+        // the block's Lambda_j and eta_j first: the stores below may alias them
+        float lv[16], ev[16], v[16];
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
-            const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
-            lv[i] = lj.x; lv[i + 1] = lj.y; lv[i + 2] = lj.z; lv[i + 3] = lj.w;
-            ev[i] = ej.x; ev[i + 1] = ej.y; ev[i + 2] = ej.z; ev[i + 3] = ej.w;
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            v[i] = (live && jb + i < t) ? -exp2_fast(lp - lv[i]) * ev[i] * g[jb + i] : 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) neg_a_row(sm, jb + i)[t] = v[i];
+        for (int i = 0; i < 16; i += 4) {
+          const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[j0 + jb + i]);
+          const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[j0 + jb + i]);
+          lv[i] = lj.x; lv[i + 1] = lj.y; lv[i + 2] = lj.z; lv[i + 3] = lj.w;
+          ev[i] = ej.x; ev[i + 1] = ej.y; ev[i + 2] = ej.z; ev[i + 3] = ej.w;
         }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] = (live && j0 + jb + i < t) ? -exp2_fast(lp - lv[i]) * ev[i] * g[jb + i] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) neg_a_row(sm, j0 + jb + i)[t] = v[i];
+      }
+      if (is_k) {
         const float cp = live ? exp2_fast(lp) : 0.f;
 #pragma unroll
         for (int i = 0; i < kD; ++i) rhs_row(sm, i)[t] = cp * bv[i];
       }
+    }
+    if (is_k) {
+      const int gt = tid - 128;
+      named_bar_arrive(5, 128);  // this half of A and the right-hand sides are written
+      if (ne + 1 < nst) tc_prefetch(sm, stage_info(ne + 1, N, L), a, r, tok0, ch0, gt);
+      if (pend) {  // y of the previous stage: the Y product was issued in (A)
+        mbar_wait(&sm.mbar_y, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
+        float y[kD];
+        SRNL_LD16(y, tmem_lane + phb + kColM1);
+        SRNL_LD16(y + 16, tmem_lane + phb + kColM1 + 16);
+        tmem_wait_ld();
+        if (gt < pst.T) {
+          const int p = route_pos(r, pst.t0 + gt, a.H, a.W);
+          float* dst = a.yr + ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0;
+#pragma unroll
+          for (int i = 0; i < kD; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(sm.scale[i] * y[i], sm.scale[i + 1] * y[i + 1], sm.scale[i + 2] * y[i + 2],
+                            sm.scale[i + 3] * y[i + 3]);
+        }
+      }
+      cp_async_wait_all();
+      fence_async_smem();
     } else if (is_r) {
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
       const int t = tid - 64;
@@ -490,53 +570,41 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       }
       fence_async_smem();
       ct_pend = live ? exp2_fast(lt) : 0.f;
-    } else {
-      const int gt = tid - 128;
-      mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
-      if (ne + 1 < nst) tc_prefetch(sm, stage_info(ne + 1, N, L), a, r, tok0, ch0, gt);
-      if (pend) {  // y of the previous stage: the Y product was issued in (A)
-        mbar_wait(&sm.mbar_y, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
-        float y[kD];
-        SRNL_LD16(y, tmem_lane + phb + kColM1);
-        SRNL_LD16(y + 16, tmem_lane + phb + kColM1 + 16);
-        tmem_wait_ld();
-        if (gt < pst.T) {
-          const int p = route_pos(r, pst.t0 + gt, a.H, a.W);
-          float* dst = a.yr + ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0;
-#pragma unroll
-          for (int i = 0; i < kD; i += 4)
-            *reinterpret_cast<float4*>(dst + i) =
-                make_float4(sm.scale[i] * y[i], sm.scale[i + 1] * y[i + 1], sm.scale[i + 2] * y[i + 2],
-                            sm.scale[i + 3] * y[i + 3]);
-        }
-      }
-      cp_async_wait_all();
-      fence_async_smem();
     }
-    // ---- forward substitution (warps 0-3).  Thread: rows rg + 8 m (m = 0..3, rg = 2 warp +
-    // (lane & 1)), tokens [4 kq, 4 kq + 4) (kq = lane >> 1).  Two tokens per broadcast: the
-    // owner lanes of tokens t, t + 1 (kq == t / 4) finish s_{t+1} = b_{t+1} - A[t+1][t] s_t
+    // ---- forward substitution (solve warps).  Thread: rows rg + 8 m (m = 0..3, rg = 4 warp +
+    // (lane & 3)), tokens [8 kb, 8 kb + 8) (kb = lane >> 2).  Two tokens per broadcast: the
+    // owner lanes of tokens t, t + 1 (kb == t / 8) finish s_{t+1} = b_{t+1} - A[t+1][t] s_t
     // from their registers, then every lane subtracts A[t'][t] s_t + A[t'][t+1] s_{t+1}
     // from its tokens t' (A is zero for t' <= t, so finished tokens stay as they are).
-    if (!is_k) {
-      named_bar(5, 128);  // A, the right-hand sides and Mz^T are complete
-      const int rg = 2 * warp + (lane & 1), kq = lane >> 1;
-      float sv[4][4];
+    if (is_s) {
+      named_bar(5, 128);  // A and the right-hand sides (the token warps arrive without waiting)
+      const int rg = 4 * warp + (lane & 3), kb = lane >> 2;
+      float sv[4][8];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const float4 v = *reinterpret_cast<const float4*>(rhs_row(sm, rg + 8 * m) + 4 * kq);
-        sv[m][0] = v.x; sv[m][1] = v.y; sv[m][2] = v.z; sv[m][3] = v.w;
+        const float* src = rhs_row(sm, rg + 8 * m) + 8 * kb;
+        const float4 v0 = *reinterpret_cast<const float4*>(src);
+        const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+        sv[m][0] = v0.x; sv[m][1] = v0.y; sv[m][2] = v0.z; sv[m][3] = v0.w;
+        sv[m][4] = v1.x; sv[m][5] = v1.y; sv[m][6] = v1.z; sv[m][7] = v1.w;
       }
-      const int nb4 = (T + 3) >> 2;
+      const int nblk = (T + 7) >> 3;
 #pragma unroll 1
-      for (int bt = 0; bt < nb4; ++bt) {
-        const int src = (bt << 1) | (lane & 1);
-        const float* abase = neg_a_row(sm, 4 * bt) + 4 * kq;
+      for (int bt = 0; bt < nblk; ++bt) {
+        const int src = (bt << 2) | (lane & 3);
+        const float* abase = neg_a_row(sm, 8 * bt) + 8 * kb;
 #pragma unroll
-        for (int tl = 0; tl < 4; tl += 2) {
-          const float4 p0 = *reinterpret_cast<const float4*>(abase + tl * kStage);
-          const float4 p1 = *reinterpret_cast<const float4*>(abase + (tl + 1) * kStage);
-          const float a0[4] = {p0.x, p0.y, p0.z, p0.w}, a1[4] = {p1.x, p1.y, p1.z, p1.w};
+        for (int tl = 0; tl < 8; tl += 2) {
+          float a0[8], a1[8];
+          {
+            const float* ar = abase + tl * kStage;
+            const float4 p0 = *reinterpret_cast<const float4*>(ar);
+            const float4 p1 = *reinterpret_cast<const float4*>(ar + 4);
+            const float4 p2 = *reinterpret_cast<const float4*>(ar + kStage);
+            const float4 p3 = *reinterpret_cast<const float4*>(ar + kStage + 4);
+            a0[0] = p0.x; a0[1] = p0.y; a0[2] = p0.z; a0[3] = p0.w; a0[4] = p1.x; a0[5] = p1.y; a0[6] = p1.z; a0[7] = p1.w;
+            a1[0] = p2.x; a1[1] = p2.y; a1[2] = p2.z; a1[3] = p2.w; a1[4] = p3.x; a1[5] = p3.y; a1[6] = p3.z; a1[7] = p3.w;
+          }
           float xs[4], ys[4];
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
@@ -547,8 +615,8 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
           }
           // the pair of tokens t + 2, t + 3 first: it feeds the next broadcast
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int i = ((tl + 2) & 3) ^ (2 * q);
+          for (int q = 0; q < 4; ++q) {
+            const int i = ((tl + 2) & 7) ^ (2 * q);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
               const float2 r2 = __ffma2_rn(f2(a1[i], a1[i + 1]), f2(ys[m], ys[m]),
@@ -559,23 +627,20 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
           }
         }
       }
-      // -S into the Z B operand (row r, K = token): half a core-matrix row per (row, hi/lo)
+      // -S into the Z B operand (row r, K = token): one core-matrix row per (row, hi/lo)
       {
-        unsigned char* th = sm.zbh[kq >> 3];
-        unsigned char* tl = sm.zbl[kq >> 3];
-        const int k0 = (4 * kq) & 31;
+        unsigned char* th = sm.zbh[kb >> 2];
+        unsigned char* tl = sm.zbl[kb >> 2];
+        const int k0 = 8 * (kb & 3);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const __nv_bfloat162 h0 = __floats2bfloat162_rn(-sv[m][0], -sv[m][1]);
-          const __nv_bfloat162 h1 = __floats2bfloat162_rn(-sv[m][2], -sv[m][3]);
-          const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
-          const __nv_bfloat162 l0 = __floats2bfloat162_rn(-sv[m][0] - f0.x, -sv[m][1] - f0.y);
-          const __nv_bfloat162 l1 = __floats2bfloat162_rn(-sv[m][2] - f1.x, -sv[m][3] - f1.y);
-          uint2 hv, lv;
-          hv.x = *reinterpret_cast<const uint32_t*>(&h0); hv.y = *reinterpret_cast<const uint32_t*>(&h1);
-          lv.x = *reinterpret_cast<const uint32_t*>(&l0); lv.y = *reinterpret_cast<const uint32_t*>(&l1);
-          *reinterpret_cast<uint2*>(th + umma_off(rg + 8 * m, k0)) = hv;
-          *reinterpret_cast<uint2*>(tl + umma_off(rg + 8 * m, k0)) = lv;
+          float v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = -sv[m][i];
+          uint4 hi, lo;
+          split8(v, hi, lo);
+          *reinterpret_cast<uint4*>(th + umma_off(rg + 8 * m, k0)) = hi;
+          *reinterpret_cast<uint4*>(tl + umma_off(rg + 8 * m, k0)) = lo;
         }
       }
       fence_async_smem();
@@ -614,7 +679,8 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
 #pragma unroll
       for (int c = 0; c < kD; ++c) row[c] = sm.qsT[c][lane];
       store_row_split(sm.b1h, sm.b1l, 64 + lane, row);
-      if (ne + 1 < nst && stage_info(ne + 1, N, L).chunk_start) store_row_split(sm.qbh, sm.qbl, lane, row);
+      if (!qb_is_qs && ne + 1 < nst && stage_info(ne + 1, N, L).chunk_start)
+        store_row_split(sm.qbh, sm.qbl, lane, row);
       fence_async_smem();
     }
     pend = true;

@@ -139,9 +139,23 @@ __device__ __forceinline__ float quad_sum(float v) {
   return v;
 }
 
+// Gate scalars of one token from ||k||^2 (stabilized key), ||k - v||^2, a and beta:
+// retention clamp, softplus step, soft injection cap, spectral clamp.
+__device__ __forceinline__ void gate_scalars(float kn2, float dk2, float a, float beta, float alpha_max,
+                                             float& al, float& eta) {
+  const float gain = sqrtf(dk2 * kn2);
+  const float eb = __expf(-fabsf(beta));  // sigmoid without overflow
+  const float sg = (beta >= 0.f) ? __fdividef(1.f, 1.f + eb) : __fdividef(eb, 1.f + eb);
+  al = fminf(sg, alpha_max);
+  const float eta0 = fmaxf(a, 0.f) + log1pf(__expf(-fabsf(a)));
+  const float zc = __fdividef(eta0 * gain, 1.f - al);
+  const float phi = (zc < 1e-4f) ? (1.f - zc * zc * (1.f / 3.f)) : __fdividef(tanhf(zc), zc);
+  eta = eta0 * phi;
+  if (eta * kn2 > 2.f) eta = __fdividef(2.f, kn2);
+}
+
 // Gates of one token from its generated row (k~[32], v[32], a, beta): kt becomes the
-// stabilized key and vv becomes u.  Stabilized key, retention clamp, softplus step,
-// soft injection cap, spectral clamp.
+// stabilized key and vv becomes u.
 __device__ __forceinline__ void gates_row(float (&kt)[kD], float (&vv)[kD], float a, float beta,
                                           float alpha_max, float eps, float& al, float& eta) {
   float n0 = 0.f, n1 = 0.f, n2 = 0.f, n3 = 0.f;
@@ -165,16 +179,7 @@ __device__ __forceinline__ void gates_row(float (&kt)[kD], float (&vv)[kD], floa
     d0 = fmaf(da, da, d0);
     d1 = fmaf(db, db, d1);
   }
-  const float kn2 = k0 + k1;
-  const float gain = sqrtf((d0 + d1) * kn2);
-  const float eb = __expf(-fabsf(beta));  // sigmoid without overflow
-  const float sg = (beta >= 0.f) ? __fdividef(1.f, 1.f + eb) : __fdividef(eb, 1.f + eb);
-  al = fminf(sg, alpha_max);
-  const float eta0 = fmaxf(a, 0.f) + log1pf(__expf(-fabsf(a)));
-  const float zc = __fdividef(eta0 * gain, 1.f - al);
-  const float phi = (zc < 1e-4f) ? (1.f - zc * zc * (1.f / 3.f)) : __fdividef(tanhf(zc), zc);
-  eta = eta0 * phi;
-  if (eta * kn2 > 2.f) eta = __fdividef(2.f, kn2);
+  gate_scalars(k0 + k1, d0 + d1, a, beta, alpha_max, al, eta);
 #pragma unroll
   for (int i = 0; i < kD; ++i) vv[i] = (1.f + al) * kt[i] - vv[i];
 }
