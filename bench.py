@@ -295,7 +295,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                      "kernel": "srnl_scan_chunkwise_kernel" if gen == "bf16" else "srnl_scan_sequential_kernel",
                      "kernel_ms": scan_ms,
                      "peak_note": "fp32 FMA peak 148 SM x 128 lanes x 2 x sm_max_mhz (derived)"},
-        "north_star_roofline": {"bound": "hbm" if t_bytes_us >= t_tensor_us else "tensor",
+        "forward_roofline": {"bound": "hbm" if t_bytes_us >= t_tensor_us else "tensor",
                                 "roofline_us": roof_us, "forward_us": ms_step * 1e3,
                                 "frac": roof_us / (ms_step * 1e3),
                                 "hbm_bytes": wm["hbm_bytes"], "tensor_flops": wm["gen_flops"] + wm["qproj_flops"],
