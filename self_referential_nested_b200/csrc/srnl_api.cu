@@ -21,6 +21,7 @@ struct srnl_scan {
   int device = 0;
   // packed parameters (device)
   float* Wq = nullptr;
+  void* Wqb = nullptr;       // W_q in bf16 (bf16 path only)
   float* G = nullptr;
   float* Mm = nullptr;
   float* scales = nullptr;
@@ -63,10 +64,11 @@ size_t act_bytes(const srnl_scan_config& c) {
 }
 
 void free_all(srnl_scan* h) {
-  void* ptrs[] = {h->Wq, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err};
+  void* ptrs[] = {h->Wq, h->Wqb, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->Wq = h->G = h->Mm = h->scales = nullptr;
+  h->Wqb = nullptr;
   h->q = h->x_stage = h->y_stage = nullptr;
   h->yr = nullptr;
   h->dev_err = nullptr;
@@ -154,6 +156,8 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
   // ---- pack parameters on the host, then upload
   std::vector<float> Wq((size_t)c.C * c.C);
   for (size_t i = 0; i < Wq.size(); ++i) Wq[i] = g.gen_bf16 ? bf16_round_host(prm->W_q[i]) : prm->W_q[i];
+  std::vector<__nv_bfloat16> Wqb(g.gen_bf16 ? Wq.size() : 0);
+  for (size_t i = 0; i < Wqb.size(); ++i) Wqb[i] = __float2bfloat16_rn(Wq[i]);  // exact: already rounded
   std::vector<float> G((size_t)4 * nh * srnl::kGen * d);
   for (int r = 0; r < 4; ++r)
     for (int hh = 0; hh < nh; ++hh) {
@@ -175,8 +179,9 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
       {(void**)&h->Mm, n_mm * sizeof(float)},      {(void**)&h->scales, n_sc * sizeof(float)},
       {&h->q, q_bytes},                            {(void**)&h->yr, yr_bytes},
       {&h->x_stage, stage_bytes},                  {&h->y_stage, stage_bytes},
-      {(void**)&h->dev_err, sizeof(int)}};
+      {(void**)&h->dev_err, sizeof(int)},          {&h->Wqb, Wqb.size() * sizeof(__nv_bfloat16)}};
   for (auto& a : allocs) {
+    if (a.n == 0) continue;
     e = cudaMalloc(a.p, a.n);
     if (e != cudaSuccess) {
       st = cuda_fail(nullptr, e, "cudaMalloc");
@@ -186,8 +191,10 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
   h->ws_bytes = q_bytes + yr_bytes + 2 * stage_bytes;
   struct { void* dst; const void* src; size_t n; } copies[] = {
       {h->Wq, Wq.data(), Wq.size() * sizeof(float)}, {h->G, G.data(), G.size() * sizeof(float)},
-      {h->Mm, prm->M_mem0, n_mm * sizeof(float)},    {h->scales, prm->scales, n_sc * sizeof(float)}};
+      {h->Mm, prm->M_mem0, n_mm * sizeof(float)},    {h->scales, prm->scales, n_sc * sizeof(float)},
+      {h->Wqb, Wqb.data(), Wqb.size() * sizeof(__nv_bfloat16)}};
   for (auto& cp : copies) {
+    if (cp.n == 0) continue;
     e = cudaMemcpy(cp.dst, cp.src, cp.n, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemcpy (params)"); free_all(h); delete h; return st; }
   }
@@ -200,11 +207,11 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
 }
 
 static srnl_status run_forward(srnl_scan* h, const void* x, void* y, float* finals, cudaStream_t s) {
-  srnl::ScanParamsDev p{h->Wq, h->G, h->Mm, h->scales};
+  srnl::ScanParamsDev p{h->Wq, h->Wqb, h->G, h->Mm, h->scales};
   cudaError_t e;
   cudaEvent_t* ev = h->ring > 0 ? &h->ev[(size_t)(h->recorded % h->ring) * 4] : nullptr;
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
-  e = srnl::launch_query_projection(h->geom, p, x, h->q, s);
+  e = srnl::launch_query_projection(h->geom, p, x, h->q, h->dev_err, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, finals, h->dev_err, s);

@@ -144,10 +144,15 @@ __global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-cudaError_t prepare_kernels() { return prepare_scan_kernels(); }
+cudaError_t prepare_kernels() {
+  const cudaError_t e = prepare_scan_kernels();
+  if (e != cudaSuccess) return e;
+  return prepare_projection_kernel();
+}
 
 cudaError_t launch_query_projection(const ScanGeom& g, const ScanParamsDev& p, const void* x,
-                                    void* q, cudaStream_t s) {
+                                    void* q, int* err, cudaStream_t s) {
+  if (p.Wqb != nullptr && query_projection_tc_supported(g)) return launch_query_projection_tc(g, p, x, q, err, s);
   const int64_t M = (int64_t)g.B * g.H * g.W;
   dim3 grid((unsigned)((M + kQpBM - 1) / kQpBM), (unsigned)((g.C + kQpBO - 1) / kQpBO));
   query_projection_kernel<<<grid, kQpThreads, 0, s>>>(x, p.Wq, q, M, g.C, g.act_bf16, g.gen_bf16);

@@ -16,14 +16,20 @@ struct ScanGeom {
 
 struct ScanParamsDev {
   const float* Wq;      // [C][C] (bf16-rounded values when gen_bf16)
+  const void* Wqb;      // [C][C] W_q as bf16 (bf16 path), else nullptr
   const float* G;       // [4][heads][kGen][kD]  generating initials per route/head
   const float* Mm;      // [4][heads][kD][kD]    content-memory initials
   const float* scales;  // [4][C]
 };
 
-// q[B*N][C] = x W_q^T ; q is fp32 or bf16 (gen_bf16).
+// q[B*N][C] = x W_q^T ; q is fp32 or bf16 (gen_bf16).  bf16 activations with a bf16 W_q
+// run on the tensor cores; `err` (device int) receives SRNL_E_TIMEOUT if a bounded wait
+// gives up.
 cudaError_t launch_query_projection(const ScanGeom& g, const ScanParamsDev& p, const void* x,
-                                    void* q, cudaStream_t s);
+                                    void* q, int* err, cudaStream_t s);
+bool query_projection_tc_supported(const ScanGeom& g);
+cudaError_t launch_query_projection_tc(const ScanGeom& g, const ScanParamsDev& p, const void* x, void* q,
+                                       int* err, cudaStream_t s);
 
 // Route partials yr[4][B*N][C] (fp32, already scaled by the fusion scales),
 // optional final states.
@@ -44,5 +50,6 @@ cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, con
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)
 cudaError_t prepare_scan_kernels();
 cudaError_t prepare_scan_chunkwise_kernel();
+cudaError_t prepare_projection_kernel();
 
 }  // namespace srnl

@@ -66,9 +66,10 @@ srnl_status scratch_address(void** out) {
 
 size_t round_up(size_t n) { return (n + 255) & ~size_t(255); }
 
-// W_q copy (bf16-rounded on the bf16 path) and G = [M_k0; M_v0; m_eta0; m_alpha0]
-// per (route, head), the layouts the scan kernels read.
+// W_q copy (bf16-rounded on the bf16 path, plus a bf16 copy for the tensor-core projection)
+// and G = [M_k0; M_v0; m_eta0; m_alpha0] per (route, head), the layouts the kernels read.
 __global__ void noalloc_pack_kernel(const float* __restrict__ Wq_src, float* __restrict__ Wq_dst,
+                                    __nv_bfloat16* __restrict__ Wqb_dst,
                                     int64_t n_wq, bool round_bf16_wq, const float* __restrict__ Mk,
                                     const float* __restrict__ Mv, const float* __restrict__ me,
                                     const float* __restrict__ ma, float* __restrict__ G,
@@ -77,6 +78,7 @@ __global__ void noalloc_pack_kernel(const float* __restrict__ Wq_src, float* __r
   if (i < n_wq) {
     const float w = Wq_src[i];
     Wq_dst[i] = round_bf16_wq ? srnl::round_bf16(w) : w;
+    if (Wqb_dst != nullptr) Wqb_dst[i] = __float2bfloat16_rn(w);
   }
   if (i < n_g) {
     constexpr int per = srnl::kGen * srnl::kD;
@@ -131,10 +133,11 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   const size_t n_wq = (size_t)cfg->C * cfg->C;
   const size_t n_g = (size_t)4 * cfg->heads * srnl::kGen * srnl::kD;
   const size_t wq_b = round_up(n_wq * 4), g_b = round_up(n_g * 4);
+  const size_t wqb_b = gen_bf16 ? round_up(n_wq * 2) : 0;
   const size_t q_b = round_up(tokens * cfg->C * (gen_bf16 ? 2 : 4));
   const size_t yr_b = round_up(4 * tokens * cfg->C * sizeof(float));
   const size_t err_b = 256;  // device status word of the scan kernel
-  const size_t need = err_b + wq_b + g_b + q_b + yr_b;
+  const size_t need = err_b + wq_b + wqb_b + g_b + q_b + yr_b;
   if (need > kNoallocScratchBytes) {
     srnl::set_thread_error("workload needs " + std::to_string(need) +
                            " bytes of scratch; the no-allocation forward holds " +
@@ -148,14 +151,16 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   int* dev_err = reinterpret_cast<int*>(s8);
   s8 += err_b;
   float* Wq = reinterpret_cast<float*>(s8);
-  float* G = reinterpret_cast<float*>(s8 + wq_b);
-  void* q = s8 + wq_b + g_b;
-  float* yr = reinterpret_cast<float*>(s8 + wq_b + g_b + q_b);
+  __nv_bfloat16* Wqb = gen_bf16 ? reinterpret_cast<__nv_bfloat16*>(s8 + wq_b) : nullptr;
+  s8 += wq_b + wqb_b;
+  float* G = reinterpret_cast<float*>(s8);
+  void* q = s8 + g_b;
+  float* yr = reinterpret_cast<float*>(s8 + g_b + q_b);
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const size_t n_pack = n_wq > n_g ? n_wq : n_g;
   noalloc_pack_kernel<<<(unsigned)((n_pack + 255) / 256), 256, 0, cs>>>(
-      p->W_q, Wq, (int64_t)n_wq, gen_bf16, p->M_k0, p->M_v0, p->m_eta0, p->m_alpha0, G, (int64_t)n_g);
+      p->W_q, Wq, Wqb, (int64_t)n_wq, gen_bf16, p->M_k0, p->M_v0, p->m_eta0, p->m_alpha0, G, (int64_t)n_g);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) e = srnl::prepare_kernels();
 
@@ -165,8 +170,8 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   g.Lcol = cfg->chunk_col > 0 ? cfg->chunk_col : cfg->H;
   g.alpha = cfg->alpha; g.eps = cfg->eps;
   g.act_bf16 = act_bf16; g.gen_bf16 = gen_bf16;
-  const srnl::ScanParamsDev dp{Wq, G, p->M_mem0, p->scales};
-  if (e == cudaSuccess) e = srnl::launch_query_projection(g, dp, x, q, cs);
+  const srnl::ScanParamsDev dp{Wq, Wqb, G, p->M_mem0, p->scales};
+  if (e == cudaSuccess) e = srnl::launch_query_projection(g, dp, x, q, dev_err, cs);
   if (e == cudaSuccess) e = srnl::launch_scan(g, dp, x, q, yr, nullptr, dev_err, cs);
   if (e == cudaSuccess) e = srnl::launch_fuse(g, yr, y, cs);
   if (e != cudaSuccess) {
