@@ -184,6 +184,36 @@ def run_reference(args, cfg, rank, world):
 
 
 # ----------------------------------------------------------------- GPU arm
+def stages_per_sequence(cfg, stage=64):
+    """Dependent stages of the longest route: chunks x ceil(chunk / stage)."""
+    n = 0
+    N = cfg.H * cfg.W
+    for L in (cfg.chunk_row or cfg.W, cfg.chunk_col or cfg.H):
+        chunks = -(-N // L)
+        last = N - (chunks - 1) * L
+        n = max(n, (chunks - 1) * (-(-L // stage)) + -(-last // stage))
+    return n
+
+
+def chain_latency_ms(S, cfgd, params, x, stream, steps=5):
+    """Scan time of one image.  Its 4 x heads sequences each get an SM of their own, so the
+    time is one sequence's chain of dependent stages with nothing else on the GPU: the bound
+    that batching cannot go below."""
+    import torch
+    h1 = S.srnl_scan_create(dict(cfgd, B=1), params)
+    x1 = x[:1].contiguous()
+    y1 = torch.empty_like(x1)
+    for _ in range(3):
+        S.srnl_scan_forward(h1, x1, y1, None, stream)
+    S.srnl_scan_enable_stage_timing(h1, steps)
+    for _ in range(steps):
+        S.srnl_scan_forward(h1, x1, y1, None, stream)
+    torch.cuda.synchronize()
+    stage, n = S.srnl_scan_stage_times(h1)
+    h1.close()
+    return float(stage[1])
+
+
 def run_ours(args, cfg, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -263,6 +293,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     h.close()
     if rank != 0:
         return
+    chain_ms = chain_latency_ms(S, cfgd, inp.params(), x, stream)
+    n_stages = stages_per_sequence(cfg)
 
     wm = work_model(cfg)
     peaks = load_peaks()
@@ -301,6 +333,10 @@ def run_ours(args, cfg, rank, world, local_rank):
                                 "hbm_bytes": wm["hbm_bytes"], "tensor_flops": wm["gen_flops"] + wm["qproj_flops"],
                                 "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TF/s bf16"},
         "stage_ms": {"query_projection": float(stage_ms[0]), "scan": scan_ms, "fusion": float(stage_ms[2])},
+        "chain": {"stages_per_sequence": n_stages, "one_image_scan_us": chain_ms * 1e3,
+                  "per_stage_us": chain_ms * 1e3 / n_stages, "scan_us": scan_ms * 1e3,
+                  "frac": chain_ms / scan_ms,
+                  "note": "scan of one image (each sequence alone on an SM) over the full scan"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * elt),
                 "d2h_bytes_per_step": int(y.numel() * elt), "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": 3 * args.steps,

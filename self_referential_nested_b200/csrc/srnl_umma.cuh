@@ -37,18 +37,22 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kUmmaM >> 4) << 24);
 }
 
-// D[tmem] (+)= A B^T over K = 32 (two K = 16 steps).
+// D[tmem] (+)= A B^T over one K = 16 step.
+__device__ __forceinline__ void mma_k16(uint32_t tmem, uint32_t a_smem, uint32_t b_smem, uint32_t idesc,
+                                        bool accumulate) {
+  const uint64_t ad = umma_desc(a_smem), bd = umma_desc(b_smem);
+  const uint32_t acc = accumulate ? 1u : 0u;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
+}
+
+// D[tmem] (+)= A B^T over K = 32 (two K = 16 steps; the second core-matrix pair is 256 B on).
 __device__ __forceinline__ void mma_k32(uint32_t tmem, uint32_t a_smem, uint32_t b_smem, uint32_t idesc,
                                         bool accumulate) {
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-    const uint64_t ad = umma_desc(a_smem + ks * 256), bd = umma_desc(b_smem + ks * 256);
-    const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-        "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
-  }
+  mma_k16(tmem, a_smem, b_smem, idesc, accumulate);
+  mma_k16(tmem, a_smem + 256, b_smem + 256, idesc, true);
 }
 
 __device__ __forceinline__ void mma_commit(unsigned long long* bar) {
