@@ -33,7 +33,10 @@ tests/test_oracle_pins.py:
   * chunk length 1 equals an independently written token-wise loop; one chunk
     spanning the sequence generates every token from the initial states;
   * five-memory form equals the single-product form to 1e-12;
-  * one-hot fusion scales isolate routes; batch permutation equivariance.
+  * one-hot fusion scales isolate routes; batch permutation equivariance;
+  * standalone sequence layer: chunk 1 equals the token-wise loop, outputs are causal
+    (a prefix of the input gives the prefix of the output), absent queries mean x, and
+    it equals route 0 of the operator with W_q = I and a one-hot route-0 scale.
 The end-to-end numbers are *not* pinned by printed values (the pages print
 none); they are pinned only through the properties above.
 """
@@ -417,6 +420,42 @@ def operator_forward(x, params, *, alpha_max, eps=1e-6, chunk_row=0, chunk_col=0
                                fin["m_alpha"].reshape(B * heads, -1)], axis=1)
         finals[r] = flat.reshape(B, heads, -1)
     return out, finals, (traces if trace else None)
+
+
+def sequence_forward(x, params, *, alpha_max, eps=1e-6, chunk=64, heads, queries=None, scan="five"):
+    """Standalone SRNL layer on sequences ([README] "SRNL and VisionHOPE operator": a layer
+    on [batch, tokens, dim] that returns the same shape, one pass in token order, 64-token
+    chunks unless told otherwise, an incomplete final chunk allowed; queries of the same shape
+    may be supplied, otherwise x itself is the query; every call starts a new sequence).
+
+    x, queries: [B, T, D].  params: M_mem0/M_k0/M_v0 [heads, d, d], m_eta0/m_alpha0
+    [heads, d] (one set of initial states: a sequence has no routes).  Head h reads its own
+    d-slice of x and of the queries (reading: no input or output projection).  chunk <= 0
+    means 64.  Returns y [B, T, D] and finals [B, heads, 3 d^2 + 2 d].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, T, D = x.shape
+    d = D // heads
+    q = x if queries is None else np.asarray(queries, dtype=np.float64)
+    L = chunk if chunk > 0 else 64
+    xs = x.reshape(B, T, heads, d).transpose(0, 2, 1, 3).reshape(B * heads, T, d)
+    qs = q.reshape(B, T, heads, d).transpose(0, 2, 1, 3).reshape(B * heads, T, d)
+    inits = {}
+    for key, name in (("M_mem0", "M_mem"), ("M_k0", "M_k"), ("M_v0", "M_v"),
+                      ("m_eta0", "m_eta"), ("m_alpha0", "m_alpha")):
+        arr = np.asarray(params[key], dtype=np.float64)  # [heads, ...]
+        inits[name] = np.broadcast_to(arr[None], (B,) + arr.shape).reshape((-1,) + arr.shape[1:]).copy()
+    if scan == "five":
+        y, fin, _ = scan_five_memory(xs, qs, inits, L, alpha_max, eps)
+    elif scan == "tokenwise":
+        y, fin = scan_tokenwise(xs, qs, inits, alpha_max, eps)
+    else:
+        raise ValueError(scan)
+    y = y.reshape(B, heads, T, d).transpose(0, 2, 1, 3).reshape(B, T, D)
+    finals = np.concatenate([fin["M_mem"].reshape(B * heads, -1), fin["M_k"].reshape(B * heads, -1),
+                             fin["M_v"].reshape(B * heads, -1), fin["m_eta"].reshape(B * heads, -1),
+                             fin["m_alpha"].reshape(B * heads, -1)], axis=1).reshape(B, heads, -1)
+    return y, finals
 
 
 def forward_from_inputs(inp, **kw):

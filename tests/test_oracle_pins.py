@@ -371,3 +371,52 @@ def test_pr1_config_qform_and_tokenwise_consistency():
     o3, _, _ = O.forward_from_inputs(inp1)
     o4, _, _ = O.forward_from_inputs(inp1, scan="tokenwise")
     assert O.rel_fro(o4, o3) < 1e-12
+
+
+# ------------------------------------------------ standalone sequence layer
+def _seq_params(heads, d, rng, mem_scale=0.3, vec_scale=1.0):
+    return dict(M_mem0=rng.normal(0, mem_scale, (heads, d, d)), M_k0=rng.normal(0, mem_scale, (heads, d, d)),
+                M_v0=rng.normal(0, mem_scale, (heads, d, d)), m_eta0=rng.normal(0, vec_scale, (heads, d)),
+                m_alpha0=rng.normal(0, vec_scale, (heads, d)))
+
+
+def test_sequence_chunk1_equals_tokenwise():
+    rng = np.random.default_rng(11)
+    x = rng.normal(size=(2, 13, 8))
+    p = _seq_params(2, 4, rng)
+    y1, f1 = O.sequence_forward(x, p, alpha_max=0.9, chunk=1, heads=2)
+    y2, f2 = O.sequence_forward(x, p, alpha_max=0.9, chunk=1, heads=2, scan="tokenwise")
+    assert np.allclose(y1, y2, rtol=1e-12, atol=1e-14) and np.allclose(f1, f2, rtol=1e-12, atol=1e-14)
+
+
+def test_sequence_causal_prefix_and_default_queries():
+    # README: an incomplete final chunk is allowed (257 tokens, chunks of 64); the output at
+    # token t depends on tokens <= t only, so a prefix of the input gives a prefix of the output
+    rng = np.random.default_rng(12)
+    x = rng.normal(size=(1, 257, 8))
+    q = rng.normal(size=(1, 257, 8))
+    p = _seq_params(2, 4, rng)
+    y, _ = O.sequence_forward(x, p, alpha_max=0.95, heads=2, queries=q)
+    yp, _ = O.sequence_forward(x[:, :200], p, alpha_max=0.95, heads=2, queries=q[:, :200])
+    assert np.array_equal(y[:, :200], yp)
+    ya, _ = O.sequence_forward(x, p, alpha_max=0.95, heads=2)
+    yb, _ = O.sequence_forward(x, p, alpha_max=0.95, heads=2, queries=x)
+    assert np.array_equal(ya, yb)
+    assert not np.allclose(y, ya)
+
+
+def test_sequence_equals_operator_route0():
+    rng = np.random.default_rng(13)
+    B, T, heads, d = 2, 21, 2, 4
+    D = heads * d
+    x = rng.normal(size=(B, T, D))
+    p = _seq_params(heads, d, rng)
+    ys, fs = O.sequence_forward(x, p, alpha_max=0.9, chunk=5, heads=heads)
+    op = {k: np.repeat(np.asarray(v)[None], 4, axis=0) for k, v in p.items()}
+    op["W_q"] = np.eye(D)
+    op["scales"] = np.zeros((4, D))
+    op["scales"][0] = 1.0
+    out, fin, _ = O.operator_forward(x.reshape(B, 1, T, D), op, alpha_max=0.9, chunk_row=5, chunk_col=5,
+                                     heads=heads)
+    assert np.allclose(out.reshape(B, T, D), ys, rtol=1e-12, atol=1e-14)
+    assert np.allclose(fin[0], fs, rtol=1e-12, atol=1e-14)
