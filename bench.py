@@ -348,6 +348,52 @@ def run_ours(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_seq(args):
+    """Standalone SRNL layer on sequences ([B, T, D], 64-token chunks, x as the query):
+    B sequences x heads of T tokens, one direction.  One GPU; prints one JSON line."""
+    import torch
+    import self_referential_nested_b200 as S
+    from self_referential_nested_b200 import build as Bld
+    from srnl_inputs import make_seq_inputs
+
+    Bld.build()
+    B, T, D, heads = args.seq_batch, args.seq_tokens, 64, 2
+    inp = make_seq_inputs(B, T, D, heads, "bf16", seed=0)
+    cfg = dict(B=B, T=T, D=D, heads=heads, d=32, alpha=0.95, eps=1e-6, chunk=64, act_dtype="bf16",
+               gen_dtype="bf16")
+    h = S.srnl_seq_create(cfg, inp.params())
+    x = torch.from_numpy(inp.x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        S.srnl_seq_forward(h, x, y, stream=stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    ts = []
+    for i in range(args.steps):
+        flush.fill_((i + 1) & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        S.srnl_seq_forward(h, x, y, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    clocks.stop()
+    S.srnl_seq_device_status(h)
+    h.close()
+    ms = float(np.mean(ts))
+    print(json.dumps({"metric": "SRNL sequence layer tokens/s (fwd, 1xB200)", "value": B * T / (ms * 1e-3),
+                      "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": f"seq_b{B}_t{T}_d{D}", "B": B, "T": T, "D": D, "heads": heads,
+                                 "d": 32, "chunk": 64, "queries": "x", "l2": "flushed before each step"},
+                      "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -358,7 +404,13 @@ def main():
     ap.add_argument("--gen", default=None, choices=[None, "f32", "bf16"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
+    ap.add_argument("--seq", action="store_true", help="time the standalone sequence layer instead")
+    ap.add_argument("--seq-batch", type=int, default=128)
+    ap.add_argument("--seq-tokens", type=int, default=3136)
     args = ap.parse_args()
+    if args.seq:
+        run_seq(args)
+        return
     cfg = CONFIGS[args.config]
     if args.batch > 0:
         cfg = cfg.replace(B=args.batch)

@@ -45,7 +45,10 @@
  * boundary are G Q_b (G their initial states, Q_b the product of the
  * transitions so far), and each token's k~, v, a, beta = G (Q_b x); G and
  * Q_b x are rounded to bfloat16.  It also rounds the query-projection operands
- * (x, W_q) and the stored q to bfloat16.
+ * (x, W_q) and the stored q to bfloat16, and runs the token-order write in its
+ * chunkwise form: within a chunk every row of the state solves one shared
+ * triangular system (fp32), and the products around it run on the tensor cores
+ * with each fp32 operand split into bf16 high + low parts (about fp32 accuracy).
  *
  * Errors.  Every entry point returns an srnl_status and never aborts.  On
  * failure the outputs are unspecified and srnl_scan_last_error() describes
@@ -201,6 +204,66 @@ SRNL_API const char* srnl_status_string(int status);
 /* Free the handle and all its device memory.  Accepts NULL.  Synchronises the
  * device before freeing. */
 SRNL_API void srnl_scan_destroy(srnl_scan* h);
+
+/* ------------------------------------------------------------------------
+ * Standalone SRNL layer on sequences ("VisionHOPE" README, section "SRNL and
+ * VisionHOPE operator": a layer on [batch, tokens, dim] returning the same
+ * shape; queries of the same shape may be passed, otherwise x is the query;
+ * 64-token chunks unless a positive length is given; an incomplete final chunk
+ * is allowed; every call starts a new sequence).
+ *
+ * One pass in token order (no routes, no fusion).  Per (batch, head) the five
+ * memories start from the layer's initial states and follow the recurrence
+ * above with x_t and q_t the head's d-slices of x and of the queries;
+ * y[b][t][h*d + i] = (M_mem q_t)[i] after token t's write.  There is no input
+ * or output projection.  Precision paths as above (gen_dtype = SRNL_BF16:
+ * bf16 queries and generation, chunkwise write; SRNL_F32: fp32 throughout).
+ * ---------------------------------------------------------------------- */
+typedef struct srnl_seq srnl_seq; /* opaque; owned by the library */
+
+typedef struct {
+  int B, T, D;    /* batch, tokens, dim (D = heads * d) */
+  int heads, d;   /* heads and head dim; d = 32 is built */
+  float alpha;    /* retention cap, 0 < alpha < 1 */
+  float eps;      /* key normalisation epsilon, > 0 */
+  int chunk;      /* chunk length; 0 means 64 */
+  int act_dtype;  /* srnl_dtype of x, the queries and y */
+  int gen_dtype;  /* srnl_dtype of generation / query operands */
+} srnl_seq_config;
+
+/* Initial states, HOST pointers to dense fp32 arrays, copied by create. */
+typedef struct {
+  const float* M_mem0;   /* [heads][d][d] */
+  const float* M_k0;     /* [heads][d][d] */
+  const float* M_v0;     /* [heads][d][d] */
+  const float* m_eta0;   /* [heads][d]    */
+  const float* m_alpha0; /* [heads][d]    */
+} srnl_seq_params;
+
+/* Validate, allocate the handle and its workspace on the CURRENT device.
+ * *out is NULL on failure; the message is srnl_seq_last_error(NULL). */
+SRNL_API srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg,
+                                     const srnl_seq_params* params);
+
+/* Forward pass.  x, q, y: DEVICE pointers, 16-byte aligned, [B][T][D] of
+ * act_dtype; q may be NULL (x is then the query); y must not overlap x or q.
+ * final_states: optional DEVICE fp32 [B][heads][3*d*d + 2*d] (M_mem, M_k,
+ * M_v row-major, m_eta, m_alpha after the last token), NULL skips it.
+ * Asynchronous on `stream` (a cudaStream_t, NULL = legacy default stream). */
+SRNL_API srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
+                                      float* final_states, void* stream);
+
+/* Synchronously reads the status word of the handle's kernels (SRNL_OK or
+ * SRNL_E_TIMEOUT, as srnl_scan_device_status). */
+SRNL_API srnl_status srnl_seq_device_status(srnl_seq* h);
+
+/* Message for the last failure on this handle (h == NULL: the calling
+ * thread's last srnl_seq_create failure).  Never NULL. */
+SRNL_API const char* srnl_seq_last_error(const srnl_seq* h);
+
+/* Free the handle and its device memory.  Accepts NULL.  Synchronises the
+ * device before freeing. */
+SRNL_API void srnl_seq_destroy(srnl_seq* h);
 
 #ifdef __cplusplus
 }

@@ -29,7 +29,9 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_scan_forward_noalloc",
             "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
             "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_scan_workspace_bytes",
-            "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy")
+            "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy",
+            "srnl_seq_create", "srnl_seq_forward", "srnl_seq_device_status", "srnl_seq_last_error",
+            "srnl_seq_destroy")
 
 
 class SrnlError(RuntimeError):
@@ -48,6 +50,16 @@ class _Config(ctypes.Structure):
 class _Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("W_q", "scales", "M_mem0", "M_k0", "M_v0",
                                                 "m_eta0", "m_alpha0")]
+
+
+class _SeqConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("D", ctypes.c_int), ("heads", ctypes.c_int),
+                ("d", ctypes.c_int), ("alpha", ctypes.c_float), ("eps", ctypes.c_float),
+                ("chunk", ctypes.c_int), ("act_dtype", ctypes.c_int), ("gen_dtype", ctypes.c_int)]
+
+
+class _SeqParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -80,9 +92,17 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_status_string.restype = ctypes.c_char_p
     lib.srnl_scan_destroy.argtypes = [vp]
     lib.srnl_scan_destroy.restype = None
+    lib.srnl_seq_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(_SeqConfig), ctypes.POINTER(_SeqParams)]
+    lib.srnl_seq_forward.argtypes = [vp, vp, vp, vp, vp, vp]
+    lib.srnl_seq_device_status.argtypes = [vp]
+    lib.srnl_seq_last_error.argtypes = [vp]
+    lib.srnl_seq_last_error.restype = ctypes.c_char_p
+    lib.srnl_seq_destroy.argtypes = [vp]
+    lib.srnl_seq_destroy.restype = None
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
-                 "srnl_scan_stage_times", "srnl_scan_device_status"):
+                 "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_seq_create", "srnl_seq_forward",
+                 "srnl_seq_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -235,3 +255,68 @@ def srnl_status_string(status: int) -> str:
 
 def srnl_scan_last_error(h: Optional[SrnlScan] = None) -> str:
     return load_library().srnl_scan_last_error(h._h if h is not None else None).decode()
+
+
+# ------------------------------------------------ standalone sequence layer
+class SrnlSeq:
+    """Owns one ``srnl_seq*`` handle (the standalone SRNL layer on [B, T, D])."""
+
+    def __init__(self, handle: int, cfg: Dict):
+        self._h = handle
+        self.cfg = dict(cfg)
+
+    @property
+    def handle(self) -> int:
+        if not self._h:
+            raise RuntimeError("srnl_seq handle is closed")
+        return self._h
+
+    def _check(self, status: int, where: str):
+        if status != SRNL_OK:
+            raise SrnlError(status, where, load_library().srnl_seq_last_error(self._h).decode())
+
+    def close(self):
+        if self._h:
+            load_library().srnl_seq_destroy(self._h)
+            self._h = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def srnl_seq_create(cfg: Dict, params: Dict[str, np.ndarray]) -> SrnlSeq:
+    """cfg keys: B, T, D, heads, d, alpha, eps, chunk (0 = 64), act_dtype, gen_dtype.
+    params: float32 host arrays M_mem0, M_k0, M_v0 [heads, d, d], m_eta0, m_alpha0 [heads, d]."""
+    lib = load_library()
+
+    def dt(v):
+        return {"f32": SRNL_F32, "bf16": SRNL_BF16}.get(v, v)
+
+    c = _SeqConfig(B=cfg["B"], T=cfg["T"], D=cfg["D"], heads=cfg["heads"], d=cfg["d"], alpha=cfg["alpha"],
+                   eps=cfg.get("eps", 1e-6), chunk=cfg.get("chunk", 0), act_dtype=dt(cfg["act_dtype"]),
+                   gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])))
+    keep = {k: np.ascontiguousarray(params[k], dtype=np.float32)
+            for k in ("M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")}
+    p = _SeqParams(**{k: v.ctypes.data for k, v in keep.items()})
+    h = ctypes.c_void_p()
+    st = lib.srnl_seq_create(ctypes.byref(h), ctypes.byref(c), ctypes.byref(p))
+    if st != SRNL_OK:
+        raise SrnlError(st, "srnl_seq_create", lib.srnl_seq_last_error(None).decode())
+    return SrnlSeq(h.value, cfg)
+
+
+def srnl_seq_forward(h: SrnlSeq, x, y, q=None, final_states=None, stream=None) -> None:
+    """x, q, y: CUDA tensors [B, T, D] of act_dtype; q None means x is the query."""
+    h._check(load_library().srnl_seq_forward(h.handle, _ptr(x), _ptr(q), _ptr(y), _ptr(final_states),
+                                             _stream(stream)), "srnl_seq_forward")
+
+
+def srnl_seq_device_status(h: SrnlSeq) -> None:
+    h._check(load_library().srnl_seq_device_status(h.handle), "srnl_seq_device_status")
+
+
+def srnl_seq_destroy(h: SrnlSeq) -> None:
+    h.close()

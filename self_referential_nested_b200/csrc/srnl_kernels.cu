@@ -88,8 +88,18 @@ query_projection_kernel(const void* __restrict__ x, const float* __restrict__ Wq
 // Fusion epilogue: y = yr0 + yr1 + yr2 + yr3 (fixed order), 8 channels per
 // thread, 16-byte loads and stores.
 // ---------------------------------------------------------------------------
+// Element-wise bf16 <-> fp32 conversion (fp32 -> bf16 rounds to nearest even).
+__global__ void convert_kernel(const void* __restrict__ src, bool src_bf16, void* __restrict__ dst, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  if (src_bf16)
+    reinterpret_cast<float*>(dst)[i] = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(src)[i]);
+  else
+    reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(reinterpret_cast<const float*>(src)[i]);
+}
+
 __global__ void fuse_kernel(const float* __restrict__ yr, void* __restrict__ y, int64_t total,
-                            bool act_bf16) {
+                            int routes, bool act_bf16) {
   const int64_t i8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (i8 >= total) return;
   float acc[8];
@@ -101,6 +111,7 @@ __global__ void fuse_kernel(const float* __restrict__ yr, void* __restrict__ y, 
   }
 #pragma unroll
   for (int r = 1; r < 4; ++r) {
+    if (r >= routes) break;
     const float4 a = *reinterpret_cast<const float4*>(yr + r * total + i8);
     const float4 b = *reinterpret_cast<const float4*>(yr + r * total + i8 + 4);
     acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
@@ -163,7 +174,13 @@ cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_
   const int64_t total = (int64_t)g.B * g.H * g.W * g.C;
   const int64_t threads = total / 8;
   const int bs = 256;
-  fuse_kernel<<<(unsigned)((threads + bs - 1) / bs), bs, 0, s>>>(yr, y, total, g.act_bf16);
+  fuse_kernel<<<(unsigned)((threads + bs - 1) / bs), bs, 0, s>>>(yr, y, total, g.routes, g.act_bf16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert(const void* src, bool src_bf16, void* dst, int64_t n, cudaStream_t s) {
+  const int bs = 256;
+  convert_kernel<<<(unsigned)((n + bs - 1) / bs), bs, 0, s>>>(src, src_bf16, dst, n);
   return cudaGetLastError();
 }
 

@@ -9,6 +9,7 @@ namespace srnl {
 struct ScanGeom {
   int B, H, W, C, heads;
   int Lrow, Lcol;    // resolved chunk lengths (> 0)
+  int routes = 4;    // 4: the image operator; 1: a sequence (H = 1, route r0 only)
   float alpha, eps;
   bool act_bf16;     // x / y element type
   bool gen_bf16;     // generation + projection operands in bf16
@@ -37,10 +38,12 @@ cudaError_t launch_query_projection_tc(const ScanGeom& g, const ScanParamsDev& p
 cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
                         float* yr, float* finals, int* err, cudaStream_t s);
 
-// y = yr[0] + yr[1] + yr[2] + yr[3] in act dtype.
+// y = yr[0] + ... + yr[routes - 1] in act dtype, summed in route order.
 cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_t s);
 
 cudaError_t launch_route_index(int route, int H, int W, int32_t* out, cudaStream_t s);
+// dst[i] = src[i] converted between bf16 and fp32 (src_bf16: bf16 -> fp32, else fp32 -> bf16).
+cudaError_t launch_convert(const void* src, bool src_bf16, void* dst, int64_t n, cudaStream_t s);
 cudaError_t launch_gather(const ScanGeom& g, int route, const void* x, void* xr, cudaStream_t s);
 
 // The chunkwise tensor-core scan (bf16 generation); launch_scan dispatches to it.

@@ -420,7 +420,7 @@ cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x
   a.B = g.B; a.H = g.H; a.W = g.W; a.C = g.C; a.heads = g.heads;
   a.Lrow = g.Lrow; a.Lcol = g.Lcol; a.alpha = g.alpha; a.eps = g.eps;
   a.act_bf16 = g.act_bf16;
-  const unsigned nseq = 4u * (unsigned)g.B * (unsigned)g.heads;
+  const unsigned nseq = (unsigned)g.routes * (unsigned)g.B * (unsigned)g.heads;
   srnl_scan_sequential_kernel<<<nseq, kThreads, sizeof(Smem), s>>>(a);
   return cudaGetLastError();
 }

@@ -767,7 +767,7 @@ cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, con
   a.B = g.B; a.H = g.H; a.W = g.W; a.C = g.C; a.heads = g.heads;
   a.Lrow = g.Lrow; a.Lcol = g.Lcol; a.alpha = g.alpha; a.eps = g.eps;
   a.act_bf16 = g.act_bf16;
-  const unsigned nseq = 4u * (unsigned)g.B * (unsigned)g.heads;
+  const unsigned nseq = (unsigned)g.routes * (unsigned)g.B * (unsigned)g.heads;
   srnl_scan_chunkwise_kernel<<<nseq, kThreadsTc, sizeof(TcSmem), s>>>(a);
   return cudaGetLastError();
 }

@@ -1,0 +1,199 @@
+// C ABI of the standalone SRNL layer on sequences ("VisionHOPE" README, section "SRNL and
+// VisionHOPE operator": [batch, tokens, dim] in and out, optional queries, 64-token chunks
+// by default, an incomplete final chunk allowed, a new sequence on every call).
+//
+// A sequence is the image scan's route 0 on a 1 x T map with no fusion: the same scan
+// kernels run with one route, the fusion kernel reduces to a cast of the single partial
+// (scale 1), and the queries come from the caller instead of a projection.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "srnl_common.cuh"
+#include "srnl_internal.h"
+#include "srnl_launch.h"
+#include "srnl_scan.h"
+
+struct srnl_seq {
+  srnl_seq_config cfg{};
+  srnl::ScanGeom geom{};
+  int device = 0;
+  float* G = nullptr;       // [1][heads][66][32] generating initials
+  float* Mm = nullptr;      // [1][heads][32][32] content-memory initials
+  float* scales = nullptr;  // [1][D] ones
+  void* qbuf = nullptr;     // queries in the generation dtype when it differs from act_dtype
+  float* yr = nullptr;      // [1][B*T][D] fp32 partial
+  int* dev_err = nullptr;
+  std::string err;
+};
+
+namespace {
+
+thread_local std::string g_seq_create_error;
+
+srnl_status seq_fail(srnl_seq* h, srnl_status st, const std::string& msg) {
+  if (h != nullptr) h->err = msg; else g_seq_create_error = msg;
+  return st;
+}
+
+srnl_status seq_cuda_fail(srnl_seq* h, cudaError_t e, const char* what) {
+  return seq_fail(h, e == cudaErrorMemoryAllocation ? SRNL_E_NOMEM : SRNL_E_CUDA,
+                  std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
+}
+
+void seq_free(srnl_seq* h) {
+  void* ptrs[] = {h->G, h->Mm, h->scales, h->qbuf, h->yr, h->dev_err};
+  for (void* p : ptrs)
+    if (p != nullptr) cudaFree(p);
+  h->G = h->Mm = h->scales = h->yr = nullptr;
+  h->qbuf = nullptr;
+  h->dev_err = nullptr;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, const void* b, size_t n) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + n && y < x + n;
+}
+
+}  // namespace
+
+extern "C" {
+
+srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const srnl_seq_params* prm) {
+  if (out == nullptr) return seq_fail(nullptr, SRNL_E_INVAL, "out is NULL");
+  *out = nullptr;
+  if (cfg == nullptr || prm == nullptr) return seq_fail(nullptr, SRNL_E_INVAL, "cfg or params is NULL");
+  if (prm->M_mem0 == nullptr || prm->M_k0 == nullptr || prm->M_v0 == nullptr || prm->m_eta0 == nullptr ||
+      prm->m_alpha0 == nullptr)
+    return seq_fail(nullptr, SRNL_E_INVAL, "a parameter pointer is NULL");
+  if (cfg->B <= 0 || cfg->T <= 0 || cfg->D <= 0 || cfg->heads <= 0 || cfg->d <= 0)
+    return seq_fail(nullptr, SRNL_E_INVAL, "B, T, D, heads and d must be positive");
+  if (cfg->chunk < 0) return seq_fail(nullptr, SRNL_E_INVAL, "chunk must be >= 0 (0 = 64)");
+  // the rest of the checks are those of a 1 x T image
+  srnl_scan_config sc{};
+  sc.B = cfg->B; sc.H = 1; sc.W = cfg->T; sc.C = cfg->D; sc.heads = cfg->heads; sc.d = cfg->d;
+  sc.alpha = cfg->alpha; sc.eps = cfg->eps;
+  sc.chunk_row = sc.chunk_col = cfg->chunk > 0 ? cfg->chunk : 64;
+  sc.act_dtype = cfg->act_dtype; sc.gen_dtype = cfg->gen_dtype;
+  srnl_status st = srnl::validate_scan_config(&sc);
+  if (st != SRNL_OK) {
+    return seq_fail(nullptr, st, std::string("invalid sequence config: ") + srnl_scan_last_error(nullptr));
+  }
+  srnl_seq* h = new (std::nothrow) srnl_seq;
+  if (h == nullptr) return seq_fail(nullptr, SRNL_E_NOMEM, "host allocation failed");
+  h->cfg = *cfg;
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "cudaGetDevice"); delete h; return st; }
+
+  const int d = srnl::kD, nh = cfg->heads;
+  srnl::ScanGeom& g = h->geom;
+  g.B = cfg->B; g.H = 1; g.W = cfg->T; g.C = cfg->D; g.heads = nh;
+  g.Lrow = g.Lcol = sc.chunk_row;
+  g.alpha = cfg->alpha; g.eps = cfg->eps;
+  g.act_bf16 = cfg->act_dtype == SRNL_BF16;
+  g.gen_bf16 = cfg->gen_dtype == SRNL_BF16;
+  g.routes = 1;
+
+  std::vector<float> G((size_t)nh * srnl::kGen * d);
+  for (int hh = 0; hh < nh; ++hh) {
+    float* dst = G.data() + (size_t)hh * srnl::kGen * d;
+    std::memcpy(dst, prm->M_k0 + (size_t)hh * d * d, sizeof(float) * d * d);
+    std::memcpy(dst + d * d, prm->M_v0 + (size_t)hh * d * d, sizeof(float) * d * d);
+    std::memcpy(dst + 2 * d * d, prm->m_eta0 + (size_t)hh * d, sizeof(float) * d);
+    std::memcpy(dst + 2 * d * d + d, prm->m_alpha0 + (size_t)hh * d, sizeof(float) * d);
+  }
+  const std::vector<float> ones((size_t)cfg->D, 1.f);
+  const size_t tokens = (size_t)cfg->B * cfg->T;
+  const size_t n_mm = (size_t)nh * d * d;
+  const size_t qbuf_bytes = g.act_bf16 != g.gen_bf16 ? tokens * cfg->D * (g.gen_bf16 ? 2 : 4) : 0;
+  struct { void** p; size_t n; } allocs[] = {
+      {(void**)&h->G, G.size() * sizeof(float)}, {(void**)&h->Mm, n_mm * sizeof(float)},
+      {(void**)&h->scales, ones.size() * sizeof(float)}, {&h->qbuf, qbuf_bytes},
+      {(void**)&h->yr, tokens * cfg->D * sizeof(float)}, {(void**)&h->dev_err, sizeof(int)}};
+  for (auto& a : allocs) {
+    if (a.n == 0) continue;
+    e = cudaMalloc(a.p, a.n);
+    if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "cudaMalloc"); seq_free(h); delete h; return st; }
+  }
+  struct { void* dst; const void* src; size_t n; } copies[] = {
+      {h->G, G.data(), G.size() * sizeof(float)}, {h->Mm, prm->M_mem0, n_mm * sizeof(float)},
+      {h->scales, ones.data(), ones.size() * sizeof(float)}};
+  for (auto& cp : copies) {
+    e = cudaMemcpy(cp.dst, cp.src, cp.n, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "cudaMemcpy (params)"); seq_free(h); delete h; return st; }
+  }
+  e = cudaMemset(h->dev_err, 0, sizeof(int));
+  if (e == cudaSuccess) e = srnl::prepare_kernels();
+  if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "set-up"); seq_free(h); delete h; return st; }
+  *out = h;
+  return SRNL_OK;
+}
+
+srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y, float* final_states,
+                             void* stream) {
+  if (h == nullptr) return SRNL_E_INVAL;
+  h->err.clear();
+  if (x == nullptr || y == nullptr) return seq_fail(h, SRNL_E_INVAL, "x or y is NULL");
+  if (!aligned16(x) || !aligned16(y) || (q != nullptr && !aligned16(q)) ||
+      (final_states != nullptr && !aligned16(final_states)))
+    return seq_fail(h, SRNL_E_INVAL, "x, q, y and final_states must be 16-byte aligned");
+  const srnl::ScanGeom& g = h->geom;
+  const size_t n = (size_t)g.B * g.W * g.C;
+  const size_t bytes = n * (g.act_bf16 ? 2 : 4);
+  if (overlap(x, y, bytes) || (q != nullptr && overlap(q, y, bytes)))
+    return seq_fail(h, SRNL_E_INVAL, "y overlaps x or q");
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "cudaGetDevice");
+  if (cur != h->device) return seq_fail(h, SRNL_E_INVAL, "the current device is not the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* qk = q != nullptr ? q : x;
+  if (g.act_bf16 != g.gen_bf16) {  // queries in the generation dtype
+    e = srnl::launch_convert(qk, g.act_bf16, h->qbuf, (int64_t)n, s);
+    if (e != cudaSuccess) return seq_cuda_fail(h, e, "query conversion launch");
+    qk = h->qbuf;
+  }
+  const srnl::ScanParamsDev p{nullptr, nullptr, h->G, h->Mm, h->scales};
+  e = srnl::launch_scan(g, p, x, qk, h->yr, final_states, h->dev_err, s);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "scan launch");
+  e = srnl::launch_fuse(g, h->yr, y, s);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "output launch");
+  return SRNL_OK;
+}
+
+srnl_status srnl_seq_device_status(srnl_seq* h) {
+  if (h == nullptr) return SRNL_E_INVAL;
+  int v = 0;
+  const cudaError_t e = cudaMemcpy(&v, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "status read");
+  if (v != 0) {
+    h->err = "a bounded in-kernel wait gave up";
+    return static_cast<srnl_status>(v);
+  }
+  return SRNL_OK;
+}
+
+const char* srnl_seq_last_error(const srnl_seq* h) {
+  return h != nullptr ? h->err.c_str() : g_seq_create_error.c_str();
+}
+
+void srnl_seq_destroy(srnl_seq* h) {
+  if (h == nullptr) return;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  if (prev != h->device) cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  seq_free(h);
+  if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
+  delete h;
+}
+
+}  // extern "C"

@@ -135,3 +135,53 @@ def make_inputs(cfg: ScanConfig, seed: int = 0, *, x_scale: float = 1.0,
     return ScanInputs(cfg=cfg, x32=np.ascontiguousarray(x), x_bits=x_bits, W_q=W_q,
                       scales=scales, M_mem0=M_mem0, M_k0=M_k0, M_v0=M_v0,
                       m_eta0=m_eta0, m_alpha0=m_alpha0)
+
+
+# ------------------------------------------------ standalone sequence layer
+@dataclasses.dataclass
+class SeqInputs:
+    """Seeded inputs of the standalone sequence layer: x and queries [B, T, D] (fp32 values,
+    bf16-exact when act_dtype is bf16) and one set of initial states per head."""
+    B: int
+    T: int
+    D: int
+    heads: int
+    act_dtype: str
+    x32: np.ndarray
+    q32: np.ndarray
+    x_bits: Optional[np.ndarray]
+    q_bits: Optional[np.ndarray]
+    M_mem0: np.ndarray
+    M_k0: np.ndarray
+    M_v0: np.ndarray
+    m_eta0: np.ndarray
+    m_alpha0: np.ndarray
+
+    def params(self) -> Dict[str, np.ndarray]:
+        return dict(M_mem0=self.M_mem0, M_k0=self.M_k0, M_v0=self.M_v0, m_eta0=self.m_eta0,
+                    m_alpha0=self.m_alpha0)
+
+
+def make_seq_inputs(B: int, T: int, D: int, heads: int, act_dtype: str = F32, seed: int = 0, *,
+                    mem_scale: float = 0.02, vec_scale: float = 0.1) -> SeqInputs:
+    """Draw x, queries ~ N(0, 1) [B, T, D], then M_mem0, M_k0, M_v0 ~ N(0, mem_scale^2)
+    [heads, d, d] and m_eta0, m_alpha0 ~ N(0, vec_scale^2) [heads, d], in that order."""
+    rng = np.random.default_rng(seed)
+    d = D // heads
+    x = rng.standard_normal((B, T, D), dtype=np.float32)
+    q = rng.standard_normal((B, T, D), dtype=np.float32)
+    M_mem0 = (rng.standard_normal((heads, d, d)) * mem_scale).astype(np.float32)
+    M_k0 = (rng.standard_normal((heads, d, d)) * mem_scale).astype(np.float32)
+    M_v0 = (rng.standard_normal((heads, d, d)) * mem_scale).astype(np.float32)
+    m_eta0 = (rng.standard_normal((heads, d)) * vec_scale).astype(np.float32)
+    m_alpha0 = (rng.standard_normal((heads, d)) * vec_scale).astype(np.float32)
+    x_bits = q_bits = None
+    if act_dtype == BF16:
+        x_bits, q_bits = bf16_round_bits(x), bf16_round_bits(q)
+        x = bf16_bits_to_f32(x_bits).reshape(x.shape)
+        q = bf16_bits_to_f32(q_bits).reshape(q.shape)
+    elif act_dtype != F32:
+        raise ValueError(f"unknown act_dtype {act_dtype!r}")
+    return SeqInputs(B=B, T=T, D=D, heads=heads, act_dtype=act_dtype, x32=np.ascontiguousarray(x),
+                     q32=np.ascontiguousarray(q), x_bits=x_bits, q_bits=q_bits, M_mem0=M_mem0, M_k0=M_k0,
+                     M_v0=M_v0, m_eta0=m_eta0, m_alpha0=m_alpha0)

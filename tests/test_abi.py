@@ -98,3 +98,35 @@ def test_product_package_never_imports_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, f), errors="ignore").read()
                 assert not pat.search(src), f
+
+
+# ------------------------------------------------ standalone sequence layer
+def _seq_cfg(**kw):
+    c = dict(B=2, T=257, D=64, heads=2, d=32, alpha=0.95, eps=1e-6, chunk=0, act_dtype="f32", gen_dtype="f32")
+    c.update(kw)
+    return c
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(B=0), S.SRNL_E_INVAL),
+    (dict(T=-1), S.SRNL_E_INVAL),
+    (dict(D=63), S.SRNL_E_INVAL),
+    (dict(alpha=1.0), S.SRNL_E_INVAL),
+    (dict(eps=0.0), S.SRNL_E_INVAL),
+    (dict(chunk=-1), S.SRNL_E_INVAL),
+    (dict(gen_dtype=5), S.SRNL_E_INVAL),
+    (dict(D=32, heads=2, d=16), S.SRNL_E_UNSUPPORTED),
+])
+def test_seq_create_rejects_bad_config_before_cuda(lib, bad, status):
+    from srnl_inputs import make_seq_inputs
+    inp = make_seq_inputs(1, 4, 64, 2)
+    with pytest.raises(S.SrnlError) as e:
+        S.srnl_seq_create(_seq_cfg(**bad), inp.params())
+    assert e.value.status == status
+
+
+def test_seq_null_handle_calls_fail_cleanly(lib):
+    assert lib.srnl_seq_forward(None, None, None, None, None, None) == S.SRNL_E_INVAL
+    assert lib.srnl_seq_device_status(None) == S.SRNL_E_INVAL
+    lib.srnl_seq_destroy(None)
+    assert isinstance(lib.srnl_seq_last_error(None), bytes)
