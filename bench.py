@@ -34,6 +34,12 @@ sys.path.insert(0, ROOT)
 from srnl_inputs import CONFIGS, make_inputs  # noqa: E402
 
 METRIC = "SRNL 4-dir scan tokens/s (fwd, 1xB200) and % of roofline at 56x56x64"
+
+# DRAM bytes (read + write) of one scan launch, from a 1-pass ncu capture of the current
+# chunkwise kernel on the full workload (profiles/scan_kernel_hier_s1_56x56_b4.md):
+# 29.02 MB read + 48.13 MB written.  Keyed by (workload, B, generation dtype); absent
+# entries report null.
+SCAN_TRAFFIC_BYTES = {("hier_s1_56x56", 32, "bf16"): 29.02e6 + 48.13e6}
 UNIT = "route-tokens/s"
 DEFAULT_CONFIG = "hier_s1_56x56"
 L2_FLUSH_BYTES = 256 << 20
@@ -323,7 +329,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "raster_tokens_per_s": value / 4},
         "roofline": {"bound": "alu", "achieved": scan_tflops, "peak": fp32_peak_tflops,
-                     "unit": "TFLOP/s", "frac": scan_tflops / fp32_peak_tflops, "traffic": None,
+                     "unit": "TFLOP/s", "frac": scan_tflops / fp32_peak_tflops,
+                     "traffic": SCAN_TRAFFIC_BYTES.get((cfg.name, cfg.B, gen)), "traffic_unit": "bytes/launch",
                      "kernel": "srnl_scan_chunkwise_kernel" if gen == "bf16" else "srnl_scan_sequential_kernel",
                      "kernel_ms": scan_ms,
                      "peak_note": "fp32 FMA peak 148 SM x 128 lanes x 2 x sm_max_mhz (derived)"},
