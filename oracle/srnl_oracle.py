@@ -34,6 +34,10 @@ tests/test_oracle_pins.py:
     spanning the sequence generates every token from the initial states;
   * five-memory form equals the single-product form to 1e-12;
   * one-hot fusion scales isolate routes; batch permutation equivariance;
+  * hard injection clamp: eta1 g <= 1 - alpha_t with equality where it binds, eta1 =
+    eta0 elsewhere; no binds for tiny steps (then it matches the soft cap to O(z^2)),
+    every token binds for huge steps; norms stay non-increasing; chunk 1 equals the
+    token-wise loop;
   * standalone sequence layer: chunk 1 equals the token-wise loop, outputs are causal
     (a prefix of the input gives the prefix of the output), absent queries mean x, and
     it equals route 0 of the operator with W_q = I and a one-hot route-0 scale.
@@ -139,6 +143,19 @@ def soft_cap(eta0: np.ndarray, gain: np.ndarray, alpha_t: np.ndarray) -> np.ndar
     return eta0 * phi
 
 
+def hard_cap(eta0: np.ndarray, gain: np.ndarray, alpha_t: np.ndarray):
+    """Hard injection clamp, the ablation of the soft cap ([SUMMARY] results paragraph:
+    "hard injection clamp", active on a share of token updates; [SUMMARY] stability list:
+    the soft cap limits the step smoothly rather than by clipping).  Reading: clip the
+    step so that eta1 * g <= 1 - alpha_t, i.e. eta1 = min(eta0, (1 - alpha_t) / g).
+    Returns (eta1, binds) with binds = eta0 * g > 1 - alpha_t (the clamp is active).
+    """
+    margin = 1.0 - alpha_t
+    binds = eta0 * gain > margin
+    safe = np.where(binds, gain, 1.0)
+    return np.where(binds, margin / safe, eta0), binds
+
+
 def spectral_clamp(eta1: np.ndarray, knorm2: np.ndarray) -> np.ndarray:
     """eta = min(eta1, 2 / ||k||^2): then alpha_t (I - eta k k^T) has norm alpha_t."""
     over = eta1 * knorm2 > 2.0
@@ -146,20 +163,26 @@ def spectral_clamp(eta1: np.ndarray, knorm2: np.ndarray) -> np.ndarray:
     return np.where(over, 2.0 / safe, eta1)
 
 
-def gates(ktil, v, a, beta, alpha_max, eps):
+def gates(ktil, v, a, beta, alpha_max, eps, cap="soft"):
     """All per-token scalars/vectors from the generated quantities.
 
     Returns dict with k (normalised key), alpha_t, eta0 (proposed step), eta1
-    (after the soft cap), eta (after the spectral clamp), gain.
+    (after the injection cap: ``cap`` = "soft" or "hard"), eta (after the spectral
+    clamp), gain, and binds (where the hard clamp is active; all False for "soft").
     """
     k = stabilized_key(ktil, eps)
     alpha_t = retention(beta, alpha_max)
     eta0 = softplus(a)
     kn = np.sqrt(np.sum(k * k, axis=-1))
     gain = np.sqrt(np.sum((k - v) ** 2, axis=-1)) * kn
-    eta1 = soft_cap(eta0, gain, alpha_t)
+    if cap == "soft":
+        eta1, binds = soft_cap(eta0, gain, alpha_t), np.zeros(eta0.shape, dtype=bool)
+    elif cap == "hard":
+        eta1, binds = hard_cap(eta0, gain, alpha_t)
+    else:
+        raise ValueError(cap)
     eta = spectral_clamp(eta1, kn * kn)
-    return dict(k=k, alpha_t=alpha_t, eta0=eta0, eta1=eta1, eta=eta, gain=gain)
+    return dict(k=k, alpha_t=alpha_t, eta0=eta0, eta1=eta1, eta=eta, gain=gain, binds=binds)
 
 
 # --------------------------------------------------------------------------
@@ -217,7 +240,7 @@ def _generate(mem, d, X):
 
 
 def scan_five_memory(xs, qs, inits, chunk, alpha_max, eps, *, readout="post",
-                     eta_override=None, alpha_override=None, trace=False):
+                     eta_override=None, alpha_override=None, trace=False, cap="soft", counter=None):
     """The chunked scan over S independent sequences, literally with five memories.
 
     xs, qs: [S, N, d] float64 (memory input x_t and query q_t, route order).
@@ -229,6 +252,8 @@ def scan_five_memory(xs, qs, inits, chunk, alpha_max, eps, *, readout="post",
     readout).  The boundary refreshes at the end of the chunk.  The final chunk
     may be shorter than ``chunk`` ([README] "SRNL and VisionHOPE operator").
 
+    ``cap`` selects the soft cap or the hard clamp; ``counter`` (a one-element list) collects
+    the number of token updates where the hard clamp is active.
     Returns y [S, N, d], final memories dict, and a trace dict when asked.
     """
     S, N, d = xs.shape
@@ -253,7 +278,9 @@ def scan_five_memory(xs, qs, inits, chunk, alpha_max, eps, *, readout="post",
     for c0 in range(0, N, chunk):
         c1 = min(c0 + chunk, N)
         ktil, v, a, beta = _generate(mem, d, xs[:, c0:c1])
-        gt = gates(ktil, v, a, beta, alpha_max, eps)
+        gt = gates(ktil, v, a, beta, alpha_max, eps, cap)
+        if counter is not None:
+            counter[0] += int(np.count_nonzero(gt["binds"]))
         eta = gt["eta"] if eta_override is None else np.full_like(gt["eta"], eta_override)
         alpha_t = gt["alpha_t"] if alpha_override is None else np.full_like(gt["alpha_t"], alpha_override)
         for j in range(c1 - c0):
@@ -315,7 +342,7 @@ def scan_qform(xs, qs, inits, chunk, alpha_max, eps):
     return y, final
 
 
-def scan_tokenwise(xs, qs, inits, alpha_max, eps):
+def scan_tokenwise(xs, qs, inits, alpha_max, eps, cap="soft"):
     """Pure token-wise recurrence: every token is generated from X_{t-1}.
 
     Written without any chunk bookkeeping; the chunked scan with chunk length 1
@@ -339,7 +366,8 @@ def scan_tokenwise(xs, qs, inits, alpha_max, eps):
         e0 = softplus(a)
         kn2 = np.sum(k ** 2, axis=1)
         g = np.sqrt(np.sum((k - v) ** 2, axis=1) * kn2)
-        e = spectral_clamp(soft_cap(e0, g, al), kn2)
+        e1 = soft_cap(e0, g, al) if cap == "soft" else np.minimum(e0, (1.0 - al) / np.maximum(g, 1e-300))
+        e = spectral_clamp(e1, kn2)
 
         def write(X):  # X: [S, m, d]
             Xk = np.einsum("smd,sd->sm", X, k)
@@ -378,7 +406,7 @@ def _route_inits(inputs_params, route, B):
 
 def operator_forward(x, params, *, alpha_max, eps=1e-6, chunk_row=0, chunk_col=0,
                      heads, scan="five", readout="post", eta_override=None,
-                     alpha_override=None, trace=False):
+                     alpha_override=None, trace=False, cap="soft", counter=None):
     """Full forward of the four-direction scan.
 
     x: [B, H, W, C] (any float; promoted to float64).  params: dict with W_q
@@ -405,12 +433,12 @@ def operator_forward(x, params, *, alpha_max, eps=1e-6, chunk_row=0, chunk_col=0
         if scan == "five":
             y, fin, tr = scan_five_memory(xr, qr, inits, L, alpha_max, eps, readout=readout,
                                           eta_override=eta_override, alpha_override=alpha_override,
-                                          trace=trace)
+                                          trace=trace, cap=cap, counter=counter)
             traces.append(tr)
         elif scan == "qform":
             y, fin = scan_qform(xr, qr, inits, L, alpha_max, eps)
         elif scan == "tokenwise":
-            y, fin = scan_tokenwise(xr, qr, inits, alpha_max, eps)
+            y, fin = scan_tokenwise(xr, qr, inits, alpha_max, eps, cap)
         else:
             raise ValueError(scan)
         yr = y.reshape(B, heads, N, d).transpose(0, 2, 1, 3).reshape(B, N, C)
@@ -422,7 +450,8 @@ def operator_forward(x, params, *, alpha_max, eps=1e-6, chunk_row=0, chunk_col=0
     return out, finals, (traces if trace else None)
 
 
-def sequence_forward(x, params, *, alpha_max, eps=1e-6, chunk=64, heads, queries=None, scan="five"):
+def sequence_forward(x, params, *, alpha_max, eps=1e-6, chunk=64, heads, queries=None, scan="five",
+                     cap="soft", counter=None):
     """Standalone SRNL layer on sequences ([README] "SRNL and VisionHOPE operator": a layer
     on [batch, tokens, dim] that returns the same shape, one pass in token order, 64-token
     chunks unless told otherwise, an incomplete final chunk allowed; queries of the same shape
@@ -446,9 +475,9 @@ def sequence_forward(x, params, *, alpha_max, eps=1e-6, chunk=64, heads, queries
         arr = np.asarray(params[key], dtype=np.float64)  # [heads, ...]
         inits[name] = np.broadcast_to(arr[None], (B,) + arr.shape).reshape((-1,) + arr.shape[1:]).copy()
     if scan == "five":
-        y, fin, _ = scan_five_memory(xs, qs, inits, L, alpha_max, eps)
+        y, fin, _ = scan_five_memory(xs, qs, inits, L, alpha_max, eps, cap=cap, counter=counter)
     elif scan == "tokenwise":
-        y, fin = scan_tokenwise(xs, qs, inits, alpha_max, eps)
+        y, fin = scan_tokenwise(xs, qs, inits, alpha_max, eps, cap)
     else:
         raise ValueError(scan)
     y = y.reshape(B, heads, T, d).transpose(0, 2, 1, 3).reshape(B, T, D)

@@ -420,3 +420,55 @@ def test_sequence_equals_operator_route0():
                                      heads=heads)
     assert np.allclose(out.reshape(B, T, D), ys, rtol=1e-12, atol=1e-14)
     assert np.allclose(fin[0], fs, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------ hard injection clamp
+def test_hard_cap_bound_is_tight():
+    rng = np.random.default_rng(21)
+    eta0 = rng.uniform(0, 3, 2000)
+    gain = rng.uniform(0.01, 2, 2000)
+    al = rng.uniform(0.05, 0.95, 2000)
+    e1, binds = O.hard_cap(eta0, gain, al)
+    assert np.all(e1 * gain <= (1 - al) * (1 + 1e-14))
+    assert np.allclose(e1[binds] * gain[binds], (1 - al[binds]), rtol=1e-13)
+    assert np.array_equal(e1[~binds], eta0[~binds])
+    assert 100 < np.count_nonzero(binds) < 1900
+
+
+def test_hard_cap_extremes():
+    # one chunk spanning the sequence: every token is generated from the initial states
+    rng = np.random.default_rng(22)
+    T = 24
+    x = np.abs(rng.normal(size=(2, T, 8)))  # positive inputs: a = m_eta0 . x has the sign of m_eta0
+    p = _seq_params(2, 4, rng)
+    total = 2 * 2 * T
+    for m_eta, expect in ((+5.0, "all"), (-30.0, "none")):
+        p["m_eta0"] = np.full_like(p["m_eta0"], m_eta)
+        cnt = [0]
+        yh, _ = O.sequence_forward(x, p, alpha_max=0.9, chunk=T, heads=2, cap="hard", counter=cnt)
+        ys, _ = O.sequence_forward(x, p, alpha_max=0.9, chunk=T, heads=2, cap="soft")
+        if expect == "all":
+            # huge steps: the clamp is active on every token (and the soft cap saturates at
+            # the same margin, so both give nearly the same write)
+            assert cnt[0] == total
+        else:
+            assert cnt[0] == 0  # tiny steps: never active, and the soft cap is eta0 (1 - O(z^2))
+            assert np.allclose(yh, ys, rtol=1e-9, atol=1e-15)
+
+
+def test_hard_cap_nonexpansive_and_tokenwise():
+    rng = np.random.default_rng(24)
+    S, N, d = 3, 30, 4
+    xs = rng.normal(size=(S, N, d))
+    qs = rng.normal(size=(S, N, d))
+    inits = dict(M_mem=rng.normal(0, 0.5, (S, d, d)), M_k=rng.normal(0, 0.5, (S, d, d)),
+                 M_v=rng.normal(0, 0.5, (S, d, d)), m_eta=rng.normal(0, 2, (S, d)), m_alpha=rng.normal(0, 2, (S, d)))
+    cnt = [0]
+    y, fin, tr = O.scan_five_memory(xs, qs, inits, 5, 0.9, 1e-6, trace=True, cap="hard", counter=cnt)
+    for name, f in tr["fro"].items():
+        assert np.all(np.diff(f, axis=1) <= 1e-12 * (1 + f[:, :-1])), name
+    assert cnt[0] == int(np.count_nonzero(tr["eta0"] * tr["gain"] > 1 - tr["alpha_t"]))
+    assert 0 < cnt[0] < S * N
+    y1, f1, _ = O.scan_five_memory(xs, qs, inits, 1, 0.9, 1e-6, cap="hard")
+    y2, f2 = O.scan_tokenwise(xs, qs, inits, 0.9, 1e-6, cap="hard")
+    assert np.allclose(y1, y2, rtol=1e-11, atol=1e-13)
