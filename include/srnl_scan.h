@@ -90,6 +90,13 @@ typedef enum {
 
 typedef enum { SRNL_F32 = 0, SRNL_BF16 = 1 } srnl_dtype;
 
+/* Injection cap on the proposed step ("VisionHOPE: Visual Backbones as Self-Modifying
+ * Learning Systems", stability and results paragraphs): the soft cap
+ * eta1 = eta0 tanh(z)/z, z = eta0 g / (1 - alpha_t) (the method), or the hard clamp of its
+ * ablation, eta1 = min(eta0, (1 - alpha_t) / g), which is "active" on a token update when
+ * eta0 g > 1 - alpha_t. */
+typedef enum { SRNL_CAP_SOFT = 0, SRNL_CAP_HARD = 1 } srnl_cap;
+
 typedef struct {
   int B, H, W, C; /* batch, height, width, channels (C = heads * d) */
   int heads, d;   /* heads and head dim; d = 32 is built */
@@ -99,6 +106,7 @@ typedef struct {
   int chunk_col;  /* chunk length on routes 2/3; 0 means H (full columns) */
   int act_dtype;  /* srnl_dtype of x and y */
   int gen_dtype;  /* srnl_dtype of generation / projection operands */
+  int injection_cap; /* srnl_cap; 0 = SRNL_CAP_SOFT */
 } srnl_scan_config;
 
 /* Parameters, HOST pointers to dense fp32 arrays.  srnl_scan_create copies and
@@ -191,6 +199,11 @@ SRNL_API srnl_status srnl_scan_stage_times(srnl_scan* h, float* ms_out, int* cou
  * (outputs of that forward are then unspecified). */
 SRNL_API srnl_status srnl_scan_device_status(srnl_scan* h);
 
+/* Number of token updates (all routes, batches and heads) of the last forward on which
+ * the hard injection clamp was active; 0 under the soft cap.  Synchronises the device.
+ * (srnl_scan_forward_noalloc does not count.) */
+SRNL_API srnl_status srnl_scan_cap_count(srnl_scan* h, unsigned long long* count);
+
 /* Bytes of device workspace the handle holds (packed params excluded). */
 SRNL_API size_t srnl_scan_workspace_bytes(const srnl_scan* h);
 
@@ -229,6 +242,7 @@ typedef struct {
   int chunk;      /* chunk length; 0 means 64 */
   int act_dtype;  /* srnl_dtype of x, the queries and y */
   int gen_dtype;  /* srnl_dtype of generation / query operands */
+  int injection_cap; /* srnl_cap; 0 = SRNL_CAP_SOFT */
 } srnl_seq_config;
 
 /* Initial states, HOST pointers to dense fp32 arrays, copied by create. */
@@ -256,6 +270,9 @@ SRNL_API srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q,
 /* Synchronously reads the status word of the handle's kernels (SRNL_OK or
  * SRNL_E_TIMEOUT, as srnl_scan_device_status). */
 SRNL_API srnl_status srnl_seq_device_status(srnl_seq* h);
+
+/* Hard-clamp activations of the last forward (see srnl_scan_cap_count). */
+SRNL_API srnl_status srnl_seq_cap_count(srnl_seq* h, unsigned long long* count);
 
 /* Message for the last failure on this handle (h == NULL: the calling
  * thread's last srnl_seq_create failure).  Never NULL. */

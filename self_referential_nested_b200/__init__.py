@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libsrnl_scan.so")
 
 SRNL_OK, SRNL_E_INVAL, SRNL_E_UNSUPPORTED, SRNL_E_CUDA, SRNL_E_NOMEM, SRNL_E_TIMEOUT = 0, -1, -2, -3, -4, -5
 SRNL_F32, SRNL_BF16 = 0, 1
+SRNL_CAP_SOFT, SRNL_CAP_HARD = 0, 1
 STATE_FLOATS_D32 = 3 * 32 * 32 + 2 * 32
 
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -31,7 +32,7 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_scan_workspace_bytes",
             "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy",
             "srnl_seq_create", "srnl_seq_forward", "srnl_seq_device_status", "srnl_seq_last_error",
-            "srnl_seq_destroy")
+            "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count")
 
 
 class SrnlError(RuntimeError):
@@ -44,7 +45,7 @@ class _Config(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int), ("C", ctypes.c_int),
                 ("heads", ctypes.c_int), ("d", ctypes.c_int), ("alpha", ctypes.c_float),
                 ("eps", ctypes.c_float), ("chunk_row", ctypes.c_int), ("chunk_col", ctypes.c_int),
-                ("act_dtype", ctypes.c_int), ("gen_dtype", ctypes.c_int)]
+                ("act_dtype", ctypes.c_int), ("gen_dtype", ctypes.c_int), ("injection_cap", ctypes.c_int)]
 
 
 class _Params(ctypes.Structure):
@@ -55,7 +56,8 @@ class _Params(ctypes.Structure):
 class _SeqConfig(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("D", ctypes.c_int), ("heads", ctypes.c_int),
                 ("d", ctypes.c_int), ("alpha", ctypes.c_float), ("eps", ctypes.c_float),
-                ("chunk", ctypes.c_int), ("act_dtype", ctypes.c_int), ("gen_dtype", ctypes.c_int)]
+                ("chunk", ctypes.c_int), ("act_dtype", ctypes.c_int), ("gen_dtype", ctypes.c_int),
+                ("injection_cap", ctypes.c_int)]
 
 
 class _SeqParams(ctypes.Structure):
@@ -99,10 +101,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_seq_last_error.restype = ctypes.c_char_p
     lib.srnl_seq_destroy.argtypes = [vp]
     lib.srnl_seq_destroy.restype = None
+    lib.srnl_scan_cap_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.srnl_seq_cap_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
                  "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_seq_create", "srnl_seq_forward",
-                 "srnl_seq_device_status"):
+                 "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -162,6 +166,10 @@ class SrnlScan:
         return int(load_library().srnl_scan_workspace_bytes(self.handle))
 
 
+def _cap(v) -> int:
+    return {"soft": SRNL_CAP_SOFT, "hard": SRNL_CAP_HARD}.get(v, v)
+
+
 def _config_struct(cfg: Dict) -> _Config:
     def dt(v):
         return {"f32": SRNL_F32, "bf16": SRNL_BF16}.get(v, v)
@@ -169,7 +177,8 @@ def _config_struct(cfg: Dict) -> _Config:
     return _Config(B=cfg["B"], H=cfg["H"], W=cfg["W"], C=cfg["C"], heads=cfg["heads"], d=cfg["d"],
                    alpha=cfg["alpha"], eps=cfg.get("eps", 1e-6), chunk_row=cfg.get("chunk_row", 0),
                    chunk_col=cfg.get("chunk_col", 0), act_dtype=dt(cfg["act_dtype"]),
-                   gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])))
+                   gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])),
+                   injection_cap=_cap(cfg.get("injection_cap", "soft")))
 
 
 def srnl_scan_create(cfg: Dict, params: Dict[str, np.ndarray]) -> SrnlScan:
@@ -245,6 +254,13 @@ def srnl_scan_device_status(h: SrnlScan) -> None:
     h._check(load_library().srnl_scan_device_status(h.handle), "srnl_scan_device_status")
 
 
+def srnl_scan_cap_count(h: SrnlScan) -> int:
+    """Token updates of the last forward on which the hard clamp was active (synchronises)."""
+    v = ctypes.c_ulonglong(0)
+    h._check(load_library().srnl_scan_cap_count(h.handle, ctypes.byref(v)), "srnl_scan_cap_count")
+    return int(v.value)
+
+
 def srnl_scan_destroy(h: SrnlScan) -> None:
     h.close()
 
@@ -297,7 +313,8 @@ def srnl_seq_create(cfg: Dict, params: Dict[str, np.ndarray]) -> SrnlSeq:
 
     c = _SeqConfig(B=cfg["B"], T=cfg["T"], D=cfg["D"], heads=cfg["heads"], d=cfg["d"], alpha=cfg["alpha"],
                    eps=cfg.get("eps", 1e-6), chunk=cfg.get("chunk", 0), act_dtype=dt(cfg["act_dtype"]),
-                   gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])))
+                   gen_dtype=dt(cfg.get("gen_dtype", cfg["act_dtype"])),
+                   injection_cap=_cap(cfg.get("injection_cap", "soft")))
     keep = {k: np.ascontiguousarray(params[k], dtype=np.float32)
             for k in ("M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")}
     p = _SeqParams(**{k: v.ctypes.data for k, v in keep.items()})
@@ -316,6 +333,13 @@ def srnl_seq_forward(h: SrnlSeq, x, y, q=None, final_states=None, stream=None) -
 
 def srnl_seq_device_status(h: SrnlSeq) -> None:
     h._check(load_library().srnl_seq_device_status(h.handle), "srnl_seq_device_status")
+
+
+def srnl_seq_cap_count(h: SrnlSeq) -> int:
+    """Token updates of the last forward on which the hard clamp was active (synchronises)."""
+    v = ctypes.c_ulonglong(0)
+    h._check(load_library().srnl_seq_cap_count(h.handle, ctypes.byref(v)), "srnl_seq_cap_count")
+    return int(v.value)
 
 
 def srnl_seq_destroy(h: SrnlSeq) -> None:

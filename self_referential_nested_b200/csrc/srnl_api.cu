@@ -31,6 +31,7 @@ struct srnl_scan {
   void* x_stage = nullptr;  // staging for srnl_scan_forward_host
   void* y_stage = nullptr;
   int* dev_err = nullptr;   // device status word written by the scan kernel
+  unsigned long long* binds = nullptr;  // hard-clamp activations of the last forward
   size_t ws_bytes = 0;
   // optional stage timing: a ring of event sets, 4 events per forward
   std::vector<cudaEvent_t> ev;
@@ -64,7 +65,7 @@ size_t act_bytes(const srnl_scan_config& c) {
 }
 
 void free_all(srnl_scan* h) {
-  void* ptrs[] = {h->Wq, h->Wqb, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err};
+  void* ptrs[] = {h->Wq, h->Wqb, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err, h->binds};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->Wq = h->G = h->Mm = h->scales = nullptr;
@@ -72,6 +73,7 @@ void free_all(srnl_scan* h) {
   h->q = h->x_stage = h->y_stage = nullptr;
   h->yr = nullptr;
   h->dev_err = nullptr;
+  h->binds = nullptr;
 }
 
 srnl_status validate_config(const srnl_scan_config* c) {
@@ -90,6 +92,8 @@ srnl_status validate_config(const srnl_scan_config* c) {
   if ((c->act_dtype != SRNL_F32 && c->act_dtype != SRNL_BF16) ||
       (c->gen_dtype != SRNL_F32 && c->gen_dtype != SRNL_BF16))
     return fail(nullptr, SRNL_E_INVAL, "act_dtype and gen_dtype must be SRNL_F32 or SRNL_BF16");
+  if (c->injection_cap != SRNL_CAP_SOFT && c->injection_cap != SRNL_CAP_HARD)
+    return fail(nullptr, SRNL_E_INVAL, "injection_cap must be SRNL_CAP_SOFT or SRNL_CAP_HARD");
   const int64_t N = (int64_t)c->H * c->W;
   if (N > (int64_t)1 << 30) return fail(nullptr, SRNL_E_INVAL, "H*W too large");
   if ((int64_t)4 * c->B * c->heads > (int64_t)INT32_MAX)
@@ -152,6 +156,7 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
   g.alpha = c.alpha; g.eps = c.eps;
   g.act_bf16 = c.act_dtype == SRNL_BF16;
   g.gen_bf16 = c.gen_dtype == SRNL_BF16;
+  g.hard_cap = c.injection_cap == SRNL_CAP_HARD;
 
   // ---- pack parameters on the host, then upload
   std::vector<float> Wq((size_t)c.C * c.C);
@@ -179,7 +184,8 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
       {(void**)&h->Mm, n_mm * sizeof(float)},      {(void**)&h->scales, n_sc * sizeof(float)},
       {&h->q, q_bytes},                            {(void**)&h->yr, yr_bytes},
       {&h->x_stage, stage_bytes},                  {&h->y_stage, stage_bytes},
-      {(void**)&h->dev_err, sizeof(int)},          {&h->Wqb, Wqb.size() * sizeof(__nv_bfloat16)}};
+      {(void**)&h->dev_err, sizeof(int)},          {&h->Wqb, Wqb.size() * sizeof(__nv_bfloat16)},
+      {(void**)&h->binds, sizeof(unsigned long long)}};
   for (auto& a : allocs) {
     if (a.n == 0) continue;
     e = cudaMalloc(a.p, a.n);
@@ -199,6 +205,7 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
     if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemcpy (params)"); free_all(h); delete h; return st; }
   }
   e = cudaMemset(h->dev_err, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(h->binds, 0, sizeof(unsigned long long));
   if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemset (status)"); free_all(h); delete h; return st; }
   e = srnl::prepare_kernels();
   if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "kernel attributes"); free_all(h); delete h; return st; }
@@ -214,7 +221,9 @@ static srnl_status run_forward(srnl_scan* h, const void* x, void* y, float* fina
   e = srnl::launch_query_projection(h->geom, p, x, h->q, h->dev_err, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
-  e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, finals, h->dev_err, s);
+  if (h->geom.hard_cap && (e = cudaMemsetAsync(h->binds, 0, sizeof(unsigned long long), s)) != cudaSuccess)
+    return cuda_fail(h, e, "counter reset");
+  e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, finals, h->dev_err, h->binds, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "scan launch");
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   e = srnl::launch_fuse(h->geom, h->yr, y, s);
@@ -346,6 +355,14 @@ srnl_status srnl_scan_device_status(srnl_scan* h) {
   cudaError_t e = cudaMemcpy(&v, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(h, e, "status read");
   if (v != 0) return fail(h, static_cast<srnl_status>(v), "a bounded in-kernel wait gave up");
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_cap_count(srnl_scan* h, unsigned long long* count) {
+  if (h == nullptr || count == nullptr) return SRNL_E_INVAL;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(count, h->binds, sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "counter read");
   return SRNL_OK;
 }
 

@@ -13,6 +13,7 @@ struct ScanGeom {
   float alpha, eps;
   bool act_bf16;     // x / y element type
   bool gen_bf16;     // generation + projection operands in bf16
+  bool hard_cap = false;  // hard injection clamp instead of the soft cap
 };
 
 struct ScanParamsDev {
@@ -35,8 +36,9 @@ cudaError_t launch_query_projection_tc(const ScanGeom& g, const ScanParamsDev& p
 // Route partials yr[4][B*N][C] (fp32, already scaled by the fusion scales),
 // optional final states.
 // `err` (device int) receives SRNL_E_TIMEOUT if a bounded in-kernel wait gives up.
+// `binds` (device counter or nullptr) accumulates the tokens on which the hard clamp acts.
 cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
-                        float* yr, float* finals, int* err, cudaStream_t s);
+                        float* yr, float* finals, int* err, unsigned long long* binds, cudaStream_t s);
 
 // y = yr[0] + ... + yr[routes - 1] in act dtype, summed in route order.
 cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_t s);
@@ -48,7 +50,8 @@ cudaError_t launch_gather(const ScanGeom& g, int route, const void* x, void* xr,
 
 // The chunkwise tensor-core scan (bf16 generation); launch_scan dispatches to it.
 cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
-                                  float* yr, float* finals, int* err, cudaStream_t s);
+                                  float* yr, float* finals, int* err, unsigned long long* binds,
+                                  cudaStream_t s);
 
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)
 cudaError_t prepare_scan_kernels();

@@ -170,9 +170,10 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   g.Lcol = cfg->chunk_col > 0 ? cfg->chunk_col : cfg->H;
   g.alpha = cfg->alpha; g.eps = cfg->eps;
   g.act_bf16 = act_bf16; g.gen_bf16 = gen_bf16;
+  g.hard_cap = cfg->injection_cap == SRNL_CAP_HARD;
   const srnl::ScanParamsDev dp{Wq, Wqb, G, p->M_mem0, p->scales};
   if (e == cudaSuccess) e = srnl::launch_query_projection(g, dp, x, q, dev_err, cs);
-  if (e == cudaSuccess) e = srnl::launch_scan(g, dp, x, q, yr, nullptr, dev_err, cs);
+  if (e == cudaSuccess) e = srnl::launch_scan(g, dp, x, q, yr, nullptr, dev_err, nullptr, cs);
   if (e == cudaSuccess) e = srnl::launch_fuse(g, yr, y, cs);
   if (e != cudaSuccess) {
     srnl::set_thread_error(std::string("no-allocation forward launch: ") + cudaGetErrorString(e));

@@ -88,12 +88,14 @@ struct Args {
   float* yr;
   float* finals;
   int* err;
+  unsigned long long* binds;  // hard-clamp activations (nullptr: not counted)
   const float* G;
   const float* Mm;
   const float* scales;
   int B, H, W, C, heads, Lrow, Lcol;
   float alpha, eps;
   bool act_bf16;  // q is fp32 on this path
+  bool hard_cap;
 };
 
 // Token warps: asynchronous copies of a stage's q (fp32) and x (source dtype) head slices.
@@ -245,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_sequential_kernel(const
         for (int tt = tid >> 6; tt < T; tt += kThreads / 64) sm.simt.gen[tt][m] = dot32(grow, sm.simt.w[tt]);
       }
       __syncthreads();
+      bool binds = false;
       if (is_tok && gt < T) {
         float kt[kD], vv[kD], ga = 0.f, gb = 0.f;
         const float* wt = sm.simt.w[gt];
@@ -256,11 +259,12 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_sequential_kernel(const
           gb = fmaf(Gsrc[2 * kD * kD + kD + i], wt[i], gb);
         }
         float al, eta;
-        gates_row(kt, vv, ga, gb, a.alpha, a.eps, al, eta);
+        binds = gates_row(kt, vv, ga, gb, a.alpha, a.eps, al, eta, a.hard_cap);
         store_row(sm.k[gt], kt);
         store_row(sm.u[gt], vv);
         sm.ae[gt] = make_float4(al, eta, 0.f, 0.f);
       }
+      if (is_tok && a.hard_cap) count_binds(binds, a.binds);
     }
     if (is_tok && T > 0) {
       tok_bar();
@@ -412,14 +416,15 @@ cudaError_t prepare_scan_kernels() {
 }
 
 cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
-                        float* yr, float* finals, int* err, cudaStream_t s) {
-  if (g.gen_bf16) return launch_scan_chunkwise(g, p, x, q, yr, finals, err, s);
+                        float* yr, float* finals, int* err, unsigned long long* binds, cudaStream_t s) {
+  if (g.gen_bf16) return launch_scan_chunkwise(g, p, x, q, yr, finals, err, binds, s);
   Args a;
   a.x = x; a.q = q; a.yr = yr; a.finals = finals; a.err = err;
   a.G = p.G; a.Mm = p.Mm; a.scales = p.scales;
   a.B = g.B; a.H = g.H; a.W = g.W; a.C = g.C; a.heads = g.heads;
   a.Lrow = g.Lrow; a.Lcol = g.Lcol; a.alpha = g.alpha; a.eps = g.eps;
   a.act_bf16 = g.act_bf16;
+  a.hard_cap = g.hard_cap; a.binds = binds;
   const unsigned nseq = (unsigned)g.routes * (unsigned)g.B * (unsigned)g.heads;
   srnl_scan_sequential_kernel<<<nseq, kThreads, sizeof(Smem), s>>>(a);
   return cudaGetLastError();

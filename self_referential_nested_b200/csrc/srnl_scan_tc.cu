@@ -114,12 +114,14 @@ struct TcArgs {
   float* yr;
   float* finals;
   int* err;
+  unsigned long long* binds;  // hard-clamp activations (nullptr: not counted)
   const float* G;
   const float* Mm;
   const float* scales;
   int B, H, W, C, heads, Lrow, Lcol;
   float alpha, eps;
   bool act_bf16;
+  bool hard_cap;
 };
 
 // -A[t][j] for j in [16p, 16p + 16) lives in the first 4 KB of a1h, a1l, b1h, b1l
@@ -418,14 +420,16 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         const float nk = (nk0 + nk1) + o.x, kv = (kv0 + kv1) + o.y, nv = (nv0 + nv1) + o.z;
         const bool live = t < T;
         float l2a = 0.f, et = 0.f, al = 1.f, inv = 0.f;
+        bool binds = false;
         if (live) {
           inv = rsqrtf(nk + a.eps);
           // ||k||^2 and ||k - v||^2 of the stabilized key k = inv k~
           const float kn2 = nk * inv * inv;
           const float dk2 = fmaxf(fmaf(inv, fmaf(-2.f, kv, inv * nk), nv), 0.f);
-          gate_scalars(kn2, dk2, ga, gbeta, a.alpha, al, et);
+          binds = gate_scalars(kn2, dk2, ga, gbeta, a.alpha, al, et, a.hard_cap);
           l2a = fmaxf(log2f(al), -126.f);  // a retention that underflows acts as 2^-126
         }
+        if (a.hard_cap) count_binds(binds, a.binds);
         sm.eta[t] = et;
         // inclusive prefix of log2 alpha over the stage
         float pre = l2a;
@@ -760,13 +764,15 @@ cudaError_t prepare_scan_chunkwise_kernel() {
 }
 
 cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
-                                  float* yr, float* finals, int* err, cudaStream_t s) {
+                                  float* yr, float* finals, int* err, unsigned long long* binds,
+                                  cudaStream_t s) {
   TcArgs a;
   a.x = x; a.q = static_cast<const __nv_bfloat16*>(q); a.yr = yr; a.finals = finals; a.err = err;
   a.G = p.G; a.Mm = p.Mm; a.scales = p.scales;
   a.B = g.B; a.H = g.H; a.W = g.W; a.C = g.C; a.heads = g.heads;
   a.Lrow = g.Lrow; a.Lcol = g.Lcol; a.alpha = g.alpha; a.eps = g.eps;
   a.act_bf16 = g.act_bf16;
+  a.hard_cap = g.hard_cap; a.binds = binds;
   const unsigned nseq = (unsigned)g.routes * (unsigned)g.B * (unsigned)g.heads;
   srnl_scan_chunkwise_kernel<<<nseq, kThreadsTc, sizeof(TcSmem), s>>>(a);
   return cudaGetLastError();

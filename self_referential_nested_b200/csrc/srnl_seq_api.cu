@@ -30,6 +30,7 @@ struct srnl_seq {
   void* qbuf = nullptr;     // queries in the generation dtype when it differs from act_dtype
   float* yr = nullptr;      // [1][B*T][D] fp32 partial
   int* dev_err = nullptr;
+  unsigned long long* binds = nullptr;  // hard-clamp activations of the last forward
   std::string err;
 };
 
@@ -48,12 +49,13 @@ srnl_status seq_cuda_fail(srnl_seq* h, cudaError_t e, const char* what) {
 }
 
 void seq_free(srnl_seq* h) {
-  void* ptrs[] = {h->G, h->Mm, h->scales, h->qbuf, h->yr, h->dev_err};
+  void* ptrs[] = {h->G, h->Mm, h->scales, h->qbuf, h->yr, h->dev_err, h->binds};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->G = h->Mm = h->scales = h->yr = nullptr;
   h->qbuf = nullptr;
   h->dev_err = nullptr;
+  h->binds = nullptr;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -83,6 +85,7 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
   sc.alpha = cfg->alpha; sc.eps = cfg->eps;
   sc.chunk_row = sc.chunk_col = cfg->chunk > 0 ? cfg->chunk : 64;
   sc.act_dtype = cfg->act_dtype; sc.gen_dtype = cfg->gen_dtype;
+  sc.injection_cap = cfg->injection_cap;
   srnl_status st = srnl::validate_scan_config(&sc);
   if (st != SRNL_OK) {
     return seq_fail(nullptr, st, std::string("invalid sequence config: ") + srnl_scan_last_error(nullptr));
@@ -101,6 +104,7 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
   g.act_bf16 = cfg->act_dtype == SRNL_BF16;
   g.gen_bf16 = cfg->gen_dtype == SRNL_BF16;
   g.routes = 1;
+  g.hard_cap = cfg->injection_cap == SRNL_CAP_HARD;
 
   std::vector<float> G((size_t)nh * srnl::kGen * d);
   for (int hh = 0; hh < nh; ++hh) {
@@ -117,7 +121,8 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
   struct { void** p; size_t n; } allocs[] = {
       {(void**)&h->G, G.size() * sizeof(float)}, {(void**)&h->Mm, n_mm * sizeof(float)},
       {(void**)&h->scales, ones.size() * sizeof(float)}, {&h->qbuf, qbuf_bytes},
-      {(void**)&h->yr, tokens * cfg->D * sizeof(float)}, {(void**)&h->dev_err, sizeof(int)}};
+      {(void**)&h->yr, tokens * cfg->D * sizeof(float)}, {(void**)&h->dev_err, sizeof(int)},
+      {(void**)&h->binds, sizeof(unsigned long long)}};
   for (auto& a : allocs) {
     if (a.n == 0) continue;
     e = cudaMalloc(a.p, a.n);
@@ -131,6 +136,7 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
     if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "cudaMemcpy (params)"); seq_free(h); delete h; return st; }
   }
   e = cudaMemset(h->dev_err, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(h->binds, 0, sizeof(unsigned long long));
   if (e == cudaSuccess) e = srnl::prepare_kernels();
   if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "set-up"); seq_free(h); delete h; return st; }
   *out = h;
@@ -162,7 +168,9 @@ srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
     qk = h->qbuf;
   }
   const srnl::ScanParamsDev p{nullptr, nullptr, h->G, h->Mm, h->scales};
-  e = srnl::launch_scan(g, p, x, qk, h->yr, final_states, h->dev_err, s);
+  if (g.hard_cap && (e = cudaMemsetAsync(h->binds, 0, sizeof(unsigned long long), s)) != cudaSuccess)
+    return seq_cuda_fail(h, e, "counter reset");
+  e = srnl::launch_scan(g, p, x, qk, h->yr, final_states, h->dev_err, h->binds, s);
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "scan launch");
   e = srnl::launch_fuse(g, h->yr, y, s);
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "output launch");
@@ -178,6 +186,14 @@ srnl_status srnl_seq_device_status(srnl_seq* h) {
     h->err = "a bounded in-kernel wait gave up";
     return static_cast<srnl_status>(v);
   }
+  return SRNL_OK;
+}
+
+srnl_status srnl_seq_cap_count(srnl_seq* h, unsigned long long* count) {
+  if (h == nullptr || count == nullptr) return SRNL_E_INVAL;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(count, h->binds, sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "counter read");
   return SRNL_OK;
 }
 

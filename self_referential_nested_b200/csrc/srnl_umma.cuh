@@ -144,24 +144,32 @@ __device__ __forceinline__ float quad_sum(float v) {
 }
 
 // Gate scalars of one token from ||k||^2 (stabilized key), ||k - v||^2, a and beta:
-// retention clamp, softplus step, soft injection cap, spectral clamp.
-__device__ __forceinline__ void gate_scalars(float kn2, float dk2, float a, float beta, float alpha_max,
-                                             float& al, float& eta) {
+// retention clamp, softplus step, injection cap (soft, or the hard clamp), spectral clamp.
+// Returns whether the hard clamp is active (eta0 g > 1 - alpha_t); false for the soft cap.
+__device__ __forceinline__ bool gate_scalars(float kn2, float dk2, float a, float beta, float alpha_max,
+                                             float& al, float& eta, bool hard) {
   const float gain = sqrtf(dk2 * kn2);
   const float eb = __expf(-fabsf(beta));  // sigmoid without overflow
   const float sg = (beta >= 0.f) ? __fdividef(1.f, 1.f + eb) : __fdividef(eb, 1.f + eb);
   al = fminf(sg, alpha_max);
   const float eta0 = fmaxf(a, 0.f) + log1pf(__expf(-fabsf(a)));
-  const float zc = __fdividef(eta0 * gain, 1.f - al);
-  const float phi = (zc < 1e-4f) ? (1.f - zc * zc * (1.f / 3.f)) : __fdividef(tanhf(zc), zc);
-  eta = eta0 * phi;
+  bool binds = false;
+  if (hard) {
+    binds = eta0 * gain > 1.f - al;
+    eta = binds ? __fdividef(1.f - al, gain) : eta0;
+  } else {
+    const float zc = __fdividef(eta0 * gain, 1.f - al);
+    const float phi = (zc < 1e-4f) ? (1.f - zc * zc * (1.f / 3.f)) : __fdividef(tanhf(zc), zc);
+    eta = eta0 * phi;
+  }
   if (eta * kn2 > 2.f) eta = __fdividef(2.f, kn2);
+  return binds;
 }
 
 // Gates of one token from its generated row (k~[32], v[32], a, beta): kt becomes the
 // stabilized key and vv becomes u.
-__device__ __forceinline__ void gates_row(float (&kt)[kD], float (&vv)[kD], float a, float beta,
-                                          float alpha_max, float eps, float& al, float& eta) {
+__device__ __forceinline__ bool gates_row(float (&kt)[kD], float (&vv)[kD], float a, float beta,
+                                          float alpha_max, float eps, float& al, float& eta, bool hard) {
   float n0 = 0.f, n1 = 0.f, n2 = 0.f, n3 = 0.f;
 #pragma unroll
   for (int i = 0; i < kD; i += 4) {
@@ -183,9 +191,16 @@ __device__ __forceinline__ void gates_row(float (&kt)[kD], float (&vv)[kD], floa
     d0 = fmaf(da, da, d0);
     d1 = fmaf(db, db, d1);
   }
-  gate_scalars(k0 + k1, d0 + d1, a, beta, alpha_max, al, eta);
+  const bool binds = gate_scalars(k0 + k1, d0 + d1, a, beta, alpha_max, al, eta, hard);
 #pragma unroll
   for (int i = 0; i < kD; ++i) vv[i] = (1.f + al) * kt[i] - vv[i];
+  return binds;
+}
+
+// Warp-wide count of active hard clamps, one atomic per warp (all lanes call it).
+__device__ __forceinline__ void count_binds(bool binds, unsigned long long* counter) {
+  const unsigned m = __ballot_sync(0xffffffffu, binds);
+  if (counter != nullptr && (threadIdx.x & 31) == 0 && m != 0u) atomicAdd(counter, (unsigned long long)__popc(m));
 }
 
 __device__ __forceinline__ void store_row(float* dst, const float (&v)[kD]) {

@@ -130,3 +130,17 @@ def test_seq_null_handle_calls_fail_cleanly(lib):
     assert lib.srnl_seq_device_status(None) == S.SRNL_E_INVAL
     lib.srnl_seq_destroy(None)
     assert isinstance(lib.srnl_seq_last_error(None), bytes)
+
+
+def test_create_rejects_bad_injection_cap(lib):
+    inp = make_inputs(CONFIGS["pr1_8x8"])
+    with pytest.raises(S.SrnlError) as e:
+        S.srnl_scan_create(_cfg_dict(inp.cfg, injection_cap=3), inp.params())
+    assert e.value.status == S.SRNL_E_INVAL
+    from srnl_inputs import make_seq_inputs
+    sinp = make_seq_inputs(1, 4, 64, 2)
+    with pytest.raises(S.SrnlError) as e:
+        S.srnl_seq_create(_seq_cfg(injection_cap=-1), sinp.params())
+    assert e.value.status == S.SRNL_E_INVAL
+    assert lib.srnl_scan_cap_count(None, None) == S.SRNL_E_INVAL
+    assert lib.srnl_seq_cap_count(None, None) == S.SRNL_E_INVAL
