@@ -190,6 +190,23 @@ def run_reference(args, cfg, rank, world):
 
 
 # ----------------------------------------------------------------- GPU arm
+def max_over_ranks(values, world, device=None):
+    """Each value's maximum over the ranks: a replica job takes as long as its slowest rank.
+    Every rank calls it (one all-reduce), with the same number of values."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def whole_job_rate(world, units_per_step, steps, total_ms):
+    """Units all ranks processed (each rank runs the whole workload) over the job's time."""
+    return world * units_per_step * steps / (total_ms * 1e-3)
+
+
 def stages_per_sequence(cfg, stage=64):
     """Dependent stages of the longest route: chunks x ceil(chunk / stage)."""
     n = 0
@@ -292,10 +309,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     clocks.stop()
     e2e_ms = e2e_s.elapsed_time(e2e_e)
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
     h.close()
     if rank != 0:
         return
@@ -305,8 +319,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     wm = work_model(cfg)
     peaks = load_peaks()
     ms_step = total_ms / args.steps
-    value = world * wm["route_tokens"] * args.steps / (total_ms * 1e-3)
-    e2e_value = world * wm["route_tokens"] * args.steps / (e2e_ms * 1e-3)
+    value = whole_job_rate(world, wm["route_tokens"], args.steps, total_ms)
+    e2e_value = whole_job_rate(world, wm["route_tokens"], args.steps, e2e_ms)
     stage_ms = np.asarray(stage)
     scan_ms = float(stage_ms[1])
     # dominant kernel: the scan.  Its algorithmic work is the fp32 recurrence (sequential-form
