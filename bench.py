@@ -251,7 +251,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     inp = make_inputs(cfg, seed=rank)
     cfgd = dict(B=cfg.B, H=cfg.H, W=cfg.W, C=cfg.C, heads=cfg.heads, d=cfg.d, alpha=cfg.alpha,
                 eps=cfg.eps, chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, act_dtype=act,
-                gen_dtype=gen)
+                gen_dtype=gen, injection_cap=args.cap)
     h = S.srnl_scan_create(cfgd, inp.params())
     if act == "bf16":
         x = torch.from_numpy(inp.x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -310,6 +310,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     e2e_ms = e2e_s.elapsed_time(e2e_e)
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
+    cap_active = S.srnl_scan_cap_count(h) if args.cap == "hard" else 0
     h.close()
     if rank != 0:
         return
@@ -354,6 +355,9 @@ def run_ours(args, cfg, rank, world, local_rank):
                                 "hbm_bytes": wm["hbm_bytes"], "tensor_flops": wm["gen_flops"] + wm["qproj_flops"],
                                 "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TF/s bf16"},
         "stage_ms": {"query_projection": float(stage_ms[0]), "scan": scan_ms, "fusion": float(stage_ms[2])},
+        "injection_cap": {"mode": args.cap,
+                          "active_frac": cap_active / (4.0 * cfg.B * cfg.H * cfg.W * cfg.heads)
+                          if args.cap == "hard" else None},
         "chain": {"stages_per_sequence": n_stages, "one_image_scan_us": chain_ms * 1e3,
                   "per_stage_us": chain_ms * 1e3 / n_stages, "scan_us": scan_ms * 1e3,
                   "frac": chain_ms / scan_ms,
@@ -424,6 +428,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--gen", default=None, choices=[None, "f32", "bf16"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cap", default="soft", choices=["soft", "hard"],
+                    help="injection cap: the soft cap (the method) or the hard clamp of its ablation")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
     ap.add_argument("--seq", action="store_true", help="time the standalone sequence layer instead")
     ap.add_argument("--seq-batch", type=int, default=128)
