@@ -99,7 +99,8 @@ typedef enum { SRNL_CAP_SOFT = 0, SRNL_CAP_HARD = 1 } srnl_cap;
 
 typedef struct {
   int B, H, W, C; /* batch, height, width, channels (C = heads * d) */
-  int heads, d;   /* heads and head dim; d = 32 is built */
+  int heads, d;   /* heads and head dim: 4, 8, 16 or 32 (below 32 the heads run zero-padded
+                     to 32 lanes, which is exact; the no-allocation forward takes 32 only) */
   float alpha;    /* retention cap, 0 < alpha < 1 (0.95 hierarchical, 0.9 plain) */
   float eps;      /* key normalisation epsilon, > 0 (1e-6) */
   int chunk_row;  /* chunk length on routes 0/1; 0 means W (full rows) */
@@ -236,7 +237,8 @@ typedef struct srnl_seq srnl_seq; /* opaque; owned by the library */
 
 typedef struct {
   int B, T, D;    /* batch, tokens, dim (D = heads * d) */
-  int heads, d;   /* heads and head dim; d = 32 is built */
+  int heads, d;   /* heads and head dim: 4, 8, 16 or 32 (below 32 the heads run zero-padded
+                     to 32 lanes, which is exact; the no-allocation forward takes 32 only) */
   float alpha;    /* retention cap, 0 < alpha < 1 */
   float eps;      /* key normalisation epsilon, > 0 */
   int chunk;      /* chunk length; 0 means 64 */

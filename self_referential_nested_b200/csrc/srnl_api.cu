@@ -32,6 +32,10 @@ struct srnl_scan {
   void* y_stage = nullptr;
   int* dev_err = nullptr;   // device status word written by the scan kernel
   unsigned long long* binds = nullptr;  // hard-clamp activations of the last forward
+  // head dims below 32 run zero-padded to 32: padded copies of x, y and the final states
+  void* x_pad = nullptr;
+  void* y_pad = nullptr;
+  float* fin_pad = nullptr;
   size_t ws_bytes = 0;
   // optional stage timing: a ring of event sets, 4 events per forward
   std::vector<cudaEvent_t> ev;
@@ -65,7 +69,8 @@ size_t act_bytes(const srnl_scan_config& c) {
 }
 
 void free_all(srnl_scan* h) {
-  void* ptrs[] = {h->Wq, h->Wqb, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err, h->binds};
+  void* ptrs[] = {h->Wq, h->Wqb, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err, h->binds,
+                  h->x_pad, h->y_pad, h->fin_pad};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->Wq = h->G = h->Mm = h->scales = nullptr;
@@ -74,6 +79,8 @@ void free_all(srnl_scan* h) {
   h->yr = nullptr;
   h->dev_err = nullptr;
   h->binds = nullptr;
+  h->x_pad = h->y_pad = nullptr;
+  h->fin_pad = nullptr;
 }
 
 srnl_status validate_config(const srnl_scan_config* c) {
@@ -81,8 +88,8 @@ srnl_status validate_config(const srnl_scan_config* c) {
     return fail(nullptr, SRNL_E_INVAL, "B, H, W, C, heads and d must be positive");
   if ((int64_t)c->heads * c->d != c->C)
     return fail(nullptr, SRNL_E_INVAL, "C must equal heads * d");
-  if (c->d != srnl::kD)
-    return fail(nullptr, SRNL_E_UNSUPPORTED, "only head dim d = 32 is built");
+  if (c->d != 4 && c->d != 8 && c->d != 16 && c->d != srnl::kD)
+    return fail(nullptr, SRNL_E_UNSUPPORTED, "head dim d must be 4, 8, 16 or 32");
   if (!(c->alpha > 0.f && c->alpha < 1.f))
     return fail(nullptr, SRNL_E_INVAL, "alpha must lie in (0, 1)");
   if (!(c->eps > 0.f) || !std::isfinite(c->eps))
@@ -148,9 +155,12 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
   if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaGetDevice"); delete h; return st; }
 
   const srnl_scan_config& c = h->cfg;
-  const int d = srnl::kD, nh = c.heads;
+  // kernels run 32-wide heads; a smaller head dim is zero-padded to 32 (exact: the padded
+  // rows and columns of every memory and transition stay zero)
+  const int d = srnl::kD, ud = c.d, nh = c.heads, Cp = nh * d;
+  const bool padded = ud != d;
   srnl::ScanGeom& g = h->geom;
-  g.B = c.B; g.H = c.H; g.W = c.W; g.C = c.C; g.heads = nh;
+  g.B = c.B; g.H = c.H; g.W = c.W; g.C = Cp; g.heads = nh;
   g.Lrow = c.chunk_row > 0 ? c.chunk_row : c.W;
   g.Lcol = c.chunk_col > 0 ? c.chunk_col : c.H;
   g.alpha = c.alpha; g.eps = c.eps;
@@ -159,25 +169,40 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
   g.hard_cap = c.injection_cap == SRNL_CAP_HARD;
 
   // ---- pack parameters on the host, then upload
-  std::vector<float> Wq((size_t)c.C * c.C);
-  for (size_t i = 0; i < Wq.size(); ++i) Wq[i] = g.gen_bf16 ? bf16_round_host(prm->W_q[i]) : prm->W_q[i];
+  std::vector<float> Wq((size_t)Cp * Cp, 0.f);
+  for (int o = 0; o < c.C; ++o)
+    for (int i = 0; i < c.C; ++i) {
+      const float w = prm->W_q[(size_t)o * c.C + i];
+      Wq[(size_t)((o / ud) * d + o % ud) * Cp + (i / ud) * d + i % ud] = g.gen_bf16 ? bf16_round_host(w) : w;
+    }
   std::vector<__nv_bfloat16> Wqb(g.gen_bf16 ? Wq.size() : 0);
   for (size_t i = 0; i < Wqb.size(); ++i) Wqb[i] = __float2bfloat16_rn(Wq[i]);  // exact: already rounded
-  std::vector<float> G((size_t)4 * nh * srnl::kGen * d);
+  std::vector<float> G((size_t)4 * nh * srnl::kGen * d, 0.f), Mm((size_t)4 * nh * d * d, 0.f);
   for (int r = 0; r < 4; ++r)
     for (int hh = 0; hh < nh; ++hh) {
       float* dst = G.data() + ((size_t)r * nh + hh) * srnl::kGen * d;
-      const size_t mo = ((size_t)r * nh + hh) * d * d, vo = ((size_t)r * nh + hh) * d;
-      std::memcpy(dst, prm->M_k0 + mo, sizeof(float) * d * d);
-      std::memcpy(dst + d * d, prm->M_v0 + mo, sizeof(float) * d * d);
-      std::memcpy(dst + 2 * d * d, prm->m_eta0 + vo, sizeof(float) * d);
-      std::memcpy(dst + 2 * d * d + d, prm->m_alpha0 + vo, sizeof(float) * d);
+      float* mdst = Mm.data() + ((size_t)r * nh + hh) * d * d;
+      const size_t mo = ((size_t)r * nh + hh) * ud * ud, vo = ((size_t)r * nh + hh) * ud;
+      for (int i = 0; i < ud; ++i) {
+        for (int j = 0; j < ud; ++j) {
+          dst[i * d + j] = prm->M_k0[mo + (size_t)i * ud + j];
+          dst[(d + i) * d + j] = prm->M_v0[mo + (size_t)i * ud + j];
+          mdst[i * d + j] = prm->M_mem0[mo + (size_t)i * ud + j];
+        }
+        dst[2 * d * d + i] = prm->m_eta0[vo + i];
+        dst[2 * d * d + d + i] = prm->m_alpha0[vo + i];
+      }
     }
-  const size_t n_mm = (size_t)4 * nh * d * d, n_sc = (size_t)4 * c.C;
+  std::vector<float> scales((size_t)4 * Cp, 0.f);
+  for (int r = 0; r < 4; ++r)
+    for (int ch = 0; ch < c.C; ++ch) scales[(size_t)r * Cp + (ch / ud) * d + ch % ud] = prm->scales[(size_t)r * c.C + ch];
+  const size_t n_mm = Mm.size(), n_sc = scales.size();
   const size_t tokens = (size_t)c.B * c.H * c.W;
-  const size_t q_bytes = tokens * c.C * (g.gen_bf16 ? 2 : 4);
-  const size_t yr_bytes = 4 * tokens * c.C * sizeof(float);
+  const size_t q_bytes = tokens * Cp * (g.gen_bf16 ? 2 : 4);
+  const size_t yr_bytes = 4 * tokens * Cp * sizeof(float);
   const size_t stage_bytes = act_bytes(c);
+  const size_t pad_bytes = padded ? tokens * Cp * (g.act_bf16 ? 2 : 4) : 0;
+  const size_t fin_pad_bytes = padded ? (size_t)4 * c.B * nh * srnl::kStateFloats * sizeof(float) : 0;
 
   struct { void** p; size_t n; } allocs[] = {
       {(void**)&h->Wq, Wq.size() * sizeof(float)}, {(void**)&h->G, G.size() * sizeof(float)},
@@ -185,7 +210,8 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
       {&h->q, q_bytes},                            {(void**)&h->yr, yr_bytes},
       {&h->x_stage, stage_bytes},                  {&h->y_stage, stage_bytes},
       {(void**)&h->dev_err, sizeof(int)},          {&h->Wqb, Wqb.size() * sizeof(__nv_bfloat16)},
-      {(void**)&h->binds, sizeof(unsigned long long)}};
+      {(void**)&h->binds, sizeof(unsigned long long)}, {&h->x_pad, pad_bytes}, {&h->y_pad, pad_bytes},
+      {(void**)&h->fin_pad, fin_pad_bytes}};
   for (auto& a : allocs) {
     if (a.n == 0) continue;
     e = cudaMalloc(a.p, a.n);
@@ -194,10 +220,10 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
       free_all(h); delete h; return st;
     }
   }
-  h->ws_bytes = q_bytes + yr_bytes + 2 * stage_bytes;
+  h->ws_bytes = q_bytes + yr_bytes + 2 * stage_bytes + 2 * pad_bytes + fin_pad_bytes;
   struct { void* dst; const void* src; size_t n; } copies[] = {
       {h->Wq, Wq.data(), Wq.size() * sizeof(float)}, {h->G, G.data(), G.size() * sizeof(float)},
-      {h->Mm, prm->M_mem0, n_mm * sizeof(float)},    {h->scales, prm->scales, n_sc * sizeof(float)},
+      {h->Mm, Mm.data(), n_mm * sizeof(float)},      {h->scales, scales.data(), n_sc * sizeof(float)},
       {h->Wqb, Wqb.data(), Wqb.size() * sizeof(__nv_bfloat16)}};
   for (auto& cp : copies) {
     if (cp.n == 0) continue;
@@ -218,16 +244,32 @@ static srnl_status run_forward(srnl_scan* h, const void* x, void* y, float* fina
   cudaError_t e;
   cudaEvent_t* ev = h->ring > 0 ? &h->ev[(size_t)(h->recorded % h->ring) * 4] : nullptr;
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
+  const bool padded = h->cfg.d != srnl::kD;
+  const int elt = h->geom.act_bf16 ? 2 : 4;
+  const int64_t tokens = (int64_t)h->geom.B * h->geom.H * h->geom.W;
+  if (padded) {  // heads of d < 32 channels run as zero-padded 32-wide heads
+    e = srnl::launch_pad_heads(x, h->x_pad, tokens, h->geom.heads, h->cfg.d, elt, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "head padding launch");
+    x = h->x_pad;
+  }
+  float* fk = padded && finals != nullptr ? h->fin_pad : finals;
+  void* yk = padded ? h->y_pad : y;
   e = srnl::launch_query_projection(h->geom, p, x, h->q, h->dev_err, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   if (h->geom.hard_cap && (e = cudaMemsetAsync(h->binds, 0, sizeof(unsigned long long), s)) != cudaSuccess)
     return cuda_fail(h, e, "counter reset");
-  e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, finals, h->dev_err, h->binds, s);
+  e = srnl::launch_scan(h->geom, p, x, h->q, h->yr, fk, h->dev_err, h->binds, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "scan launch");
   if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
-  e = srnl::launch_fuse(h->geom, h->yr, y, s);
+  e = srnl::launch_fuse(h->geom, h->yr, yk, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "fusion launch");
+  if (padded) {
+    e = srnl::launch_unpad_heads(h->y_pad, y, tokens, h->geom.heads, h->cfg.d, elt, s);
+    if (e == cudaSuccess && finals != nullptr)
+      e = srnl::launch_unpad_states(h->fin_pad, finals, (int64_t)4 * h->geom.B * h->geom.heads, h->cfg.d, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "head unpadding launch");
+  }
   if (ev) {
     if ((e = cudaEventRecord(ev[3], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
     ++h->recorded;
@@ -296,7 +338,9 @@ srnl_status srnl_scan_gather(const srnl_scan* hc, int route, const void* x, void
   if (x == nullptr || xr == nullptr) return fail(h, SRNL_E_INVAL, "x or xr is NULL");
   if (!aligned16(x) || !aligned16(xr)) return fail(h, SRNL_E_INVAL, "x and xr must be 16-byte aligned");
   if (route < 0 || route > 3) return fail(h, SRNL_E_INVAL, "route must be 0..3");
-  cudaError_t e = srnl::launch_gather(h->geom, route, x, xr, static_cast<cudaStream_t>(stream));
+  srnl::ScanGeom ug = h->geom;  // the caller's layout (C = heads * d)
+  ug.C = h->cfg.C;
+  cudaError_t e = srnl::launch_gather(ug, route, x, xr, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(h, e, "gather launch");
   return SRNL_OK;
 }

@@ -88,6 +88,42 @@ query_projection_kernel(const void* __restrict__ x, const float* __restrict__ Wq
 // Fusion epilogue: y = yr0 + yr1 + yr2 + yr3 (fixed order), 8 channels per
 // thread, 16-byte loads and stores.
 // ---------------------------------------------------------------------------
+// [n][heads][d] <-> [n][heads][32] element copies (zeros in the padded lanes).
+template <typename T>
+__global__ void pad_heads_kernel(const T* __restrict__ src, T* __restrict__ dst, int64_t n, int heads, int d) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over dst
+  if (i >= n * heads * kD) return;
+  const int j = (int)(i % kD);
+  const int64_t th = i / kD;  // token * heads + head
+  dst[i] = j < d ? src[th * d + j] : T(0);
+}
+
+template <typename T>
+__global__ void unpad_heads_kernel(const T* __restrict__ src, T* __restrict__ dst, int64_t n, int heads, int d) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over dst
+  if (i >= n * heads * d) return;
+  const int64_t th = i / d;
+  dst[i] = src[th * kD + (int)(i - th * d)];
+}
+
+__global__ void unpad_states_kernel(const float* __restrict__ src, float* __restrict__ dst, int64_t S, int d) {
+  const int per = 3 * d * d + 2 * d;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= S * per) return;
+  const int64_t sq = i / per;
+  const int e = (int)(i - sq * per);
+  const float* s = src + sq * kStateFloats;
+  int off;
+  if (e < 3 * d * d) {  // M_mem, M_k, M_v: top-left d x d of each 32 x 32
+    const int m = e / (d * d), rc = e - m * d * d;
+    off = m * kD * kD + (rc / d) * kD + rc % d;
+  } else {  // m_eta, m_alpha: first d of each 32
+    const int v = (e - 3 * d * d) / d, c = (e - 3 * d * d) % d;
+    off = 3 * kD * kD + v * kD + c;
+  }
+  dst[i] = s[off];
+}
+
 // Element-wise bf16 <-> fp32 conversion (fp32 -> bf16 rounds to nearest even).
 __global__ void convert_kernel(const void* __restrict__ src, bool src_bf16, void* __restrict__ dst, int64_t n) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -175,6 +211,34 @@ cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_
   const int64_t threads = total / 8;
   const int bs = 256;
   fuse_kernel<<<(unsigned)((threads + bs - 1) / bs), bs, 0, s>>>(yr, y, total, g.routes, g.act_bf16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pad_heads(const void* src, void* dst, int64_t n, int heads, int d, int elt, cudaStream_t s) {
+  const int64_t total = n * heads * kD;
+  const unsigned grid = (unsigned)((total + 255) / 256);
+  if (elt == 2)
+    pad_heads_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst),
+                                          n, heads, d);
+  else
+    pad_heads_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(src), static_cast<float*>(dst), n, heads, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpad_heads(const void* src, void* dst, int64_t n, int heads, int d, int elt, cudaStream_t s) {
+  const int64_t total = n * heads * d;
+  const unsigned grid = (unsigned)((total + 255) / 256);
+  if (elt == 2)
+    unpad_heads_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src),
+                                            static_cast<__nv_bfloat16*>(dst), n, heads, d);
+  else
+    unpad_heads_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(src), static_cast<float*>(dst), n, heads, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpad_states(const float* src, float* dst, int64_t S, int d, cudaStream_t s) {
+  const int64_t total = S * (3 * d * d + 2 * d);
+  unpad_states_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(src, dst, S, d);
   return cudaGetLastError();
 }
 

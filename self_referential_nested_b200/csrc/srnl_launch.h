@@ -44,6 +44,12 @@ cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x
 cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_t s);
 
 cudaError_t launch_route_index(int route, int H, int W, int32_t* out, cudaStream_t s);
+// Head dims below 32 run as zero-padded 32-wide heads (exact: the padded rows and columns of
+// every memory stay zero).  pad: [n][heads*d] -> [n][heads*32]; unpad: the reverse; states:
+// [S][3*32*32 + 2*32] -> [S][3*d*d + 2*d] (the top-left blocks).  elt: bytes per element.
+cudaError_t launch_pad_heads(const void* src, void* dst, int64_t n, int heads, int d, int elt, cudaStream_t s);
+cudaError_t launch_unpad_heads(const void* src, void* dst, int64_t n, int heads, int d, int elt, cudaStream_t s);
+cudaError_t launch_unpad_states(const float* src, float* dst, int64_t S, int d, cudaStream_t s);
 // dst[i] = src[i] converted between bf16 and fp32 (src_bf16: bf16 -> fp32, else fp32 -> bf16).
 cudaError_t launch_convert(const void* src, bool src_bf16, void* dst, int64_t n, cudaStream_t s);
 cudaError_t launch_gather(const ScanGeom& g, int route, const void* x, void* xr, cudaStream_t s);

@@ -111,6 +111,10 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   }
   srnl_status st = srnl::validate_scan_config(cfg);
   if (st != SRNL_OK) return st;
+  if (cfg->d != srnl::kD) {
+    srnl::set_thread_error("the no-allocation forward is built for head dim d = 32 only");
+    return SRNL_E_UNSUPPORTED;
+  }
   if (x == nullptr || y == nullptr) {
     srnl::set_thread_error("x or y is NULL");
     return SRNL_E_INVAL;

@@ -31,6 +31,11 @@ struct srnl_seq {
   float* yr = nullptr;      // [1][B*T][D] fp32 partial
   int* dev_err = nullptr;
   unsigned long long* binds = nullptr;  // hard-clamp activations of the last forward
+  // head dims below 32 run zero-padded to 32: padded copies of x, q, y and the final states
+  void* x_pad = nullptr;
+  void* q_pad = nullptr;
+  void* y_pad = nullptr;
+  float* fin_pad = nullptr;
   std::string err;
 };
 
@@ -49,13 +54,16 @@ srnl_status seq_cuda_fail(srnl_seq* h, cudaError_t e, const char* what) {
 }
 
 void seq_free(srnl_seq* h) {
-  void* ptrs[] = {h->G, h->Mm, h->scales, h->qbuf, h->yr, h->dev_err, h->binds};
+  void* ptrs[] = {h->G, h->Mm, h->scales, h->qbuf, h->yr, h->dev_err, h->binds, h->x_pad, h->q_pad, h->y_pad,
+                  h->fin_pad};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->G = h->Mm = h->scales = h->yr = nullptr;
   h->qbuf = nullptr;
   h->dev_err = nullptr;
   h->binds = nullptr;
+  h->x_pad = h->q_pad = h->y_pad = nullptr;
+  h->fin_pad = nullptr;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -96,9 +104,11 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
   cudaError_t e = cudaGetDevice(&h->device);
   if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "cudaGetDevice"); delete h; return st; }
 
-  const int d = srnl::kD, nh = cfg->heads;
+  // kernels run 32-wide heads; a smaller head dim is zero-padded to 32 (exact)
+  const int d = srnl::kD, ud = cfg->d, nh = cfg->heads, Dp = nh * d;
+  const bool padded = ud != d;
   srnl::ScanGeom& g = h->geom;
-  g.B = cfg->B; g.H = 1; g.W = cfg->T; g.C = cfg->D; g.heads = nh;
+  g.B = cfg->B; g.H = 1; g.W = cfg->T; g.C = Dp; g.heads = nh;
   g.Lrow = g.Lcol = sc.chunk_row;
   g.alpha = cfg->alpha; g.eps = cfg->eps;
   g.act_bf16 = cfg->act_dtype == SRNL_BF16;
@@ -106,30 +116,40 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
   g.routes = 1;
   g.hard_cap = cfg->injection_cap == SRNL_CAP_HARD;
 
-  std::vector<float> G((size_t)nh * srnl::kGen * d);
+  std::vector<float> G((size_t)nh * srnl::kGen * d, 0.f), Mm((size_t)nh * d * d, 0.f);
   for (int hh = 0; hh < nh; ++hh) {
     float* dst = G.data() + (size_t)hh * srnl::kGen * d;
-    std::memcpy(dst, prm->M_k0 + (size_t)hh * d * d, sizeof(float) * d * d);
-    std::memcpy(dst + d * d, prm->M_v0 + (size_t)hh * d * d, sizeof(float) * d * d);
-    std::memcpy(dst + 2 * d * d, prm->m_eta0 + (size_t)hh * d, sizeof(float) * d);
-    std::memcpy(dst + 2 * d * d + d, prm->m_alpha0 + (size_t)hh * d, sizeof(float) * d);
+    float* mdst = Mm.data() + (size_t)hh * d * d;
+    const size_t mo = (size_t)hh * ud * ud, vo = (size_t)hh * ud;
+    for (int i = 0; i < ud; ++i) {
+      for (int j = 0; j < ud; ++j) {
+        dst[i * d + j] = prm->M_k0[mo + (size_t)i * ud + j];
+        dst[(d + i) * d + j] = prm->M_v0[mo + (size_t)i * ud + j];
+        mdst[i * d + j] = prm->M_mem0[mo + (size_t)i * ud + j];
+      }
+      dst[2 * d * d + i] = prm->m_eta0[vo + i];
+      dst[2 * d * d + d + i] = prm->m_alpha0[vo + i];
+    }
   }
-  const std::vector<float> ones((size_t)cfg->D, 1.f);
+  const std::vector<float> ones((size_t)Dp, 1.f);
   const size_t tokens = (size_t)cfg->B * cfg->T;
-  const size_t n_mm = (size_t)nh * d * d;
-  const size_t qbuf_bytes = g.act_bf16 != g.gen_bf16 ? tokens * cfg->D * (g.gen_bf16 ? 2 : 4) : 0;
+  const size_t n_mm = Mm.size();
+  const size_t qbuf_bytes = g.act_bf16 != g.gen_bf16 ? tokens * Dp * (g.gen_bf16 ? 2 : 4) : 0;
+  const size_t pad_bytes = padded ? tokens * Dp * (g.act_bf16 ? 2 : 4) : 0;
+  const size_t fin_pad_bytes = padded ? (size_t)cfg->B * nh * srnl::kStateFloats * sizeof(float) : 0;
   struct { void** p; size_t n; } allocs[] = {
       {(void**)&h->G, G.size() * sizeof(float)}, {(void**)&h->Mm, n_mm * sizeof(float)},
       {(void**)&h->scales, ones.size() * sizeof(float)}, {&h->qbuf, qbuf_bytes},
-      {(void**)&h->yr, tokens * cfg->D * sizeof(float)}, {(void**)&h->dev_err, sizeof(int)},
-      {(void**)&h->binds, sizeof(unsigned long long)}};
+      {(void**)&h->yr, tokens * Dp * sizeof(float)}, {(void**)&h->dev_err, sizeof(int)},
+      {(void**)&h->binds, sizeof(unsigned long long)}, {&h->x_pad, pad_bytes}, {&h->q_pad, pad_bytes},
+      {&h->y_pad, pad_bytes}, {(void**)&h->fin_pad, fin_pad_bytes}};
   for (auto& a : allocs) {
     if (a.n == 0) continue;
     e = cudaMalloc(a.p, a.n);
     if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "cudaMalloc"); seq_free(h); delete h; return st; }
   }
   struct { void* dst; const void* src; size_t n; } copies[] = {
-      {h->G, G.data(), G.size() * sizeof(float)}, {h->Mm, prm->M_mem0, n_mm * sizeof(float)},
+      {h->G, G.data(), G.size() * sizeof(float)}, {h->Mm, Mm.data(), n_mm * sizeof(float)},
       {h->scales, ones.data(), ones.size() * sizeof(float)}};
   for (auto& cp : copies) {
     e = cudaMemcpy(cp.dst, cp.src, cp.n, cudaMemcpyHostToDevice);
@@ -152,8 +172,8 @@ srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
       (final_states != nullptr && !aligned16(final_states)))
     return seq_fail(h, SRNL_E_INVAL, "x, q, y and final_states must be 16-byte aligned");
   const srnl::ScanGeom& g = h->geom;
-  const size_t n = (size_t)g.B * g.W * g.C;
-  const size_t bytes = n * (g.act_bf16 ? 2 : 4);
+  const size_t n = (size_t)g.B * g.W * g.C;  // padded element count
+  const size_t bytes = (size_t)g.B * g.W * h->cfg.D * (g.act_bf16 ? 2 : 4);
   if (overlap(x, y, bytes) || (q != nullptr && overlap(q, y, bytes)))
     return seq_fail(h, SRNL_E_INVAL, "y overlaps x or q");
   int cur = -1;
@@ -161,7 +181,21 @@ srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "cudaGetDevice");
   if (cur != h->device) return seq_fail(h, SRNL_E_INVAL, "the current device is not the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool padded = h->cfg.d != srnl::kD;
+  const int elt = g.act_bf16 ? 2 : 4;
+  const int64_t tokens = (int64_t)g.B * g.W;
   const void* qk = q != nullptr ? q : x;
+  void* yk = y;
+  float* fk = final_states;
+  if (padded) {  // heads of d < 32 channels run as zero-padded 32-wide heads
+    e = srnl::launch_pad_heads(x, h->x_pad, tokens, g.heads, h->cfg.d, elt, s);
+    if (e == cudaSuccess && q != nullptr) e = srnl::launch_pad_heads(q, h->q_pad, tokens, g.heads, h->cfg.d, elt, s);
+    if (e != cudaSuccess) return seq_cuda_fail(h, e, "head padding launch");
+    qk = q != nullptr ? h->q_pad : h->x_pad;
+    x = h->x_pad;
+    yk = h->y_pad;
+    if (final_states != nullptr) fk = h->fin_pad;
+  }
   if (g.act_bf16 != g.gen_bf16) {  // queries in the generation dtype
     e = srnl::launch_convert(qk, g.act_bf16, h->qbuf, (int64_t)n, s);
     if (e != cudaSuccess) return seq_cuda_fail(h, e, "query conversion launch");
@@ -170,10 +204,16 @@ srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
   const srnl::ScanParamsDev p{nullptr, nullptr, h->G, h->Mm, h->scales};
   if (g.hard_cap && (e = cudaMemsetAsync(h->binds, 0, sizeof(unsigned long long), s)) != cudaSuccess)
     return seq_cuda_fail(h, e, "counter reset");
-  e = srnl::launch_scan(g, p, x, qk, h->yr, final_states, h->dev_err, h->binds, s);
+  e = srnl::launch_scan(g, p, x, qk, h->yr, fk, h->dev_err, h->binds, s);
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "scan launch");
-  e = srnl::launch_fuse(g, h->yr, y, s);
+  e = srnl::launch_fuse(g, h->yr, yk, s);
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "output launch");
+  if (padded) {
+    e = srnl::launch_unpad_heads(h->y_pad, y, tokens, g.heads, h->cfg.d, elt, s);
+    if (e == cudaSuccess && final_states != nullptr)
+      e = srnl::launch_unpad_states(h->fin_pad, final_states, (int64_t)g.B * g.heads, h->cfg.d, s);
+    if (e != cudaSuccess) return seq_cuda_fail(h, e, "head unpadding launch");
+  }
   return SRNL_OK;
 }
 
