@@ -194,6 +194,18 @@ SRNL_API srnl_status srnl_scan_gather(const srnl_scan* h, int route, const void*
 SRNL_API srnl_status srnl_scan_enable_stage_timing(srnl_scan* h, int n);
 SRNL_API srnl_status srnl_scan_stage_times(srnl_scan* h, float* ms_out, int* count);
 
+/* Pipelined forward with HOST buffers, for a loop of steps: copies x host->device on
+ * an internal copy stream, runs the forward on `stream`, copies y device->host on a
+ * second internal copy stream, and returns without waiting.  Two staging slots alternate,
+ * so one call's copies overlap the neighbouring calls' forwards.  x_host must stay
+ * unchanged and y_host unread until the copies are done: srnl_scan_host_sync(h) waits
+ * for them on the host, srnl_scan_host_join(h, stream) makes `stream` wait for them.
+ * Pinned host memory is needed for the copies to overlap. */
+SRNL_API srnl_status srnl_scan_forward_host_async(srnl_scan* h, const void* x_host, void* y_host,
+                                                 void* stream);
+SRNL_API srnl_status srnl_scan_host_join(srnl_scan* h, void* stream);
+SRNL_API srnl_status srnl_scan_host_sync(srnl_scan* h);
+
 /* Device status of the handle's kernels: synchronously reads the status word
  * the scan kernel sets when one of its bounded waits (for its own tensor-core
  * work) gives up.  Returns SRNL_OK, or SRNL_E_TIMEOUT once that has happened

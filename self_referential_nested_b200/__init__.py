@@ -32,7 +32,8 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_scan_workspace_bytes",
             "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy",
             "srnl_seq_create", "srnl_seq_forward", "srnl_seq_device_status", "srnl_seq_last_error",
-            "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count")
+            "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count",
+            "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync")
 
 
 class SrnlError(RuntimeError):
@@ -102,11 +103,15 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_seq_destroy.argtypes = [vp]
     lib.srnl_seq_destroy.restype = None
     lib.srnl_scan_cap_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.srnl_scan_forward_host_async.argtypes = [vp, vp, vp, vp]
+    lib.srnl_scan_host_join.argtypes = [vp, vp]
+    lib.srnl_scan_host_sync.argtypes = [vp]
     lib.srnl_seq_cap_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
                  "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_seq_create", "srnl_seq_forward",
-                 "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count"):
+                 "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count",
+                 "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -205,6 +210,20 @@ def srnl_scan_forward(h: SrnlScan, x, y, final_states=None, stream=None) -> None
 def srnl_scan_forward_host(h: SrnlScan, x_host, y_host, stream=None) -> None:
     st = load_library().srnl_scan_forward_host(h.handle, _ptr(x_host), _ptr(y_host), _stream(stream))
     h._check(st, "srnl_scan_forward_host")
+
+
+def srnl_scan_forward_host_async(h: SrnlScan, x_host, y_host, stream=None) -> None:
+    """Pipelined host-buffer forward (pinned tensors); y_host is ready after srnl_scan_host_sync."""
+    st = load_library().srnl_scan_forward_host_async(h.handle, _ptr(x_host), _ptr(y_host), _stream(stream))
+    h._check(st, "srnl_scan_forward_host_async")
+
+
+def srnl_scan_host_join(h: SrnlScan, stream=None) -> None:
+    h._check(load_library().srnl_scan_host_join(h.handle, _stream(stream)), "srnl_scan_host_join")
+
+
+def srnl_scan_host_sync(h: SrnlScan) -> None:
+    h._check(load_library().srnl_scan_host_sync(h.handle), "srnl_scan_host_sync")
 
 
 def srnl_scan_forward_noalloc(cfg: Dict, params_dev: Dict, x, y, stream=None) -> None:

@@ -28,8 +28,16 @@ struct srnl_scan {
   // workspace (device)
   void* q = nullptr;        // [B*N][C] fp32 or bf16
   float* yr = nullptr;      // [4][B*N][C] fp32 route partials
-  void* x_stage = nullptr;  // staging for srnl_scan_forward_host
+  void* x_stage = nullptr;  // staging for srnl_scan_forward_host (slot 0 of the pipeline)
   void* y_stage = nullptr;
+  // pipelined host-buffer forwards: a second staging slot, one copy stream per direction and
+  // the events that order slot reuse (created on first use)
+  void* x_stage1 = nullptr;
+  void* y_stage1 = nullptr;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t h2d_done[2] = {}, fwd_done[2] = {}, d2h_done[2] = {};
+  bool slot_used[2] = {false, false};
+  int slot = 0;
   int* dev_err = nullptr;   // device status word written by the scan kernel
   unsigned long long* binds = nullptr;  // hard-clamp activations of the last forward
   // head dims below 32 run zero-padded to 32: padded copies of x, y and the final states
@@ -70,7 +78,7 @@ size_t act_bytes(const srnl_scan_config& c) {
 
 void free_all(srnl_scan* h) {
   void* ptrs[] = {h->Wq, h->Wqb, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err, h->binds,
-                  h->x_pad, h->y_pad, h->fin_pad};
+                  h->x_pad, h->y_pad, h->fin_pad, h->x_stage1, h->y_stage1};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->Wq = h->G = h->Mm = h->scales = nullptr;
@@ -81,6 +89,14 @@ void free_all(srnl_scan* h) {
   h->binds = nullptr;
   h->x_pad = h->y_pad = nullptr;
   h->fin_pad = nullptr;
+  h->x_stage1 = h->y_stage1 = nullptr;
+  for (int k = 0; k < 2; ++k) {
+    cudaEvent_t* evs[] = {&h->h2d_done[k], &h->fwd_done[k], &h->d2h_done[k]};
+    for (cudaEvent_t* e : evs)
+      if (*e != nullptr) { cudaEventDestroy(*e); *e = nullptr; }
+  }
+  if (h->h2d != nullptr) { cudaStreamDestroy(h->h2d); h->h2d = nullptr; }
+  if (h->d2h != nullptr) { cudaStreamDestroy(h->d2h); h->d2h = nullptr; }
 }
 
 srnl_status validate_config(const srnl_scan_config* c) {
@@ -317,6 +333,75 @@ srnl_status srnl_scan_forward_host(srnl_scan* h, const void* x_host, void* y_hos
   if (e != cudaSuccess) return cuda_fail(h, e, "device-to-host copy");
   e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
+  return SRNL_OK;
+}
+
+static srnl_status pipeline_setup(srnl_scan* h) {
+  if (h->h2d != nullptr) return SRNL_OK;
+  const size_t n = act_bytes(h->cfg);
+  cudaError_t e = cudaMalloc(&h->x_stage1, n);
+  if (e == cudaSuccess) e = cudaMalloc(&h->y_stage1, n);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking);
+  for (int k = 0; k < 2 && e == cudaSuccess; ++k) {
+    cudaEvent_t* evs[] = {&h->h2d_done[k], &h->fwd_done[k], &h->d2h_done[k]};
+    for (cudaEvent_t* ev : evs)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  }
+  if (e != cudaSuccess) return cuda_fail(h, e, "pipeline set-up");
+  h->ws_bytes += 2 * n;
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_forward_host_async(srnl_scan* h, const void* x_host, void* y_host, void* stream) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (x_host == nullptr || y_host == nullptr) return fail(h, SRNL_E_INVAL, "x or y is NULL");
+  srnl_status st = check_device(h);
+  if (st != SRNL_OK) return st;
+  st = pipeline_setup(h);
+  if (st != SRNL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t n = act_bytes(h->cfg);
+  const int k = h->slot;
+  h->slot ^= 1;
+  void* xs = k == 0 ? h->x_stage : h->x_stage1;
+  void* ys = k == 0 ? h->y_stage : h->y_stage1;
+  cudaError_t e = cudaSuccess;
+  // the slot's x buffer is free once the forward that last read it has run
+  if (h->slot_used[k]) e = cudaStreamWaitEvent(h->h2d, h->fwd_done[k], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(xs, x_host, n, cudaMemcpyHostToDevice, h->h2d);
+  if (e == cudaSuccess) e = cudaEventRecord(h->h2d_done[k], h->h2d);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, h->h2d_done[k], 0);
+  // its y buffer is free once the copy that last read it is done
+  if (e == cudaSuccess && h->slot_used[k]) e = cudaStreamWaitEvent(s, h->d2h_done[k], 0);
+  if (e != cudaSuccess) return cuda_fail(h, e, "pipelined host-to-device copy");
+  st = run_forward(h, xs, ys, nullptr, s);
+  if (st != SRNL_OK) return st;
+  e = cudaEventRecord(h->fwd_done[k], s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->d2h, h->fwd_done[k], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(y_host, ys, n, cudaMemcpyDeviceToHost, h->d2h);
+  if (e == cudaSuccess) e = cudaEventRecord(h->d2h_done[k], h->d2h);
+  if (e != cudaSuccess) return cuda_fail(h, e, "pipelined device-to-host copy");
+  h->slot_used[k] = true;
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_host_join(srnl_scan* h, void* stream) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  for (int k = 0; k < 2; ++k)
+    if (h->slot_used[k]) {
+      const cudaError_t e = cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), h->d2h_done[k], 0);
+      if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamWaitEvent");
+    }
+  return SRNL_OK;
+}
+
+srnl_status srnl_scan_host_sync(srnl_scan* h) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  if (h->d2h == nullptr) return SRNL_OK;
+  const cudaError_t e = cudaStreamSynchronize(h->d2h);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamSynchronize");
   return SRNL_OK;
 }
 
