@@ -185,3 +185,17 @@ def make_seq_inputs(B: int, T: int, D: int, heads: int, act_dtype: str = F32, se
     return SeqInputs(B=B, T=T, D=D, heads=heads, act_dtype=act_dtype, x32=np.ascontiguousarray(x),
                      q32=np.ascontiguousarray(q), x_bits=x_bits, q_bits=q_bits, M_mem0=M_mem0, M_k0=M_k0,
                      M_v0=M_v0, m_eta0=m_eta0, m_alpha0=m_alpha0)
+
+
+# ------------------------------------------------ upstream gradients
+def make_cotangent(shape, seed: int = 0, act_dtype: str = F32) -> np.ndarray:
+    """Seeded upstream gradient dL/d(output) ~ N(0, 1) of the given shape (float32), drawn
+    from its own stream (``default_rng([seed, 1])``) so that it never shifts the draws of
+    ``make_inputs``.  For bf16 activations it is rounded to bfloat16 like x."""
+    rng = np.random.default_rng([seed, 1])
+    g = rng.standard_normal(tuple(shape), dtype=np.float32)
+    if act_dtype == BF16:
+        g = bf16_bits_to_f32(bf16_round_bits(g)).reshape(g.shape)
+    elif act_dtype != F32:
+        raise ValueError(f"unknown act_dtype {act_dtype!r}")
+    return np.ascontiguousarray(g)
