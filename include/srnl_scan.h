@@ -217,6 +217,38 @@ SRNL_API srnl_status srnl_scan_device_status(srnl_scan* h);
  * (srnl_scan_forward_noalloc does not count.) */
 SRNL_API srnl_status srnl_scan_cap_count(srnl_scan* h, unsigned long long* count);
 
+/* ------------------------------------------------------------------------
+ * Backward pass (reverse-mode gradient of the forward above; the layer is trained end to
+ * end inside the backbone: "VisionHOPE" README, "SRNL and VisionHOPE operator").
+ * For a loss L with upstream gradient dy = dL/dy, it returns dL/dx and the gradients of
+ * every parameter of srnl_scan_params, taking the active branch of each clamp (the
+ * retention clamp, the hard injection clamp, the spectral clamp).
+ *
+ * Gradient buffers: DEVICE pointers to dense fp32 arrays in the layouts of
+ * srnl_scan_params; each is OVERWRITTEN (not accumulated) and each may be NULL to skip it.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  float* W_q;      /* [C][C]            */
+  float* scales;   /* [4][C]            */
+  float* M_mem0;   /* [4][heads][d][d]  */
+  float* M_k0;     /* [4][heads][d][d]  */
+  float* M_v0;     /* [4][heads][d][d]  */
+  float* m_eta0;   /* [4][heads][d]     */
+  float* m_alpha0; /* [4][heads][d]     */
+} srnl_scan_grads;
+
+/* Backward pass.  x: the forward's input; dy: dL/dy; dx: receives dL/dx.  DEVICE
+ * pointers, 16-byte aligned, [B][H][W][C] of act_dtype; dx must not overlap x or dy.
+ * grads may be NULL (only dx).  The handle must have gen_dtype SRNL_F32 (otherwise
+ * SRNL_E_UNSUPPORTED): all arithmetic is fp32; act_dtype SRNL_BF16 means bf16 x, dy and dx.
+ * The forward is recomputed from x (boundary products are kept per chunk and the states
+ * inside a chunk recomputed), so no forward state is needed.  The first call allocates the
+ * backward workspace (cudaMalloc, synchronous; about 20 fp32 values per activation element
+ * plus 4 KB per chunk and per chunk token of every (route, batch, head) sequence); later calls
+ * reuse it.  Asynchronous on `stream`; shares the handle's workspace with the forward. */
+SRNL_API srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void* dx,
+                                       const srnl_scan_grads* grads, void* stream);
+
 /* Bytes of device workspace the handle holds (packed params excluded). */
 SRNL_API size_t srnl_scan_workspace_bytes(const srnl_scan* h);
 

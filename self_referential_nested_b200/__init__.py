@@ -33,7 +33,8 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_scan_last_error", "srnl_status_string", "srnl_scan_destroy",
             "srnl_seq_create", "srnl_seq_forward", "srnl_seq_device_status", "srnl_seq_last_error",
             "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count",
-            "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync")
+            "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
+            "srnl_scan_backward")
 
 
 class SrnlError(RuntimeError):
@@ -52,6 +53,14 @@ class _Config(ctypes.Structure):
 class _Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("W_q", "scales", "M_mem0", "M_k0", "M_v0",
                                                 "m_eta0", "m_alpha0")]
+
+
+class _Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W_q", "scales", "M_mem0", "M_k0", "M_v0",
+                                                "m_eta0", "m_alpha0")]
+
+
+GRAD_KEYS = ("W_q", "scales", "M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")
 
 
 class _SeqConfig(ctypes.Structure):
@@ -107,11 +116,13 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_scan_host_join.argtypes = [vp, vp]
     lib.srnl_scan_host_sync.argtypes = [vp]
     lib.srnl_seq_cap_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.srnl_scan_backward.argtypes = [vp, vp, vp, vp, ctypes.POINTER(_Grads), vp]
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
                  "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_seq_create", "srnl_seq_forward",
                  "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count",
-                 "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync"):
+                 "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
+                 "srnl_scan_backward"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -205,6 +216,17 @@ def srnl_scan_create(cfg: Dict, params: Dict[str, np.ndarray]) -> SrnlScan:
 def srnl_scan_forward(h: SrnlScan, x, y, final_states=None, stream=None) -> None:
     st = load_library().srnl_scan_forward(h.handle, _ptr(x), _ptr(y), _ptr(final_states), _stream(stream))
     h._check(st, "srnl_scan_forward")
+
+
+def srnl_scan_backward(h: SrnlScan, x, dy, dx, grads: Optional[Dict] = None, stream=None) -> None:
+    """Backward pass: dx <- dL/dx for upstream dy = dL/dy (CUDA tensors [B,H,W,C] of the handle's
+    act dtype); ``grads`` maps any of GRAD_KEYS to fp32 CUDA tensors in the parameter layouts,
+    which are overwritten with the parameter gradients (missing keys are skipped)."""
+    g = grads or {}
+    gs = _Grads(**{k: _ptr(g.get(k)) for k in GRAD_KEYS})
+    st = load_library().srnl_scan_backward(h.handle, _ptr(x), _ptr(dy), _ptr(dx),
+                                           ctypes.byref(gs) if grads is not None else None, _stream(stream))
+    h._check(st, "srnl_scan_backward")
 
 
 def srnl_scan_forward_host(h: SrnlScan, x_host, y_host, stream=None) -> None:

@@ -44,6 +44,10 @@ struct srnl_scan {
   void* x_pad = nullptr;
   void* y_pad = nullptr;
   float* fin_pad = nullptr;
+  // backward pass (allocated on first use): workspace and padded dy / dx for d < 32
+  float* bws = nullptr;
+  void* dy_pad = nullptr;
+  void* dx_pad = nullptr;
   size_t ws_bytes = 0;
   // optional stage timing: a ring of event sets, 4 events per forward
   std::vector<cudaEvent_t> ev;
@@ -78,7 +82,7 @@ size_t act_bytes(const srnl_scan_config& c) {
 
 void free_all(srnl_scan* h) {
   void* ptrs[] = {h->Wq, h->Wqb, h->G, h->Mm, h->scales, h->q, h->yr, h->x_stage, h->y_stage, h->dev_err, h->binds,
-                  h->x_pad, h->y_pad, h->fin_pad, h->x_stage1, h->y_stage1};
+                  h->x_pad, h->y_pad, h->fin_pad, h->x_stage1, h->y_stage1, h->bws, h->dy_pad, h->dx_pad};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->Wq = h->G = h->Mm = h->scales = nullptr;
@@ -90,6 +94,8 @@ void free_all(srnl_scan* h) {
   h->x_pad = h->y_pad = nullptr;
   h->fin_pad = nullptr;
   h->x_stage1 = h->y_stage1 = nullptr;
+  h->bws = nullptr;
+  h->dy_pad = h->dx_pad = nullptr;
   for (int k = 0; k < 2; ++k) {
     cudaEvent_t* evs[] = {&h->h2d_done[k], &h->fwd_done[k], &h->d2h_done[k]};
     for (cudaEvent_t* e : evs)
@@ -315,6 +321,70 @@ srnl_status srnl_scan_forward(srnl_scan* h, const void* x, void* y, float* final
   srnl_status st = check_device(h);
   if (st != SRNL_OK) return st;
   return run_forward(h, x, y, final_states, static_cast<cudaStream_t>(stream));
+}
+
+static bool overlaps(const void* a, const void* b, size_t n) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + n && pb < pa + n;
+}
+
+srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void* dx,
+                               const srnl_scan_grads* grads, void* stream) {
+  if (h == nullptr) return fail(nullptr, SRNL_E_INVAL, "handle is NULL");
+  h->err.clear();
+  if (x == nullptr || dy == nullptr || dx == nullptr) return fail(h, SRNL_E_INVAL, "x, dy or dx is NULL");
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx))
+    return fail(h, SRNL_E_INVAL, "x, dy and dx must be 16-byte aligned");
+  const size_t n = act_bytes(h->cfg);
+  if (overlaps(dx, x, n) || overlaps(dx, dy, n)) return fail(h, SRNL_E_INVAL, "dx overlaps x or dy");
+  if (h->geom.gen_bf16)
+    return fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for gen_dtype SRNL_F32 handles");
+  if (grads != nullptr) {
+    const float* gp[] = {grads->W_q, grads->scales, grads->M_mem0, grads->M_k0, grads->M_v0, grads->m_eta0,
+                         grads->m_alpha0};
+    for (const float* q : gp)
+      if ((reinterpret_cast<uintptr_t>(q) & 3u) != 0) return fail(h, SRNL_E_INVAL, "gradient buffers must be 4-byte aligned");
+  }
+  srnl_status st = check_device(h);
+  if (st != SRNL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool padded = h->cfg.d != srnl::kD;
+  const int elt = h->geom.act_bf16 ? 2 : 4;
+  const int64_t tokens = (int64_t)h->geom.B * h->geom.H * h->geom.W;
+  cudaError_t e;
+  if (h->bws == nullptr) {
+    const size_t nb = srnl::backward_workspace_floats(h->geom, nullptr) * sizeof(float);
+    if ((e = cudaMalloc(&h->bws, nb)) != cudaSuccess) { h->bws = nullptr; return cuda_fail(h, e, "cudaMalloc (backward workspace)"); }
+    h->ws_bytes += nb;
+    if (padded) {
+      const size_t pb = (size_t)tokens * h->geom.C * elt;
+      if ((e = cudaMalloc(&h->dy_pad, pb)) != cudaSuccess) { h->dy_pad = nullptr; return cuda_fail(h, e, "cudaMalloc (dy padding)"); }
+      if ((e = cudaMalloc(&h->dx_pad, pb)) != cudaSuccess) { h->dx_pad = nullptr; return cuda_fail(h, e, "cudaMalloc (dx padding)"); }
+      h->ws_bytes += 2 * pb;
+    }
+  }
+  if (padded) {
+    e = srnl::launch_pad_heads(x, h->x_pad, tokens, h->geom.heads, h->cfg.d, elt, s);
+    if (e == cudaSuccess) e = srnl::launch_pad_heads(dy, h->dy_pad, tokens, h->geom.heads, h->cfg.d, elt, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "head padding launch");
+    x = h->x_pad;
+    dy = h->dy_pad;
+  }
+  srnl::ScanParamsDev p{h->Wq, nullptr, h->G, h->Mm, h->scales};
+  e = srnl::launch_query_projection(h->geom, p, x, h->q, h->dev_err, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
+  srnl::BwdGrads out{};
+  float* dwq = nullptr;
+  if (grads != nullptr) {
+    out = srnl::BwdGrads{grads->scales, grads->M_mem0, grads->M_k0, grads->M_v0, grads->m_eta0, grads->m_alpha0};
+    dwq = grads->W_q;
+  }
+  void* dxk = padded ? h->dx_pad : dx;
+  e = srnl::launch_backward(h->geom, p, h->cfg.d, x, static_cast<const float*>(h->q), dy, dxk, h->bws, out, dwq, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "backward launch");
+  if (padded && (e = srnl::launch_unpad_heads(h->dx_pad, dx, tokens, h->geom.heads, h->cfg.d, elt, s)) != cudaSuccess)
+    return cuda_fail(h, e, "head unpadding launch");
+  return SRNL_OK;
 }
 
 srnl_status srnl_scan_forward_host(srnl_scan* h, const void* x_host, void* y_host, void* stream) {

@@ -192,8 +192,9 @@ __global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ x
 // launchers
 // ---------------------------------------------------------------------------
 cudaError_t prepare_kernels() {
-  const cudaError_t e = prepare_scan_kernels();
+  cudaError_t e = prepare_scan_kernels();
   if (e != cudaSuccess) return e;
+  if ((e = prepare_backward_kernel()) != cudaSuccess) return e;
   return prepare_projection_kernel();
 }
 

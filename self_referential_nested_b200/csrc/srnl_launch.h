@@ -2,7 +2,10 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
+
+#include "srnl_common.cuh"
 
 namespace srnl {
 
@@ -58,6 +61,30 @@ cudaError_t launch_gather(const ScanGeom& g, int route, const void* x, void* xr,
 cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
                                   float* yr, float* finals, int* err, unsigned long long* binds,
                                   cudaStream_t s);
+
+// ---- backward (fp32 arithmetic; see srnl_scan_bwd.cu)
+constexpr int kSeqPart = kD * kD + (2 * kD + 2) * kD + kD;   // dM0, dG, dscale partials per sequence
+struct BwdGrads {      // device outputs in the caller's (unpadded) layouts; nullptr skips one
+  float* scales;       // [routes][heads * d]
+  float* M_mem0;       // [routes][heads][d][d]
+  float* M_k0;
+  float* M_v0;
+  float* m_eta0;       // [routes][heads][d]
+  float* m_alpha0;
+};
+struct BwdLayout {     // float offsets of the backward workspace
+  size_t dxr, dqr, dq, parts, ckpt, qs, dwq, total;
+  int max_chunks, Lmax, nsplit;
+};
+// Floats of backward workspace for the geometry (and the layout when lay != nullptr).
+size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay);
+// Gradient of sum(dy * y) for the forward y(x, params) of geometry g (32-wide padded heads,
+// ud = the caller's head dim).  x, dy, dx: [B][N][C] act dtype (padded); q: the fp32 query
+// projection of x; ws: backward_workspace_floats(g) floats.  dwq_out: [heads*ud]^2 or nullptr.
+cudaError_t launch_backward(const ScanGeom& g, const ScanParamsDev& p, int ud, const void* x, const float* q,
+                            const void* dy, void* dx, float* ws, const BwdGrads& out, float* dwq_out,
+                            cudaStream_t s);
+cudaError_t prepare_backward_kernel();
 
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)
 cudaError_t prepare_scan_kernels();
