@@ -388,6 +388,149 @@ def run_ours(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def backward_flops_per_token(d=32):
+    """Algorithmic fp32 flops of the backward per (route, head) token, as the scan-backward
+    kernel restates it: the forward chain twice (checkpoint pass and in-chunk recompute,
+    2 x 5 d^2), generation once (Q_b x and G w: 2 d^2 + 2 (2d+2) d), the reverse chain
+    (dQ += a q^T, dQ k, Q_{t-1} u, Q_t q, <Q_{t-1}, dQ>, the three column products and the
+    dQ update: 19 d^2), the per-token adjoints (M0^T dy, G^T dgen, Q_b x, M0 z, Q_b^T dh:
+    8 d^2 + 2 (2d+2) d) and the rank-one parameter sums (dM0, dQ_b, dG: 4 d^2 + 2 (2d+2) d)."""
+    gen = 2 * (2 * d + 2) * d
+    return 10 * d * d + (2 * d * d + gen) + 19 * d * d + (8 * d * d + gen) + (4 * d * d + gen)
+
+
+def backward_cpu_baseline(cfg, budget_s=10.0):
+    from oracle import srnl_grad as GR
+    from srnl_inputs import make_cotangent
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:  # pragma: no cover
+        threadpool_limits = None
+    inp = make_inputs(cfg, seed=0)
+    dout = make_cotangent(inp.x32.shape, seed=0, act_dtype=cfg.act_dtype)
+    n, dt = 1, 0.0
+    ctx = threadpool_limits(1) if threadpool_limits else None
+    try:
+        while True:
+            t0 = time.perf_counter()
+            GR.operator_backward(inp.x32[:n], inp.params(), dout[:n], alpha_max=cfg.alpha, eps=cfg.eps,
+                                 chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, heads=cfg.heads)
+            dt = time.perf_counter() - t0
+            if dt * 2 > budget_s or n >= cfg.B:
+                break
+            n = min(cfg.B, max(n + 1, int(n * budget_s / max(dt, 1e-3) / 2)))
+    finally:
+        if ctx is not None:
+            ctx.__exit__(None, None, None)
+    return {"value": 4.0 * n * cfg.H * cfg.W / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"backward of {n} of {cfg.B} images of {cfg.name}, float64 numpy, 1 thread, {dt:.1f} s"}
+
+
+def run_backward(args, cfg):
+    """Backward pass: dL/dx and every parameter gradient for an upstream gradient dL/dy, on one
+    GPU (fp32 arithmetic; x, dy and dx in the workload's activation dtype).  One step = one
+    srnl_scan_backward over the batch, inputs resident in HBM, L2 flushed before each step."""
+    import torch
+    import self_referential_nested_b200 as S
+    from self_referential_nested_b200 import build as Bld
+    from srnl_inputs import make_cotangent
+
+    Bld.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    act = cfg.act_dtype
+    inp = make_inputs(cfg, seed=0)
+    params = inp.params()
+    h = S.srnl_scan_create(dict(B=cfg.B, H=cfg.H, W=cfg.W, C=cfg.C, heads=cfg.heads, d=cfg.d, alpha=cfg.alpha,
+                                eps=cfg.eps, chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, act_dtype=act,
+                                gen_dtype="f32", injection_cap=args.cap), params)
+    g_np = make_cotangent(inp.x32.shape, seed=0, act_dtype=act)
+
+    def to_dev(a32):
+        if act == "bf16":
+            from srnl_inputs import bf16_round_bits
+            return torch.from_numpy(bf16_round_bits(a32).view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a32)).to(dev)
+
+    x, dy = to_dev(inp.x32), to_dev(g_np)
+    dx = torch.empty_like(x)
+    grads = {k: torch.empty(np.shape(params[k]), dtype=torch.float32, device=dev) for k in S.GRAD_KEYS}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        S.srnl_scan_backward(h, x, dy, dx, grads, stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    S.srnl_scan_enable_stage_timing(h, max(args.steps, 1))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_((i + 1) & 0xFF)
+        starts[i].record(stream)
+        S.srnl_scan_backward(h, x, dy, dx, grads, stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    stage, n_timed = S.srnl_scan_stage_times(h)
+    assert n_timed == args.steps
+    S.srnl_scan_enable_stage_timing(h, 0)
+    total_ms = float(sum(s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)))
+    # end to end: pinned x and dy copied in, dx and the parameter gradients copied out, each step
+    xh, dyh = x.cpu().pin_memory(), dy.cpu().pin_memory()
+    dxh = torch.empty_like(xh).pin_memory()
+    gh = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        x.copy_(xh, non_blocking=True)
+        dy.copy_(dyh, non_blocking=True)
+        S.srnl_scan_backward(h, x, dy, dx, grads, stream)
+        dxh.copy_(dx, non_blocking=True)
+        for k in grads:
+            gh[k].copy_(grads[k], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    e2e_ms = e0.elapsed_time(e1)
+    h.close()
+
+    peaks = load_peaks()
+    ms_step = total_ms / args.steps
+    route_tokens = 4 * cfg.B * cfg.H * cfg.W
+    scan_ms = float(stage[1])
+    flops = backward_flops_per_token(cfg.d) * route_tokens * cfg.heads
+    fp32_peak_tflops = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+    achieved = flops / (scan_ms * 1e-3) / 1e12
+    elt = 2 if act == "bf16" else 4
+    grad_bytes = int(sum(v.numel() for v in grads.values()) * 4)
+    line = {
+        "metric": "SRNL 4-dir scan backward route-tokens/s (1xB200)", "value": route_tokens / (ms_step * 1e-3),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded normal features and upstream gradients, random-init memories)",
+        "config": {"workload": cfg.name, "pass": "backward", "B": cfg.B, "H": cfg.H, "W": cfg.W, "C": cfg.C,
+                   "heads": cfg.heads, "d": cfg.d, "alpha": cfg.alpha, "act_dtype": act, "gen_dtype": "f32",
+                   "injection_cap": args.cap, "l2": "flushed (256 MiB write before each timed step)"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": fp32_peak_tflops, "unit": "TFLOP/s",
+                     "frac": achieved / fp32_peak_tflops, "traffic": None, "kernel": "srnl_scan_backward_kernel",
+                     "kernel_ms": scan_ms, "flops_per_route_head_token": backward_flops_per_token(cfg.d),
+                     "peak_note": "fp32 FMA peak 148 SM x 128 lanes x 2 x sm_max_mhz (derived)"},
+        "stage_ms": {"query_projection": float(stage[0]), "scan_backward": scan_ms, "combine": float(stage[2])},
+        "e2e": {"value": route_tokens * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(2 * x.numel() * elt), "d2h_bytes_per_step": int(dx.numel() * elt) + grad_bytes,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": (7 if cfg.d == 32 else 10) * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = backward_cpu_baseline(cfg)
+    print(json.dumps(line), flush=True)
+
+
 def run_seq(args):
     """Standalone SRNL layer on sequences ([B, T, D], 64-token chunks, x as the query):
     B sequences x heads of T tokens, one direction.  One GPU; prints one JSON line."""
@@ -447,6 +590,8 @@ def main():
                     help="injection cap: the soft cap (the method) or the hard clamp of its ablation")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
     ap.add_argument("--seq", action="store_true", help="time the standalone sequence layer instead")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (gradients of x and every parameter) instead")
     ap.add_argument("--seq-batch", type=int, default=128)
     ap.add_argument("--seq-tokens", type=int, default=3136)
     args = ap.parse_args()
@@ -464,6 +609,9 @@ def main():
         sys.exit(2)
     if args.impl == "reference":
         run_reference(args, cfg, rank, world)
+        return
+    if args.backward:
+        run_backward(args, cfg)
         return
     if world > 1:
         import datetime

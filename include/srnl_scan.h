@@ -186,7 +186,10 @@ SRNL_API srnl_status srnl_scan_gather(const srnl_scan* h, int route, const void*
 /* Stage timing.  srnl_scan_enable_stage_timing(h, n) with n > 0 makes each
  * later forward record CUDA events on its stream before and after each of its
  * three kernels (query projection, scan, fusion), keeping the events of the
- * last n forwards (n <= 1024); n = 0 turns timing off.
+ * last n forwards (n <= 1024); n = 0 turns timing off.  A backward call records
+ * its three stages in the same ring (query projection, scan backward, combine:
+ * route sums, dx, dW_q and the parameter reductions); time one kind of call per
+ * window. 
  * srnl_scan_stage_times waits for those events, writes the mean duration in
  * milliseconds of each kernel over the kept forwards to ms_out[0..2] and the
  * number of forwards averaged to *count (may be NULL), then starts a new
@@ -243,9 +246,9 @@ typedef struct {
  * SRNL_E_UNSUPPORTED): all arithmetic is fp32; act_dtype SRNL_BF16 means bf16 x, dy and dx.
  * The forward is recomputed from x (boundary products are kept per chunk and the states
  * inside a chunk recomputed), so no forward state is needed.  The first call allocates the
- * backward workspace (cudaMalloc, synchronous; about 20 fp32 values per activation element
- * plus 4 KB per chunk and per chunk token of every (route, batch, head) sequence); later calls
- * reuse it.  Asynchronous on `stream`; shares the handle's workspace with the forward. */
+ * backward workspace (cudaMalloc, synchronous; about 9 fp32 values per activation element,
+ * plus per (route, batch, head) sequence 288 bytes per token and 4 KB per chunk and per token
+ * of its longest chunk); later calls reuse it.  Asynchronous on `stream`; shares the handle's workspace with the forward. */
 SRNL_API srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void* dx,
                                        const srnl_scan_grads* grads, void* stream);
 

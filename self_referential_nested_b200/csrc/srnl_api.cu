@@ -371,19 +371,29 @@ srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void
     dy = h->dy_pad;
   }
   srnl::ScanParamsDev p{h->Wq, nullptr, h->G, h->Mm, h->scales};
+  cudaEvent_t* ev = h->ring > 0 ? &h->ev[(size_t)(h->recorded % h->ring) * 4] : nullptr;
+  if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   e = srnl::launch_query_projection(h->geom, p, x, h->q, h->dev_err, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
+  if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   srnl::BwdGrads out{};
   float* dwq = nullptr;
   if (grads != nullptr) {
     out = srnl::BwdGrads{grads->scales, grads->M_mem0, grads->M_k0, grads->M_v0, grads->m_eta0, grads->m_alpha0};
     dwq = grads->W_q;
   }
+  e = srnl::launch_backward_scan(h->geom, p, x, static_cast<const float*>(h->q), dy, h->bws, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "backward scan launch");
+  if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   void* dxk = padded ? h->dx_pad : dx;
-  e = srnl::launch_backward(h->geom, p, h->cfg.d, x, static_cast<const float*>(h->q), dy, dxk, h->bws, out, dwq, s);
-  if (e != cudaSuccess) return cuda_fail(h, e, "backward launch");
+  e = srnl::launch_backward_combine(h->geom, p, h->cfg.d, x, h->bws, dxk, out, dwq, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "backward combine launch");
   if (padded && (e = srnl::launch_unpad_heads(h->dx_pad, dx, tokens, h->geom.heads, h->cfg.d, elt, s)) != cudaSuccess)
     return cuda_fail(h, e, "head unpadding launch");
+  if (ev) {
+    if ((e = cudaEventRecord(ev[3], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
+    ++h->recorded;
+  }
   return SRNL_OK;
 }
 

@@ -73,17 +73,22 @@ struct BwdGrads {      // device outputs in the caller's (unpadded) layouts; nul
   float* m_alpha0;
 };
 struct BwdLayout {     // float offsets of the backward workspace
-  size_t dxr, dqr, dq, parts, ckpt, qs, dwq, total;
+  size_t dxr, dqr, dq, parts, ckpt, qs, grec, dwq, total;
   int max_chunks, Lmax, nsplit;
 };
 // Floats of backward workspace for the geometry (and the layout when lay != nullptr).
 size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay);
 // Gradient of sum(dy * y) for the forward y(x, params) of geometry g (32-wide padded heads,
-// ud = the caller's head dim).  x, dy, dx: [B][N][C] act dtype (padded); q: the fp32 query
-// projection of x; ws: backward_workspace_floats(g) floats.  dwq_out: [heads*ud]^2 or nullptr.
-cudaError_t launch_backward(const ScanGeom& g, const ScanParamsDev& p, int ud, const void* x, const float* q,
-                            const void* dy, void* dx, float* ws, const BwdGrads& out, float* dwq_out,
-                            cudaStream_t s);
+// ud = the caller's head dim), in two launches.  x, dy, dx: [B][N][C] act dtype (padded);
+// q: the fp32 query projection of x; ws: backward_workspace_floats(g) floats.
+// launch_backward_scan: the per-sequence reverse scan (route partials of dx and dq, and
+// per-sequence parameter partials, into ws).  launch_backward_combine: dx = sum of the route
+// partials + dq W_q, dW_q (dwq_out [heads*ud]^2, or nullptr) and the batch-ordered
+// parameter reductions into `out`.
+cudaError_t launch_backward_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const float* q,
+                                 const void* dy, float* ws, cudaStream_t s);
+cudaError_t launch_backward_combine(const ScanGeom& g, const ScanParamsDev& p, int ud, const void* x, float* ws,
+                                    void* dx, const BwdGrads& out, float* dwq_out, cudaStream_t s);
 cudaError_t prepare_backward_kernel();
 
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)

@@ -47,21 +47,23 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSeg = 64;        // tokens whose gates sit in shared memory at once
+constexpr int kSeg = 32;        // tokens whose gate records sit in shared memory at once
 constexpr int kSB = 16;         // tokens per reverse sub-block
-constexpr int kLd = kD + 1;     // padded row stride of 32-wide matrices
-constexpr int kRec = 72;        // per-token gate record: k[32] u[32] alpha eta s a beta
-constexpr int kRk = 0, kRu = 32, kRal = 64, kReta = 65, kRs = 66, kRa = 67, kRb = 68;
+constexpr int kLd = kD + 4;     // row stride of 32-wide matrices: 16-byte rows, conflict-free
+                                //   float4 row reads and scalar column reads
+constexpr int kGtLd = kGen + 2; // row stride of G^T (68 = 4 mod 32: conflict-free float4 rows)
+constexpr int kRec = 72;        // per-token gate record: k[32] u[32] alpha eta s a beta |k|^2 |k-v|^2
+constexpr int kRk = 0, kRu = 32, kRal = 64, kReta = 65, kRs = 66, kRa = 67, kRb = 68, kRkn2 = 69, kRne2 = 70;
 constexpr int kPart = 2 + 3 * kD;   // per (token, warp): dalpha, p.w, du[32], dk[32], dq[32]
 constexpr int kGenLd = kGen + 2;
 
 struct BwdSmem {
   alignas(16) float Mm[kD][kLd];            // M_mem0 of this (route, head)
   alignas(16) float Gm[kGen][kLd];          // generating initials G
+  alignas(16) float GmT[kD][kGtLd];         // G transposed (columns 66, 67 zero)
   alignas(16) float Qb[kD][kLd];            // Q at the current chunk start
   alignas(16) float rec[kSeg][kRec];        // gates of the current segment
-  alignas(16) float wx[kWarps][kD];         // per-warp scratch of the gate pass
-  alignas(16) float wh[kWarps][kD];
+  alignas(16) float wh[kWarps][kD];         // per-warp scratch of the gate pass
   alignas(16) float sx[kSB][kD];            // reverse sub-block: x, q, dout, dy (scaled), a = M0^T dy,
   alignas(16) float sq[kSB][kD];            //   Q_t q_t, dh, h = Q_b x, dgen
   alignas(16) float sdo[kSB][kD];
@@ -72,9 +74,12 @@ struct BwdSmem {
   alignas(16) float sh[kSB][kD];
   alignas(16) float sdg[kSB][kGenLd];
   alignas(16) float part[kSB][kWarps][kPart];
+  alignas(16) float sc[kSB][8];             // per-token scalars of the gate backward
   alignas(16) float ds[kWarps][kD];
 };
 static_assert(sizeof(BwdSmem) <= 112 * 1024, "two CTAs per SM");
+static_assert(offsetof(BwdSmem, sq) == offsetof(BwdSmem, sx) + sizeof(float) * kSB * kD && 2 * kSB >= kSeg,
+              "the gate pass stages a segment's x over sx and sq");
 
 struct BwdArgs {
   const void* x;       // [B][N][C] act dtype (C = heads * 32)
@@ -85,6 +90,7 @@ struct BwdArgs {
   float* parts;        // [nseq][kSeqPart] dM0, dG, dscale partials per sequence
   float* ckpt;         // [nseq][max_chunks + 1][32 * 32]
   float* qs;           // [nseq][Lmax][32 * 32]
+  float* grec;         // [nseq][N][kRec] gate records of every token (written by phase 1)
   const float* G;
   const float* Mm;
   const float* scales;
@@ -138,57 +144,142 @@ __device__ __forceinline__ float col4_sum(float c0, float c1, float c2, float c3
   return (b3 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, s, 8);
 }
 
-// Gates of one token, one warp, lane j holding component j of k~ and v (accurate math
-// functions; the same decisions as the forward's clamps).  Writes the token's record.
-__device__ __forceinline__ void gate_forward(float kt, float v, float a, float beta, const BwdArgs& A,
-                                             float* rec, int lane) {
-  const float s = sqrtf(warp_sum(kt * kt) + A.eps);
-  const float k = kt / s;
-  const float kn2 = warp_sum(k * k);
-  const float e = k - v;
-  const float gain = sqrtf(warp_sum(e * e)) * sqrtf(kn2);
-  const float sg = sigmoid_f(beta);
-  const float al = fminf(sg, A.alpha);
+// Dot product of a 16-byte-aligned shared row with a shared vector that every lane reads
+// (broadcast), n a multiple of 4; two accumulators.
+template <int n>
+__device__ __forceinline__ float dot_vec(const float* a, const float* b) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < n; i += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(a + i);
+    const float4 y = *reinterpret_cast<const float4*>(b + i);
+    float& acc = ((i >> 2) & 1) ? s1 : s0;
+    acc = fmaf(x.x, y.x, acc);
+    acc = fmaf(x.y, y.y, acc);
+    acc = fmaf(x.z, y.z, acc);
+    acc = fmaf(x.w, y.w, acc);
+  }
+  return s0 + s1;
+}
+
+// Column j of a shared matrix (row stride kLd, scalar reads) against a broadcast vector.
+__device__ __forceinline__ float dot_col(const float (*m)[kLd], int j, const float* b) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < kD; i += 4) {
+    const float4 y = *reinterpret_cast<const float4*>(b + i);
+    float& acc = ((i >> 2) & 1) ? s1 : s0;
+    acc = fmaf(m[i][j], y.x, acc);
+    acc = fmaf(m[i + 1][j], y.y, acc);
+    acc = fmaf(m[i + 2][j], y.z, acc);
+    acc = fmaf(m[i + 3][j], y.w, acc);
+  }
+  return s0 + s1;
+}
+
+// Copy n4 float4 values (16-byte aligned both sides) with the whole block.
+__device__ __forceinline__ void block_copy4(float* dst, const float* src, int n4, int tid) {
+  for (int i = tid; i < n4; i += kThreads)
+    reinterpret_cast<float4*>(dst)[i] = reinterpret_cast<const float4*>(src)[i];
+}
+
+// Scalar gates of one token from |k|^2, |k - v|^2, a and beta (accurate math functions; the
+// forward's clamp decisions): alpha_t and eta.
+__device__ __forceinline__ void gate_scalars_f(float kn2, float ne2, float a, float beta, const BwdArgs& A,
+                                               float& al, float& eta) {
+  const float gain = sqrtf(ne2) * sqrtf(kn2);
+  al = fminf(sigmoid_f(beta), A.alpha);
   const float eta0 = softplus_f(a);
   const float m = 1.f - al;
   float eta1;
   if (A.hard_cap) eta1 = (eta0 * gain > m) ? m / gain : eta0;
   else eta1 = eta0 * phi_f(eta0 * gain / m);
-  const float eta = (eta1 * kn2 > 2.f) ? 2.f / kn2 : eta1;
-  rec[kRk + lane] = k;
-  rec[kRu + lane] = (1.f + al) * k - v;
-  if (lane == 0) {
-    rec[kRal] = al; rec[kReta] = eta; rec[kRs] = s; rec[kRa] = a; rec[kRb] = beta;
-  }
+  eta = (eta1 * kn2 > 2.f) ? 2.f / kn2 : eta1;
 }
 
-// Gates of tokens [t0, t0 + T) of the sequence into sm.rec (warp per token).  Q_b in sm.Qb.
+// Gates of tokens [t0, t0 + T) of the sequence into sm.rec (T <= kSeg), by all threads:
+// the segment's x staged block-wide (over sx and sq), generation and the vector reductions
+// with a warp per token, the scalar gates with a lane per token, then u = (1 + alpha) k - v.
+// Q_b in sm.Qb.  Ends with a block barrier.
 __device__ void gates_segment(BwdSmem& sm, const BwdArgs& A, int r, int64_t tokbase_b, int ch0, int t0, int T,
-                              int warp, int lane) {
-  const int C = A.C;
-  for (int tt = warp; tt < T; tt += kWarps) {
+                              int tid) {
+  float (*xs)[kD] = reinterpret_cast<float (*)[kD]>(&sm.sx[0][0]);   // kSeg rows: sx then sq
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int idx = tid; idx < T * kD; idx += kThreads) {
+    const int tt = idx >> 5;
     const int p = route_pos(r, t0 + tt, A.H, A.W);
-    sm.wx[warp][lane] = load_act(A.x, (tokbase_b + p) * C + ch0 + lane, A.act_bf16);
-    __syncwarp();
-    float hw = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < kD; ++j) hw = fmaf(sm.Qb[lane][j], sm.wx[warp][j], hw);
-    sm.wh[warp][lane] = hw;
-    __syncwarp();
-    float kt = 0.f, vv = 0.f, ex = 0.f;
-    const int er = kD * 2 + (lane & 1);   // lanes 0/1: a / beta rows
-#pragma unroll 8
-    for (int i = 0; i < kD; ++i) {
-      const float hi = sm.wh[warp][i];
-      kt = fmaf(sm.Gm[lane][i], hi, kt);
-      vv = fmaf(sm.Gm[kD + lane][i], hi, vv);
-      ex = fmaf(sm.Gm[er][i], hi, ex);
-    }
-    const float a = __shfl_sync(0xffffffffu, ex, 0);
-    const float beta = __shfl_sync(0xffffffffu, ex, 1);
-    gate_forward(kt, vv, a, beta, A, sm.rec[tt], lane);
-    __syncwarp();
+    xs[tt][lane] = load_act(A.x, (tokbase_b + p) * A.C + ch0 + lane, A.act_bf16);
   }
+  __syncthreads();
+  for (int tt = warp; tt < T; tt += kWarps) {
+    sm.wh[warp][lane] = dot_vec<kD>(sm.Qb[lane], xs[tt]);                 // w = Q_b x
+    __syncwarp();
+    const float kt = dot_vec<kD>(sm.Gm[lane], sm.wh[warp]);               // k~
+    const float vv = dot_vec<kD>(sm.Gm[kD + lane], sm.wh[warp]);          // v
+    const float ex = dot_vec<kD>(sm.Gm[2 * kD + (lane & 1)], sm.wh[warp]);  // lanes 0/1: a / beta
+    __syncwarp();
+    const float s = sqrtf(warp_sum(kt * kt) + A.eps);
+    const float k = kt / s;
+    const float e = k - vv;
+    const float kn2 = warp_sum(k * k);
+    const float ne2 = warp_sum(e * e);
+    float* rc = sm.rec[tt];
+    rc[kRk + lane] = k;
+    rc[kRu + lane] = vv;   // v until u is formed below
+    if (lane == 0) { rc[kRs] = s; rc[kRa] = ex; rc[kRkn2] = kn2; rc[kRne2] = ne2; }
+    if (lane == 1) rc[kRb] = ex;
+  }
+  __syncthreads();
+  if (tid < T) {
+    float* rc = sm.rec[tid];
+    float al, eta;
+    gate_scalars_f(rc[kRkn2], rc[kRne2], rc[kRa], rc[kRb], A, al, eta);
+    rc[kRal] = al;
+    rc[kReta] = eta;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < T * kD; idx += kThreads) {
+    float* rc = sm.rec[idx >> 5];
+    rc[kRu + lane] = (1.f + rc[kRal]) * rc[kRk + lane] - rc[kRu + lane];
+  }
+  __syncthreads();
+}
+
+// Scalar part of the gate backward for one token (one lane per token).  In: sc[0] = dL/dalpha_t
+// so far, sc[1] = dL/deta_t, sc[2] = |k|^2, sc[3] = |k - v|^2; the token's record.  Out:
+// sc[4] = c_e, sc[5] = c_k with dk += c_e (k - v) + c_k k and dv -= c_e (k - v) (the gain and
+// spectral-clamp paths), sc[6] = dL/da, sc[7] = dL/dbeta.
+__device__ __forceinline__ void gate_backward_scalars(float* sc, const float* rc, const BwdArgs& A) {
+  float dal = sc[0];
+  const float deta = sc[1], kn2 = sc[2];
+  const float ne = sqrtf(sc[3]), kn = sqrtf(kn2), gain = ne * kn;
+  const float al = rc[kRal], a = rc[kRa], beta = rc[kRb];
+  const float sg = sigmoid_f(beta);
+  const float eta0 = softplus_f(a);
+  const float m = 1.f - al;
+  float eta1;
+  if (A.hard_cap) eta1 = (eta0 * gain > m) ? m / gain : eta0;
+  else eta1 = eta0 * phi_f(eta0 * gain / m);
+  const bool over = eta1 * kn2 > 2.f;                        // spectral clamp eta = 2 / |k|^2
+  const float deta1 = over ? 0.f : deta;
+  const float dkn2 = over ? -2.f * deta / (kn2 * kn2) : 0.f;
+  float deta0, dgain;
+  if (A.hard_cap) {                                          // eta1 = min(eta0, (1 - alpha_t) / g)
+    const bool binds = eta0 * gain > m;
+    deta0 = binds ? 0.f : deta1;
+    dgain = binds ? -deta1 * m / (gain * gain) : 0.f;
+    if (binds) dal -= deta1 / gain;
+  } else {                                                   // eta1 = eta0 phi(eta0 g / (1 - alpha_t))
+    const float z = eta0 * gain / m;
+    const float dz = deta1 * eta0 * dphi_f(z);
+    deta0 = deta1 * phi_f(z) + dz * gain / m;
+    dgain = dz * eta0 / m;
+    dal += dz * eta0 * gain / (m * m);
+  }
+  sc[4] = (ne > 0.f) ? dgain * kn / ne : 0.f;                // g = |k - v| |k|
+  sc[5] = 2.f * dkn2 + (kn > 0.f ? dgain * ne / kn : 0.f);
+  sc[6] = deta0 * sigmoid_f(a);                              // eta0 = softplus(a)
+  sc[7] = (sg > A.alpha) ? 0.f : dal * sg * (1.f - sg);      // alpha_t = min(sigmoid(beta), alpha)
 }
 
 __device__ __forceinline__ void load_row4(const float* m, int i, int j0, float (&v)[4]) {
@@ -235,7 +326,14 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_backward_kernel(const B
   float* qs = A.qs + (size_t)seq * A.Lmax * (kD * kD);
 
   for (int idx = tid; idx < kD * kD; idx += kThreads) sm.Mm[idx / kD][idx % kD] = A.Mm[(size_t)rh * kD * kD + idx];
-  for (int idx = tid; idx < kGen * kD; idx += kThreads) sm.Gm[idx / kD][idx % kD] = A.G[(size_t)rh * kGen * kD + idx];
+  for (int idx = tid; idx < kGen * kD; idx += kThreads) {
+    const float gv = A.G[(size_t)rh * kGen * kD + idx];
+    sm.Gm[idx / kD][idx % kD] = gv;
+    sm.GmT[idx % kD][idx / kD] = gv;
+  }
+  if (tid < kD) { sm.GmT[tid][kGen] = 0.f; sm.GmT[tid][kGen + 1] = 0.f; }
+  if (tid < kSB) { sm.sdg[tid][kGen] = 0.f; sm.sdg[tid][kGen + 1] = 0.f; }
+  float* grec = A.grec + (size_t)seq * N * kRec;
   for (int idx = tid; idx < kWarps * kD; idx += kThreads) sm.ds[idx / kD][idx % kD] = 0.f;
 
   // ---------------- phase 1: forward chain, checkpoints at chunk starts
@@ -250,8 +348,8 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_backward_kernel(const B
     const int c0 = c * L, Lc = min(L, N - c0);
     for (int s0 = 0; s0 < Lc; s0 += kSeg) {
       const int T = min(kSeg, Lc - s0);
-      gates_segment(sm, A, r, tokbase_b, ch0, c0 + s0, T, warp, lane);
-      __syncthreads();
+      gates_segment(sm, A, r, tokbase_b, ch0, c0 + s0, T, tid);
+      block_copy4(grec + (size_t)(c0 + s0) * kRec, sm.rec[0], T * kRec / 4, tid);
       for (int tt = 0; tt < T; ++tt) forward_step(Qr, sm.rec[tt], j0);
       __syncthreads();
     }
@@ -280,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_backward_kernel(const B
     // forward recompute of Q_t inside the chunk
     for (int sg = 0; sg < nseg; ++sg) {
       const int s0 = sg * kSeg, T = min(kSeg, Lc - s0);
-      gates_segment(sm, A, r, tokbase_b, ch0, c0 + s0, T, warp, lane);
+      block_copy4(sm.rec[0], grec + (size_t)(c0 + s0) * kRec, T * kRec / 4, tid);
       __syncthreads();
       for (int tt = 0; tt < T; ++tt) {
         forward_step(Qr, sm.rec[tt], j0);
@@ -297,13 +395,14 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_backward_kernel(const B
       const int s0 = sg * kSeg, T = min(kSeg, Lc - s0);
       if (nseg > 1) {
         __syncthreads();
-        gates_segment(sm, A, r, tokbase_b, ch0, c0 + s0, T, warp, lane);
+        block_copy4(sm.rec[0], grec + (size_t)(c0 + s0) * kRec, T * kRec / 4, tid);
         __syncthreads();
       }
       for (int sb_end = T; sb_end > 0; sb_end -= kSB) {
         const int sb0 = max(0, sb_end - kSB), nsb = sb_end - sb0;
         // stage x, q, dout, dy = scale * dout and a = M0^T dy (warp per token)
-        for (int tt = warp; tt < nsb; tt += kWarps) {
+        for (int idx = tid; idx < nsb * kD; idx += kThreads) {
+          const int tt = idx >> 5;
           const int t = c0 + s0 + sb0 + tt;
           const int64_t o = (tokbase_b + route_pos(r, t, A.H, A.W)) * C + ch0 + lane;
           sm.sx[tt][lane] = load_act(A.x, o, A.act_bf16);
@@ -311,12 +410,9 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_backward_kernel(const B
           const float g = load_act(A.dy, o, A.act_bf16);
           sm.sdo[tt][lane] = g;
           sm.sdy[tt][lane] = scale_l * g;
-          __syncwarp();
-          float av = 0.f;
-#pragma unroll 8
-          for (int j = 0; j < kD; ++j) av = fmaf(sm.Mm[j][lane], sm.sdy[tt][j], av);
-          sm.sa[tt][lane] = av;
         }
+        __syncthreads();
+        for (int tt = warp; tt < nsb; tt += kWarps) sm.sa[tt][lane] = dot_col(sm.Mm, lane, sm.sdy[tt]);  // M0^T dy
         __syncthreads();
         // reverse chain over the sub-block (no block barrier inside)
         {
@@ -382,85 +478,66 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_backward_kernel(const B
           }
         }
         __syncthreads();
-        // per token: gate backward, generation and readout adjoints (warp per token)
+        // per token, vector part (warp per token): partial sums over the warps, the write's
+        // gradients of k and v, and the reductions the scalar gate backward needs
         for (int tt = warp; tt < nsb; tt += kWarps) {
           const int t = c0 + s0 + sb0 + tt;
           const float* rc = sm.rec[sb0 + tt];
-          float dal = 0.f, pw = 0.f, du = 0.f, dkT = 0.f, dq = 0.f;
+          float ta = 0.f, pw = 0.f, du = 0.f, dkT = 0.f, dq = 0.f;
 #pragma unroll
           for (int w8 = 0; w8 < kWarps; ++w8) {
             const float* pt = sm.part[tt][w8];
-            dal += pt[0];
+            ta += pt[0];
             pw += pt[1];
             du += pt[2 + lane];
             dkT += pt[2 + kD + lane];
             dq += pt[2 + 2 * kD + lane];
           }
-          const float al = rc[kRal], eta = rc[kReta], s = rc[kRs], a = rc[kRa], beta = rc[kRb];
+          const float al = rc[kRal], eta = rc[kReta];
           const float k = rc[kRk + lane];
           const float v = (1.f + al) * k - rc[kRu + lane];
-          du *= -eta;
-          float dk = -eta * dkT + (1.f + al) * du;
-          float dv = -du;
-          dal += warp_sum(k * du);
-          const float deta = -pw;
-          // gate backward (the forward's decisions are recomputed from the same values)
-          const float kn2 = warp_sum(k * k);
+          du *= -eta;                                  // du = -eta Q_{t-1}^T w
           const float e = k - v;
-          const float ne = sqrtf(warp_sum(e * e));
-          const float kn = sqrtf(kn2);
-          const float gain = ne * kn;
-          const float sg = sigmoid_f(beta);
-          const float eta0 = softplus_f(a);
-          const float m = 1.f - al;
-          float eta1;
-          if (A.hard_cap) eta1 = (eta0 * gain > m) ? m / gain : eta0;
-          else eta1 = eta0 * phi_f(eta0 * gain / m);
-          const bool over = eta1 * kn2 > 2.f;
-          const float deta1 = over ? 0.f : deta;
-          const float dkn2 = over ? -2.f * deta / (kn2 * kn2) : 0.f;
-          float deta0, dgain;
-          if (A.hard_cap) {
-            const bool binds = eta0 * gain > m;
-            deta0 = binds ? 0.f : deta1;
-            dgain = binds ? -deta1 * m / (gain * gain) : 0.f;
-            if (binds) dal -= deta1 / gain;
-          } else {
-            const float z = eta0 * gain / m;
-            const float dz = deta1 * eta0 * dphi_f(z);
-            deta0 = deta1 * phi_f(z) + dz * gain / m;
-            dgain = dz * eta0 / m;
-            dal += dz * eta0 * gain / (m * m);
+          const float kdu = warp_sum(k * du);          // u = (1 + alpha) k - v
+          const float kn2 = warp_sum(k * k);
+          const float ne2 = warp_sum(e * e);
+          sm.sdg[tt][lane] = -eta * dkT + (1.f + al) * du;
+          sm.sdg[tt][kD + lane] = -du;
+          if (lane == 0) {
+            float* sc = sm.sc[tt];
+            sc[0] = ta + kdu;
+            sc[1] = -pw;
+            sc[2] = kn2;
+            sc[3] = ne2;
           }
-          const float de = (ne > 0.f) ? dgain * kn / ne * e : 0.f;
-          const float dkn = dgain * ne;
-          dk += de + (2.f * dkn2 + (kn > 0.f ? dkn / kn : 0.f)) * k;
-          dv -= de;
-          const float dkt = (dk - k * warp_sum(k * dk)) / s;
-          const float da = deta0 * sigmoid_f(a);
-          const float dbeta = (sg > A.alpha) ? 0.f : dal * sg * (1.f - sg);
-          sm.sdg[tt][lane] = dkt;
+          A.dqr[((int64_t)r * A.B * N + tokbase_b + route_pos(r, t, A.H, A.W)) * C + ch0 + lane] = dq;
+        }
+        __syncthreads();
+        if (tid < nsb) gate_backward_scalars(sm.sc[tid], sm.rec[sb0 + tid], A);   // lane per token
+        __syncthreads();
+        // per token, the rest (warp per token): dk~, then the generation and readout adjoints
+        for (int tt = warp; tt < nsb; tt += kWarps) {
+          const int t = c0 + s0 + sb0 + tt;
+          const float* rc = sm.rec[sb0 + tt];
+          const float* sc = sm.sc[tt];
+          const float al = rc[kRal], s = rc[kRs];
+          const float k = rc[kRk + lane];
+          const float e = k - ((1.f + al) * k - rc[kRu + lane]);
+          const float dk = sm.sdg[tt][lane] + sc[4] * e + sc[5] * k;
+          const float dv = sm.sdg[tt][kD + lane] - sc[4] * e;
+          sm.sdg[tt][lane] = (dk - k * warp_sum(k * dk)) / s;   // k = k~ / s
           sm.sdg[tt][kD + lane] = dv;
-          if (lane == 0) { sm.sdg[tt][2 * kD] = da; sm.sdg[tt][2 * kD + 1] = dbeta; }
+          if (lane == 0) { sm.sdg[tt][2 * kD] = sc[6]; sm.sdg[tt][2 * kD + 1] = sc[7]; }
           __syncwarp();
-          float dh = 0.f, hw = 0.f, y = 0.f;
-#pragma unroll 2
-          for (int rr = 0; rr < kGen; ++rr) dh = fmaf(sm.Gm[rr][lane], sm.sdg[tt][rr], dh);
-#pragma unroll 8
-          for (int j = 0; j < kD; ++j) {
-            hw = fmaf(sm.Qb[lane][j], sm.sx[tt][j], hw);
-            y = fmaf(sm.Mm[lane][j], sm.syq[tt][j], y);
-          }
+          const float dh = dot_vec<kGtLd>(sm.GmT[lane], sm.sdg[tt]);   // (G^T dgen)_lane
+          const float hw = dot_vec<kD>(sm.Qb[lane], sm.sx[tt]);         // (Q_b x)_lane
+          const float y = dot_vec<kD>(sm.Mm[lane], sm.syq[tt]);         // (M0 Q_t q)_lane
           sm.sdh[tt][lane] = dh;
           sm.sh[tt][lane] = hw;
           sm.ds[warp][lane] += sm.sdo[tt][lane] * y;
           __syncwarp();
-          float dx = 0.f;
-#pragma unroll 8
-          for (int i = 0; i < kD; ++i) dx = fmaf(sm.Qb[i][lane], sm.sdh[tt][i], dx);
-          const int64_t o = ((int64_t)r * A.B * N + tokbase_b + route_pos(r, t, A.H, A.W)) * C + ch0 + lane;
-          A.dxr[o] = dx;
-          A.dqr[o] = dq;
+          const float dx = dot_col(sm.Qb, lane, sm.sdh[tt]);             // (Q_b^T dh)_lane
+          A.dxr[((int64_t)r * A.B * N + tokbase_b + route_pos(r, t, A.H, A.W)) * C + ch0 + lane] = dx;
         }
         __syncthreads();
         // rank-one sums of the sub-block: dM0, dQ_b and dG in this thread's layout
@@ -686,6 +763,7 @@ size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay) {
   l.parts = off; off += (size_t)nseq * kSeqPart;
   l.ckpt = off; off += (size_t)nseq * (maxc + 1) * kD * kD;
   l.qs = off;   off += (size_t)nseq * Lmax * kD * kD;
+  l.grec = off; off += (size_t)nseq * N * kRec;
   l.dwq = off;  off += (size_t)l.nsplit * g.C * g.C;
   l.total = off;
   if (lay) *lay = l;
@@ -697,29 +775,42 @@ cudaError_t prepare_backward_kernel() {
                               (int)sizeof(BwdSmem));
 }
 
-cudaError_t launch_backward(const ScanGeom& g, const ScanParamsDev& p, int ud, const void* x, const float* q,
-                            const void* dy, void* dx, float* ws, const BwdGrads& out, float* dwq_out,
-                            cudaStream_t s) {
-  BwdLayout l;
-  backward_workspace_floats(g, &l);
-  const int N = g.H * g.W;
-  const int nseq = g.routes * g.B * g.heads;
+static BwdArgs backward_args(const ScanGeom& g, const ScanParamsDev& p, const void* x, const float* q,
+                             const void* dy, float* ws, const BwdLayout& l) {
   BwdArgs A;
   A.x = x; A.q = q; A.dy = dy;
   A.dxr = ws + l.dxr; A.dqr = ws + l.dqr; A.parts = ws + l.parts; A.ckpt = ws + l.ckpt; A.qs = ws + l.qs;
+  A.grec = ws + l.grec;
   A.G = p.G; A.Mm = p.Mm; A.scales = p.scales;
   A.B = g.B; A.H = g.H; A.W = g.W; A.C = g.C; A.heads = g.heads; A.Lrow = g.Lrow; A.Lcol = g.Lcol;
   A.routes = g.routes; A.max_chunks = l.max_chunks; A.Lmax = l.Lmax;
   A.alpha = g.alpha; A.eps = g.eps; A.act_bf16 = g.act_bf16; A.hard_cap = g.hard_cap;
+  return A;
+}
+
+cudaError_t launch_backward_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const float* q,
+                                 const void* dy, float* ws, cudaStream_t s) {
+  BwdLayout l;
+  backward_workspace_floats(g, &l);
+  const BwdArgs A = backward_args(g, p, x, q, dy, ws, l);
+  const int nseq = g.routes * g.B * g.heads;
   srnl_scan_backward_kernel<<<nseq, kThreads, sizeof(BwdSmem), s>>>(A);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward_combine(const ScanGeom& g, const ScanParamsDev& p, int ud, const void* x, float* ws,
+                                    void* dx, const BwdGrads& out, float* dwq_out, cudaStream_t s) {
+  BwdLayout l;
+  backward_workspace_floats(g, &l);
+  const int N = g.H * g.W;
   const int64_t M = (int64_t)g.B * N;
   const int64_t n4 = M * g.C / 4;
-  sum_routes_kernel<<<(unsigned)std::min<int64_t>((n4 + 255) / 256, 148 * 16), 256, 0, s>>>(A.dqr, ws + l.dq, n4, g.routes);
+  cudaError_t e;
+  sum_routes_kernel<<<(unsigned)std::min<int64_t>((n4 + 255) / 256, 148 * 16), 256, 0, s>>>(ws + l.dqr, ws + l.dq, n4,
+                                                                                           g.routes);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 gx((unsigned)((M + kGT - 1) / kGT), (unsigned)((g.C + kGT - 1) / kGT));
-  dx_gemm_kernel<<<gx, 256, 0, s>>>(ws + l.dq, p.Wq, A.dxr, dx, M, g.C, g.routes, g.act_bf16);
+  dx_gemm_kernel<<<gx, 256, 0, s>>>(ws + l.dq, p.Wq, ws + l.dxr, dx, M, g.C, g.routes, g.act_bf16);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (dwq_out != nullptr) {
     const int tiles = ((g.C + kGT - 1) / kGT) * ((g.C + kGT - 1) / kGT);
@@ -734,7 +825,7 @@ cudaError_t launch_backward(const ScanGeom& g, const ScanParamsDev& p, int ud, c
   }
   const int64_t nparam = (int64_t)g.routes * g.heads * (3 * ud * ud + 3 * ud);
   param_reduce_kernel<<<(unsigned)std::min<int64_t>((nparam + 255) / 256, 4096), 256, 0, s>>>(
-      A.parts, g.routes, g.B, g.heads, ud, out);
+      ws + l.parts, g.routes, g.B, g.heads, ud, out);
   return cudaGetLastError();
 }
 
