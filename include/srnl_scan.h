@@ -316,6 +316,22 @@ SRNL_API srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg,
 SRNL_API srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
                                       float* final_states, void* stream);
 
+/* Backward pass of the sequence layer (see srnl_scan_backward): for dy = dL/dy it writes
+ * dx = dL/dx and, when q is given and dq is not NULL, dq = dL/dq (DEVICE, 16-byte aligned,
+ * [B][T][D] of act_dtype; with q == NULL x is also the query, its gradient is included in
+ * dx and dq must be NULL).  grads: DEVICE fp32 buffers in the srnl_seq_params layouts,
+ * overwritten, each may be NULL (or grads NULL).  gen_dtype must be SRNL_F32 (else
+ * SRNL_E_UNSUPPORTED).  The first call allocates the backward workspace.  Asynchronous. */
+typedef struct {
+  float* M_mem0;   /* [heads][d][d] */
+  float* M_k0;     /* [heads][d][d] */
+  float* M_v0;     /* [heads][d][d] */
+  float* m_eta0;   /* [heads][d]    */
+  float* m_alpha0; /* [heads][d]    */
+} srnl_seq_grads;
+SRNL_API srnl_status srnl_seq_backward(srnl_seq* h, const void* x, const void* q, const void* dy, void* dx,
+                                      void* dq, const srnl_seq_grads* grads, void* stream);
+
 /* Synchronously reads the status word of the handle's kernels (SRNL_OK or
  * SRNL_E_TIMEOUT, as srnl_scan_device_status). */
 SRNL_API srnl_status srnl_seq_device_status(srnl_seq* h);

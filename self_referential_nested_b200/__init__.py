@@ -34,7 +34,7 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_seq_create", "srnl_seq_forward", "srnl_seq_device_status", "srnl_seq_last_error",
             "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count",
             "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
-            "srnl_scan_backward")
+            "srnl_scan_backward", "srnl_seq_backward")
 
 
 class SrnlError(RuntimeError):
@@ -61,6 +61,11 @@ class _Grads(ctypes.Structure):
 
 
 GRAD_KEYS = ("W_q", "scales", "M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")
+SEQ_GRAD_KEYS = ("M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")
+
+
+class _SeqGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in SEQ_GRAD_KEYS]
 
 
 class _SeqConfig(ctypes.Structure):
@@ -117,12 +122,13 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_scan_host_sync.argtypes = [vp]
     lib.srnl_seq_cap_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
     lib.srnl_scan_backward.argtypes = [vp, vp, vp, vp, ctypes.POINTER(_Grads), vp]
+    lib.srnl_seq_backward.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_SeqGrads), vp]
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
                  "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_seq_create", "srnl_seq_forward",
                  "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count",
                  "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
-                 "srnl_scan_backward"):
+                 "srnl_scan_backward", "srnl_seq_backward"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -370,6 +376,17 @@ def srnl_seq_forward(h: SrnlSeq, x, y, q=None, final_states=None, stream=None) -
     """x, q, y: CUDA tensors [B, T, D] of act_dtype; q None means x is the query."""
     h._check(load_library().srnl_seq_forward(h.handle, _ptr(x), _ptr(q), _ptr(y), _ptr(final_states),
                                              _stream(stream)), "srnl_seq_forward")
+
+
+def srnl_seq_backward(h: SrnlSeq, x, dy, dx, q=None, dq=None, grads: Optional[Dict] = None, stream=None) -> None:
+    """Backward of the sequence layer: dx <- dL/dx (including the query path when q is None),
+    dq <- dL/dq when q and dq are given; ``grads`` maps any of SEQ_GRAD_KEYS to fp32 CUDA
+    tensors [heads, d, d] / [heads, d], overwritten with the initial-state gradients."""
+    g = grads or {}
+    gs = _SeqGrads(**{k: _ptr(g.get(k)) for k in SEQ_GRAD_KEYS})
+    h._check(load_library().srnl_seq_backward(h.handle, _ptr(x), _ptr(q), _ptr(dy), _ptr(dx), _ptr(dq),
+                                              ctypes.byref(gs) if grads is not None else None, _stream(stream)),
+             "srnl_seq_backward")
 
 
 def srnl_seq_device_status(h: SrnlSeq) -> None:

@@ -89,6 +89,15 @@ cudaError_t launch_backward_scan(const ScanGeom& g, const ScanParamsDev& p, cons
                                  const void* dy, float* ws, cudaStream_t s);
 cudaError_t launch_backward_combine(const ScanGeom& g, const ScanParamsDev& p, int ud, const void* x, float* ws,
                                     void* dx, const BwdGrads& out, float* dwq_out, cudaStream_t s);
+// Sequence layer (routes = 1): dx = the generation partial (+ the query partial when x is also
+// the query, add_q), dq = the query partial (nullptr skips it), both in the act dtype, and the
+// parameter reductions into `out` (out.scales ignored).  ws: the workspace after
+// launch_backward_scan.
+cudaError_t launch_backward_seq_combine(const ScanGeom& g, int ud, float* ws, void* dx, void* dq, bool add_q,
+                                        const BwdGrads& out, cudaStream_t s);
+// Float offset of the region launch_backward_scan leaves free (B*N*C floats; the sequence
+// layer stages fp32 queries there).
+inline size_t backward_free_region(const ScanGeom& g) { BwdLayout l; backward_workspace_floats(g, &l); return l.dq; }
 cudaError_t prepare_backward_kernel();
 
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)

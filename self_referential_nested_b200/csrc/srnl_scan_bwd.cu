@@ -737,6 +737,22 @@ __global__ void param_reduce_kernel(const float* __restrict__ parts, int routes,
   }
 }
 
+// Sequence layer: dx = dxr (+ dqr when x is also the query), dq = dqr, in the act dtype.
+__global__ void seq_combine_kernel(const float* __restrict__ dxr, const float* __restrict__ dqr, void* dx, void* dq,
+                                   int64_t n, bool add_q, bool bf16) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float gq = dqr[i];
+    const float gx = dxr[i] + (add_q ? gq : 0.f);
+    if (bf16) {
+      reinterpret_cast<__nv_bfloat16*>(dx)[i] = __float2bfloat16_rn(gx);
+      if (dq != nullptr) reinterpret_cast<__nv_bfloat16*>(dq)[i] = __float2bfloat16_rn(gq);
+    } else {
+      reinterpret_cast<float*>(dx)[i] = gx;
+      if (dq != nullptr) reinterpret_cast<float*>(dq)[i] = gq;
+    }
+  }
+}
+
 }  // namespace
 
 size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay) {
@@ -823,6 +839,21 @@ cudaError_t launch_backward_combine(const ScanGeom& g, const ScanParamsDev& p, i
         ws + l.dwq, l.nsplit, g.C, g.heads, ud, dwq_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  const int64_t nparam = (int64_t)g.routes * g.heads * (3 * ud * ud + 3 * ud);
+  param_reduce_kernel<<<(unsigned)std::min<int64_t>((nparam + 255) / 256, 4096), 256, 0, s>>>(
+      ws + l.parts, g.routes, g.B, g.heads, ud, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward_seq_combine(const ScanGeom& g, int ud, float* ws, void* dx, void* dq, bool add_q,
+                                        const BwdGrads& out, cudaStream_t s) {
+  BwdLayout l;
+  backward_workspace_floats(g, &l);
+  const int64_t n = (int64_t)g.B * g.H * g.W * g.C;
+  seq_combine_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16), 256, 0, s>>>(
+      ws + l.dxr, ws + l.dqr, dx, dq, n, add_q, g.act_bf16);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const int64_t nparam = (int64_t)g.routes * g.heads * (3 * ud * ud + 3 * ud);
   param_reduce_kernel<<<(unsigned)std::min<int64_t>((nparam + 255) / 256, 4096), 256, 0, s>>>(
       ws + l.parts, g.routes, g.B, g.heads, ud, out);

@@ -36,6 +36,11 @@ struct srnl_seq {
   void* q_pad = nullptr;
   void* y_pad = nullptr;
   float* fin_pad = nullptr;
+  // backward (allocated on first use): workspace and padded dy / dx / dq for d < 32
+  float* bws = nullptr;
+  void* dy_pad = nullptr;
+  void* dx_pad = nullptr;
+  void* dq_pad = nullptr;
   std::string err;
 };
 
@@ -55,7 +60,7 @@ srnl_status seq_cuda_fail(srnl_seq* h, cudaError_t e, const char* what) {
 
 void seq_free(srnl_seq* h) {
   void* ptrs[] = {h->G, h->Mm, h->scales, h->qbuf, h->yr, h->dev_err, h->binds, h->x_pad, h->q_pad, h->y_pad,
-                  h->fin_pad};
+                  h->fin_pad, h->bws, h->dy_pad, h->dx_pad, h->dq_pad};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   h->G = h->Mm = h->scales = h->yr = nullptr;
@@ -64,6 +69,8 @@ void seq_free(srnl_seq* h) {
   h->binds = nullptr;
   h->x_pad = h->q_pad = h->y_pad = nullptr;
   h->fin_pad = nullptr;
+  h->bws = nullptr;
+  h->dy_pad = h->dx_pad = h->dq_pad = nullptr;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -212,6 +219,77 @@ srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
     e = srnl::launch_unpad_heads(h->y_pad, y, tokens, g.heads, h->cfg.d, elt, s);
     if (e == cudaSuccess && final_states != nullptr)
       e = srnl::launch_unpad_states(h->fin_pad, final_states, (int64_t)g.B * g.heads, h->cfg.d, s);
+    if (e != cudaSuccess) return seq_cuda_fail(h, e, "head unpadding launch");
+  }
+  return SRNL_OK;
+}
+
+srnl_status srnl_seq_backward(srnl_seq* h, const void* x, const void* q, const void* dy, void* dx, void* dq,
+                              const srnl_seq_grads* grads, void* stream) {
+  if (h == nullptr) return SRNL_E_INVAL;
+  h->err.clear();
+  if (x == nullptr || dy == nullptr || dx == nullptr) return seq_fail(h, SRNL_E_INVAL, "x, dy or dx is NULL");
+  if (q == nullptr && dq != nullptr) return seq_fail(h, SRNL_E_INVAL, "dq needs separate queries q");
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || (q != nullptr && !aligned16(q)) ||
+      (dq != nullptr && !aligned16(dq)))
+    return seq_fail(h, SRNL_E_INVAL, "x, q, dy, dx and dq must be 16-byte aligned");
+  const srnl::ScanGeom& g = h->geom;
+  const size_t bytes = (size_t)g.B * g.W * h->cfg.D * (g.act_bf16 ? 2 : 4);
+  const void* ins[] = {x, q, dy};
+  for (const void* in : ins)
+    if (in != nullptr && (overlap(in, dx, bytes) || (dq != nullptr && overlap(in, dq, bytes))))
+      return seq_fail(h, SRNL_E_INVAL, "dx or dq overlaps an input");
+  if (dq != nullptr && overlap(dx, dq, bytes)) return seq_fail(h, SRNL_E_INVAL, "dx and dq overlap");
+  if (g.gen_bf16) return seq_fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for gen_dtype SRNL_F32 handles");
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "cudaGetDevice");
+  if (cur != h->device) return seq_fail(h, SRNL_E_INVAL, "the current device is not the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool padded = h->cfg.d != srnl::kD;
+  const int elt = g.act_bf16 ? 2 : 4;
+  const int64_t tokens = (int64_t)g.B * g.W;
+  const size_t pbytes = (size_t)tokens * g.C * elt;
+  if (h->bws == nullptr) {
+    if ((e = cudaMalloc(&h->bws, srnl::backward_workspace_floats(g, nullptr) * sizeof(float))) != cudaSuccess) {
+      h->bws = nullptr;
+      return seq_cuda_fail(h, e, "cudaMalloc (backward workspace)");
+    }
+    if (padded) {
+      void** bufs[] = {&h->dy_pad, &h->dx_pad, &h->dq_pad};
+      for (void** b : bufs)
+        if ((e = cudaMalloc(b, pbytes)) != cudaSuccess) { *b = nullptr; return seq_cuda_fail(h, e, "cudaMalloc (padding)"); }
+    }
+  }
+  const void* qk = q != nullptr ? q : x;
+  if (padded) {
+    e = srnl::launch_pad_heads(x, h->x_pad, tokens, g.heads, h->cfg.d, elt, s);
+    if (e == cudaSuccess && q != nullptr) e = srnl::launch_pad_heads(q, h->q_pad, tokens, g.heads, h->cfg.d, elt, s);
+    if (e == cudaSuccess) e = srnl::launch_pad_heads(dy, h->dy_pad, tokens, g.heads, h->cfg.d, elt, s);
+    if (e != cudaSuccess) return seq_cuda_fail(h, e, "head padding launch");
+    qk = q != nullptr ? h->q_pad : h->x_pad;
+    x = h->x_pad;
+    dy = h->dy_pad;
+  }
+  const float* q32 = static_cast<const float*>(qk);
+  if (g.act_bf16) {  // the backward reads fp32 queries
+    float* qf = h->bws + srnl::backward_free_region(g);
+    e = srnl::launch_convert(qk, true, qf, tokens * g.C, s);
+    if (e != cudaSuccess) return seq_cuda_fail(h, e, "query conversion launch");
+    q32 = qf;
+  }
+  const srnl::ScanParamsDev p{nullptr, nullptr, h->G, h->Mm, h->scales};
+  e = srnl::launch_backward_scan(g, p, x, q32, dy, h->bws, s);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "backward scan launch");
+  srnl::BwdGrads out{};
+  if (grads != nullptr) out = srnl::BwdGrads{nullptr, grads->M_mem0, grads->M_k0, grads->M_v0, grads->m_eta0, grads->m_alpha0};
+  void* dxk = padded ? h->dx_pad : dx;
+  void* dqk = dq == nullptr ? nullptr : (padded ? h->dq_pad : dq);
+  e = srnl::launch_backward_seq_combine(g, h->cfg.d, h->bws, dxk, dqk, q == nullptr, out, s);
+  if (e != cudaSuccess) return seq_cuda_fail(h, e, "backward combine launch");
+  if (padded) {
+    e = srnl::launch_unpad_heads(h->dx_pad, dx, tokens, g.heads, h->cfg.d, elt, s);
+    if (e == cudaSuccess && dq != nullptr) e = srnl::launch_unpad_heads(h->dq_pad, dq, tokens, g.heads, h->cfg.d, elt, s);
     if (e != cudaSuccess) return seq_cuda_fail(h, e, "head unpadding launch");
   }
   return SRNL_OK;
