@@ -37,9 +37,9 @@ METRIC = "SRNL 4-dir scan tokens/s (fwd, 1xB200) and % of roofline at 56x56x64"
 
 # DRAM bytes (read + write) of one scan launch, from a 1-pass ncu capture of the current
 # chunkwise kernel on the full workload (profiles/scan_kernel_hier_s1_56x56_b4.md):
-# 29.02 MB read + 48.13 MB written.  Keyed by (workload, B, generation dtype); absent
+# 28.95 MB read + 48.37 MB written.  Keyed by (workload, B, generation dtype); absent
 # entries report null.
-SCAN_TRAFFIC_BYTES = {("hier_s1_56x56", 32, "bf16"): 29.02e6 + 48.13e6}
+SCAN_TRAFFIC_BYTES = {("hier_s1_56x56", 32, "bf16"): 28.95e6 + 48.37e6}
 UNIT = "route-tokens/s"
 DEFAULT_CONFIG = "hier_s1_56x56"
 L2_FLUSH_BYTES = 256 << 20

@@ -252,6 +252,14 @@ typedef struct {
 SRNL_API srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void* dx,
                                        const srnl_scan_grads* grads, void* stream);
 
+/* Self-test of the failure path of the bounded in-kernel waits: on the CURRENT device, runs
+ * the scan kernels' bounded mbarrier wait on a barrier that nothing completes, with a
+ * wall-time limit of wait_ms milliseconds (1..5000).  Returns SRNL_E_TIMEOUT when the wait
+ * gave up as designed (the expected result; the device and context stay usable),
+ * SRNL_OK if the wait wrongly completed, SRNL_E_INVAL for wait_ms out of range (no device
+ * work), SRNL_E_CUDA on a CUDA error.  Synchronous; the message is srnl_scan_last_error(NULL). */
+SRNL_API srnl_status srnl_selftest_wait_timeout(int wait_ms);
+
 /* Bytes of device workspace the handle holds (packed params excluded). */
 SRNL_API size_t srnl_scan_workspace_bytes(const srnl_scan* h);
 

@@ -34,7 +34,7 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_seq_create", "srnl_seq_forward", "srnl_seq_device_status", "srnl_seq_last_error",
             "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count",
             "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
-            "srnl_scan_backward", "srnl_seq_backward")
+            "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout")
 
 
 class SrnlError(RuntimeError):
@@ -123,12 +123,13 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_seq_cap_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
     lib.srnl_scan_backward.argtypes = [vp, vp, vp, vp, ctypes.POINTER(_Grads), vp]
     lib.srnl_seq_backward.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_SeqGrads), vp]
+    lib.srnl_selftest_wait_timeout.argtypes = [i]
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
                  "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_seq_create", "srnl_seq_forward",
                  "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count",
                  "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
-                 "srnl_scan_backward", "srnl_seq_backward"):
+                 "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -387,6 +388,12 @@ def srnl_seq_backward(h: SrnlSeq, x, dy, dx, q=None, dq=None, grads: Optional[Di
     h._check(load_library().srnl_seq_backward(h.handle, _ptr(x), _ptr(q), _ptr(dy), _ptr(dx), _ptr(dq),
                                               ctypes.byref(gs) if grads is not None else None, _stream(stream)),
              "srnl_seq_backward")
+
+
+def srnl_selftest_wait_timeout(wait_ms: int = 50) -> int:
+    """Run the bounded-wait self-test on the current device; returns the status code
+    (SRNL_E_TIMEOUT is the expected, passing result)."""
+    return int(load_library().srnl_selftest_wait_timeout(int(wait_ms)))
 
 
 def srnl_seq_device_status(h: SrnlSeq) -> None:

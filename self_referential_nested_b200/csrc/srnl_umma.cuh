@@ -14,7 +14,8 @@ namespace {
 
 constexpr int kStage = 64;                   // tokens staged per pass
 constexpr int kUmmaM = 128;                  // M of every tcgen05.mma issued here
-constexpr long long kWaitLimit = 1ll << 20;  // mbarrier polls before giving up
+constexpr long long kWaitLimit = 1ll << 20;              // mbarrier polls before giving up,
+constexpr unsigned long long kWaitNs = 2000000000ull;    // or 2 s of wall time, whichever first
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -62,9 +63,20 @@ __device__ __forceinline__ void mma_commit(unsigned long long* bar) {
 }
 
 // Bounded wait on an mbarrier phase; records a failure instead of hanging.
-__device__ __forceinline__ void mbar_wait(unsigned long long* bar, uint32_t phase, int* failed) {
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for `phase` of an mbarrier, bounded: after kWaitLimit polls or limit_ns of wall time
+// (the clock is read only once 256 polls have failed, so a normal wait never reads it) the
+// wait gives up and sets *failed, which later waits see and return at once.
+__device__ __forceinline__ void mbar_wait(unsigned long long* bar, uint32_t phase, int* failed,
+                                          unsigned long long limit_ns = kWaitNs) {
   uint32_t done = *reinterpret_cast<volatile int*>(failed);
   long long polls = 0;
+  unsigned long long t0 = 0;
   while (!done) {
     asm volatile(
         "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
@@ -72,9 +84,12 @@ __device__ __forceinline__ void mbar_wait(unsigned long long* bar, uint32_t phas
         : "=r"(done)
         : "r"(smem_u32(bar)), "r"(phase)
         : "memory");
-    if (!done && ++polls > kWaitLimit) {
-      *failed = 1;
-      break;
+    if (!done && (++polls & 255) == 0) {
+      if (polls == 256) t0 = global_ns();
+      if (polls > kWaitLimit || global_ns() - t0 > limit_ns) {
+        *failed = 1;
+        break;
+      }
     }
   }
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");

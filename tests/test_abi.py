@@ -145,3 +145,14 @@ def test_create_rejects_bad_injection_cap(lib):
     assert e.value.status == S.SRNL_E_INVAL
     assert lib.srnl_scan_cap_count(None, None) == S.SRNL_E_INVAL
     assert lib.srnl_seq_cap_count(None, None) == S.SRNL_E_INVAL
+
+
+def test_selftest_rejects_out_of_range_limits_before_cuda(lib):
+    for ms in (0, -1, 5001):
+        assert lib.srnl_selftest_wait_timeout(ms) == S.SRNL_E_INVAL
+        assert b"wait_ms" in lib.srnl_scan_last_error(None)
+
+
+def test_backward_null_arguments_fail_cleanly(lib):
+    assert lib.srnl_scan_backward(None, None, None, None, None, None) == S.SRNL_E_INVAL
+    assert lib.srnl_seq_backward(None, None, None, None, None, None, None, None) == S.SRNL_E_INVAL
