@@ -360,7 +360,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         "roofline": {"bound": "alu", "achieved": scan_tflops, "peak": fp32_peak_tflops,
                      "unit": "TFLOP/s", "frac": scan_tflops / fp32_peak_tflops,
                      "traffic": SCAN_TRAFFIC_BYTES.get((cfg.name, cfg.B, gen)), "traffic_unit": "bytes/launch",
-                     "kernel": "srnl_scan_chunkwise_kernel" if gen == "bf16" else "srnl_scan_sequential_kernel",
+                     "kernel": ("srnl_scan_d64_kernel" if cfg.d == 64 else
+                                "srnl_scan_chunkwise_kernel" if gen == "bf16" else "srnl_scan_sequential_kernel"),
                      "kernel_ms": scan_ms,
                      "peak_note": "fp32 FMA peak 148 SM x 128 lanes x 2 x sm_max_mhz (derived)"},
         "forward_roofline": {"bound": "hbm" if t_bytes_us >= t_tensor_us else "tensor",
@@ -589,6 +590,8 @@ def main():
     ap.add_argument("--cap", default="soft", choices=["soft", "hard"],
                     help="injection cap: the soft cap (the method) or the hard clamp of its ablation")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
+    ap.add_argument("--head-dim", type=int, default=0, choices=[0, 4, 8, 16, 32, 64],
+                    help="override the head dim (C = heads x d); 64 runs the fp32-generation path")
     ap.add_argument("--seq", action="store_true", help="time the standalone sequence layer instead")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (gradients of x and every parameter) instead")
@@ -601,6 +604,10 @@ def main():
     cfg = CONFIGS[args.config]
     if args.batch > 0:
         cfg = cfg.replace(B=args.batch)
+    if args.head_dim > 0:
+        cfg = cfg.replace(d=args.head_dim, C=cfg.heads * args.head_dim)
+        if args.head_dim == 64:
+            args.gen = "f32"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

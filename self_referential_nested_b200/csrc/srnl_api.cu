@@ -110,8 +110,10 @@ srnl_status validate_config(const srnl_scan_config* c) {
     return fail(nullptr, SRNL_E_INVAL, "B, H, W, C, heads and d must be positive");
   if ((int64_t)c->heads * c->d != c->C)
     return fail(nullptr, SRNL_E_INVAL, "C must equal heads * d");
-  if (c->d != 4 && c->d != 8 && c->d != 16 && c->d != srnl::kD)
-    return fail(nullptr, SRNL_E_UNSUPPORTED, "head dim d must be 4, 8, 16 or 32");
+  if (c->d != 4 && c->d != 8 && c->d != 16 && c->d != srnl::kD && c->d != 64)
+    return fail(nullptr, SRNL_E_UNSUPPORTED, "head dim d must be 4, 8, 16, 32 or 64");
+  if (c->d == 64 && c->gen_dtype == SRNL_BF16)
+    return fail(nullptr, SRNL_E_UNSUPPORTED, "head dim 64 is built for gen_dtype SRNL_F32");
   if (!(c->alpha > 0.f && c->alpha < 1.f))
     return fail(nullptr, SRNL_E_INVAL, "alpha must lie in (0, 1)");
   if (!(c->eps > 0.f) || !std::isfinite(c->eps))
@@ -177,9 +179,10 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
   if (e != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaGetDevice"); delete h; return st; }
 
   const srnl_scan_config& c = h->cfg;
-  // kernels run 32-wide heads; a smaller head dim is zero-padded to 32 (exact: the padded
-  // rows and columns of every memory and transition stay zero)
-  const int d = srnl::kD, ud = c.d, nh = c.heads, Cp = nh * d;
+  // kernels run 32-wide heads (64-wide for head dim 64); a smaller head dim is zero-padded to
+  // 32 (exact: the padded rows and columns of every memory and transition stay zero)
+  const int d = c.d == 64 ? 64 : srnl::kD, ud = c.d, nh = c.heads, Cp = nh * d;
+  const int gen = 2 * d + 2;   // generating rows: M_k, M_v, m_eta, m_alpha
   const bool padded = ud != d;
   srnl::ScanGeom& g = h->geom;
   g.B = c.B; g.H = c.H; g.W = c.W; g.C = Cp; g.heads = nh;
@@ -189,6 +192,7 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
   g.act_bf16 = c.act_dtype == SRNL_BF16;
   g.gen_bf16 = c.gen_dtype == SRNL_BF16;
   g.hard_cap = c.injection_cap == SRNL_CAP_HARD;
+  g.hd = d;
 
   // ---- pack parameters on the host, then upload
   std::vector<float> Wq((size_t)Cp * Cp, 0.f);
@@ -199,10 +203,10 @@ srnl_status srnl_scan_create(srnl_scan** out, const srnl_scan_config* cfg,
     }
   std::vector<__nv_bfloat16> Wqb(g.gen_bf16 ? Wq.size() : 0);
   for (size_t i = 0; i < Wqb.size(); ++i) Wqb[i] = __float2bfloat16_rn(Wq[i]);  // exact: already rounded
-  std::vector<float> G((size_t)4 * nh * srnl::kGen * d, 0.f), Mm((size_t)4 * nh * d * d, 0.f);
+  std::vector<float> G((size_t)4 * nh * gen * d, 0.f), Mm((size_t)4 * nh * d * d, 0.f);
   for (int r = 0; r < 4; ++r)
     for (int hh = 0; hh < nh; ++hh) {
-      float* dst = G.data() + ((size_t)r * nh + hh) * srnl::kGen * d;
+      float* dst = G.data() + ((size_t)r * nh + hh) * gen * d;
       float* mdst = Mm.data() + ((size_t)r * nh + hh) * d * d;
       const size_t mo = ((size_t)r * nh + hh) * ud * ud, vo = ((size_t)r * nh + hh) * ud;
       for (int i = 0; i < ud; ++i) {
@@ -266,7 +270,7 @@ static srnl_status run_forward(srnl_scan* h, const void* x, void* y, float* fina
   cudaError_t e;
   cudaEvent_t* ev = h->ring > 0 ? &h->ev[(size_t)(h->recorded % h->ring) * 4] : nullptr;
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
-  const bool padded = h->cfg.d != srnl::kD;
+  const bool padded = h->cfg.d < srnl::kD;
   const int elt = h->geom.act_bf16 ? 2 : 4;
   const int64_t tokens = (int64_t)h->geom.B * h->geom.H * h->geom.W;
   if (padded) {  // heads of d < 32 channels run as zero-padded 32-wide heads
@@ -348,7 +352,8 @@ srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void
   srnl_status st = check_device(h);
   if (st != SRNL_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool padded = h->cfg.d != srnl::kD;
+  if (h->cfg.d == 64) return fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for head dims up to 32");
+  const bool padded = h->cfg.d < srnl::kD;
   const int elt = h->geom.act_bf16 ? 2 : 4;
   const int64_t tokens = (int64_t)h->geom.B * h->geom.H * h->geom.W;
   cudaError_t e;

@@ -17,6 +17,7 @@ struct ScanGeom {
   bool act_bf16;     // x / y element type
   bool gen_bf16;     // generation + projection operands in bf16
   bool hard_cap = false;  // hard injection clamp instead of the soft cap
+  int hd = 32;       // kernel head width: 32 (heads of d <= 32, zero-padded) or 64
 };
 
 struct ScanParamsDev {
@@ -99,6 +100,12 @@ cudaError_t launch_backward_seq_combine(const ScanGeom& g, int ud, float* ws, vo
 // layer stages fp32 queries there).
 inline size_t backward_free_region(const ScanGeom& g) { BwdLayout l; backward_workspace_floats(g, &l); return l.dq; }
 cudaError_t prepare_backward_kernel();
+
+// Head dim 64, fp32 generation (SIMT); launch_scan dispatches to it when g.hd == 64.
+// finals: [routes][B][heads][3*64*64 + 2*64] or nullptr.
+cudaError_t launch_scan_d64(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q, float* yr,
+                            float* finals, unsigned long long* binds, cudaStream_t s);
+cudaError_t prepare_scan_d64_kernel();
 
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)
 cudaError_t prepare_scan_kernels();

@@ -417,6 +417,7 @@ cudaError_t prepare_scan_kernels() {
 
 cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
                         float* yr, float* finals, int* err, unsigned long long* binds, cudaStream_t s) {
+  if (g.hd == 64) return launch_scan_d64(g, p, x, q, yr, finals, binds, s);
   if (g.gen_bf16) return launch_scan_chunkwise(g, p, x, q, yr, finals, err, binds, s);
   Args a;
   a.x = x; a.q = q; a.yr = yr; a.finals = finals; a.err = err;

@@ -111,8 +111,10 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
   cudaError_t e = cudaGetDevice(&h->device);
   if (e != cudaSuccess) { st = seq_cuda_fail(nullptr, e, "cudaGetDevice"); delete h; return st; }
 
-  // kernels run 32-wide heads; a smaller head dim is zero-padded to 32 (exact)
-  const int d = srnl::kD, ud = cfg->d, nh = cfg->heads, Dp = nh * d;
+  // kernels run 32-wide heads (64-wide for head dim 64); a smaller head dim is zero-padded to
+  // 32 (exact)
+  const int d = cfg->d == 64 ? 64 : srnl::kD, ud = cfg->d, nh = cfg->heads, Dp = nh * d;
+  const int gen = 2 * d + 2;   // generating rows: M_k, M_v, m_eta, m_alpha
   const bool padded = ud != d;
   srnl::ScanGeom& g = h->geom;
   g.B = cfg->B; g.H = 1; g.W = cfg->T; g.C = Dp; g.heads = nh;
@@ -122,10 +124,11 @@ srnl_status srnl_seq_create(srnl_seq** out, const srnl_seq_config* cfg, const sr
   g.gen_bf16 = cfg->gen_dtype == SRNL_BF16;
   g.routes = 1;
   g.hard_cap = cfg->injection_cap == SRNL_CAP_HARD;
+  g.hd = d;
 
-  std::vector<float> G((size_t)nh * srnl::kGen * d, 0.f), Mm((size_t)nh * d * d, 0.f);
+  std::vector<float> G((size_t)nh * gen * d, 0.f), Mm((size_t)nh * d * d, 0.f);
   for (int hh = 0; hh < nh; ++hh) {
-    float* dst = G.data() + (size_t)hh * srnl::kGen * d;
+    float* dst = G.data() + (size_t)hh * gen * d;
     float* mdst = Mm.data() + (size_t)hh * d * d;
     const size_t mo = (size_t)hh * ud * ud, vo = (size_t)hh * ud;
     for (int i = 0; i < ud; ++i) {
@@ -188,7 +191,7 @@ srnl_status srnl_seq_forward(srnl_seq* h, const void* x, const void* q, void* y,
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "cudaGetDevice");
   if (cur != h->device) return seq_fail(h, SRNL_E_INVAL, "the current device is not the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool padded = h->cfg.d != srnl::kD;
+  const bool padded = h->cfg.d < srnl::kD;
   const int elt = g.act_bf16 ? 2 : 4;
   const int64_t tokens = (int64_t)g.B * g.W;
   const void* qk = q != nullptr ? q : x;
@@ -241,12 +244,13 @@ srnl_status srnl_seq_backward(srnl_seq* h, const void* x, const void* q, const v
       return seq_fail(h, SRNL_E_INVAL, "dx or dq overlaps an input");
   if (dq != nullptr && overlap(dx, dq, bytes)) return seq_fail(h, SRNL_E_INVAL, "dx and dq overlap");
   if (g.gen_bf16) return seq_fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for gen_dtype SRNL_F32 handles");
+  if (h->cfg.d == 64) return seq_fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for head dims up to 32");
   int cur = -1;
   cudaError_t e = cudaGetDevice(&cur);
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "cudaGetDevice");
   if (cur != h->device) return seq_fail(h, SRNL_E_INVAL, "the current device is not the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool padded = h->cfg.d != srnl::kD;
+  const bool padded = h->cfg.d < srnl::kD;
   const int elt = g.act_bf16 ? 2 : 4;
   const int64_t tokens = (int64_t)g.B * g.W;
   const size_t pbytes = (size_t)tokens * g.C * elt;

@@ -1,0 +1,125 @@
+"""GPU parity at head dim 64 (the fp32-generation path, 64-wide SIMT kernel) through both ABIs
+against the float64 oracle.  Tolerances: 1e-4 relative Frobenius error with fp32 activations,
+2e-2 when x and y are bf16 (as for the other paths)."""
+import numpy as np
+import pytest
+import torch
+
+import self_referential_nested_b200 as S
+from oracle import srnl_oracle as O
+from srnl_inputs import ScanConfig, bf16_round_bits, make_inputs, make_seq_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from self_referential_nested_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+
+
+def _dev(a32, act):
+    if act == "bf16":
+        return torch.from_numpy(bf16_round_bits(a32).view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a32, dtype=np.float32)).cuda()
+
+
+def _cfg(name, **kw):
+    base = dict(name=name, B=2, H=6, W=10, C=128, heads=2, d=64, alpha=0.95, act_dtype="f32")
+    base.update(kw)
+    return ScanConfig(**base)
+
+
+def run_operator(cfg, cap="soft", seed=0, mem_scale=0.02, vec_scale=0.1, finals=True):
+    inp = make_inputs(cfg, seed=seed, mem_scale=mem_scale, vec_scale=vec_scale)
+    act = cfg.act_dtype
+    h = S.srnl_scan_create(dict(B=cfg.B, H=cfg.H, W=cfg.W, C=cfg.C, heads=cfg.heads, d=cfg.d, alpha=cfg.alpha,
+                                eps=cfg.eps, chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, act_dtype=act,
+                                gen_dtype="f32", injection_cap=cap), inp.params())
+    try:
+        x = _dev(inp.x32, act)
+        y = torch.full_like(x, float("nan"))
+        nst = 3 * cfg.d * cfg.d + 2 * cfg.d
+        fin = torch.full((4, cfg.B, cfg.heads, nst), float("nan"), device="cuda") if finals else None
+        S.srnl_scan_forward(h, x, y, fin)
+        torch.cuda.synchronize()
+        count = S.srnl_scan_cap_count(h) if cap == "hard" else None
+    finally:
+        h.close()
+    counter = [0]
+    ref, ref_fin, _ = O.operator_forward(inp.x32, inp.params(), alpha_max=cfg.alpha, eps=cfg.eps,
+                                         chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, heads=cfg.heads,
+                                         cap=cap, counter=counter)
+    tol = 1e-4 if act == "f32" else 2e-2
+    err = O.rel_fro(y.float().cpu().numpy(), ref)
+    assert err <= tol, f"y: relative Frobenius error {err:.3e} > {tol:.0e}"
+    if finals:
+        ferr = O.rel_fro(fin.cpu().numpy(), ref_fin)
+        assert ferr <= 1e-4, f"final states: relative Frobenius error {ferr:.3e}"
+    return count, counter[0]
+
+
+def test_d64_operator_f32_ragged_chunks():
+    run_operator(_cfg("d64", chunk_row=4, chunk_col=0), seed=1)
+
+
+def test_d64_operator_bf16_activations():
+    run_operator(_cfg("d64b", B=2, H=7, W=9, act_dtype="bf16"), seed=2)
+
+
+def test_d64_operator_long_chunks_span_segments():
+    # 200 tokens per route at alpha_t ~ 0.5: the final states (~1e-60) lie below the fp32 range,
+    # so only the outputs are compared here (the other cases compare the states)
+    run_operator(_cfg("d64l", B=1, H=2, W=100), seed=3, finals=False)
+
+
+def test_d64_operator_one_head():
+    run_operator(_cfg("d64h1", C=64, heads=1, H=5, W=8), seed=4)
+
+
+def test_d64_operator_hard_clamp_and_count():
+    got, expect = run_operator(_cfg("d64hard", chunk_row=5, chunk_col=3), cap="hard", seed=5, mem_scale=0.2,
+                               vec_scale=0.6)
+    assert expect > 0
+    assert abs(got - expect) <= 0.001 * 4 * 2 * 2 * 60 + 2
+
+
+def test_d64_operator_56x56_shape():
+    run_operator(_cfg("d64s1", B=2, H=56, W=56), seed=6, finals=False)
+
+
+@pytest.mark.parametrize("queries", [True, False])
+def test_d64_sequence_layer(queries):
+    B, T, D, heads = 2, 130, 128, 2
+    si = make_seq_inputs(B, T, D, heads, "f32", seed=7)
+    h = S.srnl_seq_create(dict(B=B, T=T, D=D, heads=heads, d=64, alpha=0.95, eps=1e-6, chunk=0, act_dtype="f32",
+                               gen_dtype="f32"), si.params())
+    try:
+        x = _dev(si.x32, "f32")
+        q = _dev(si.q32, "f32") if queries else None
+        y = torch.full_like(x, float("nan"))
+        S.srnl_seq_forward(h, x, y, q=q)
+        torch.cuda.synchronize()
+    finally:
+        h.close()
+    ref, _ = O.sequence_forward(si.x32, si.params(), alpha_max=0.95, chunk=64, heads=heads,
+                                queries=si.q32 if queries else None)
+    err = O.rel_fro(y.cpu().numpy(), ref)
+    assert err <= 1e-4, f"relative Frobenius error {err:.3e}"
+
+
+def test_d64_backward_is_unsupported():
+    cfg = _cfg("d64bwd")
+    inp = make_inputs(cfg, seed=0)
+    h = S.srnl_scan_create(dict(B=2, H=6, W=10, C=128, heads=2, d=64, alpha=0.95, act_dtype="f32",
+                                gen_dtype="f32"), inp.params())
+    try:
+        x = _dev(inp.x32, "f32")
+        with pytest.raises(S.SrnlError) as ei:
+            S.srnl_scan_backward(h, x, x.clone(), torch.empty_like(x))
+        assert ei.value.status == S.SRNL_E_UNSUPPORTED
+    finally:
+        h.close()
