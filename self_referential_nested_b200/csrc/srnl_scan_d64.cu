@@ -12,8 +12,9 @@
 // chunk's tokens; each row of Q is then written in token order, row <- alpha_t row -
 // eta_t (row . u_t) k_t, and the readout is y_t = M_mem0 (Q_t q_t).
 //
-// One CTA per (route, batch, head) sequence, 256 threads.  Thread (row i = tid / 4, columns
-// 16 (tid % 4) .. +15) of Q: the write is row-local, so the token loop needs no block
+// One CTA per (route, batch, head) sequence, 256 threads.  Thread (row i = tid / 4) of Q owns the
+// columns 16 m + 4 (tid % 4) + e (m, e = 0..3): the four lanes of a row read the shared token
+// vectors at distinct banks.  The write is row-local, so the token loop needs no block
 // barrier.  Per segment of up to kSeg tokens of a chunk: x and q staged block-wide;
 // generation and the vector reductions with a warp per token; the scalar gates with a lane
 // per token; the token loop (which also forms z_t = Q_t q_t); then the readout
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(kThreads64, 2) srnl_scan_d64_kernel(const Args
   Smem64& sm = *reinterpret_cast<Smem64*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ri = tid >> 2;            // row of Q owned
-  const int c0 = (tid & 3) * 16;      // first of the 16 columns owned
+  const int c0 = (tid & 3) * 4;       // columns owned: 16 m + c0 + e, m, e = 0..3
   const int seq = blockIdx.x;         // ((r * B + b) * heads + h)
   const int hh = seq % A.heads;
   const int b = (seq / A.heads) % A.B;
@@ -118,16 +119,16 @@ __global__ void __launch_bounds__(kThreads64, 2) srnl_scan_d64_kernel(const Args
   for (int i = tid; i < kGen64 * kD64; i += kThreads64) sm.Gm[i / kD64][i % kD64] = A.G[(size_t)rh * kGen64 * kD64 + i];
   const float sc0 = A.scales[(size_t)r * C + ch0 + lane], sc1 = A.scales[(size_t)r * C + ch0 + 32 + lane];
 
-  float Q[16];
+  float Q[16];   // Q[4 m + e] = Q[ri][16 m + c0 + e]
 #pragma unroll
-  for (int c = 0; c < 16; ++c) Q[c] = (ri == c0 + c) ? 1.f : 0.f;
+  for (int c = 0; c < 16; ++c) Q[c] = (ri == 16 * (c >> 2) + c0 + (c & 3)) ? 1.f : 0.f;
 
   for (int c = 0; c < nc; ++c) {
     const int t0c = c * L, Lc = min(L, N - t0c);
     __syncthreads();
 #pragma unroll
     for (int cc = 0; cc < 16; cc += 4)
-      *reinterpret_cast<float4*>(&sm.Qb[ri][c0 + cc]) = make_float4(Q[cc], Q[cc + 1], Q[cc + 2], Q[cc + 3]);
+      *reinterpret_cast<float4*>(&sm.Qb[ri][4 * cc + c0]) = make_float4(Q[cc], Q[cc + 1], Q[cc + 2], Q[cc + 3]);
     for (int s0 = 0; s0 < Lc; s0 += kSeg64) {
       const int T = min(kSeg64, Lc - s0);
       const int t0 = t0c + s0;
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(kThreads64, 2) srnl_scan_d64_kernel(const Args
         float pr = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 16; cc += 4) {
-          const float4 u = *reinterpret_cast<const float4*>(rc + kRu + c0 + cc);
+          const float4 u = *reinterpret_cast<const float4*>(rc + kRu + 4 * cc + c0);
           pr = fmaf(Q[cc], u.x, pr);
           pr = fmaf(Q[cc + 1], u.y, pr);
           pr = fmaf(Q[cc + 2], u.z, pr);
@@ -199,8 +200,8 @@ __global__ void __launch_bounds__(kThreads64, 2) srnl_scan_d64_kernel(const Args
         float z = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 16; cc += 4) {
-          const float4 k = *reinterpret_cast<const float4*>(rc + kRk + c0 + cc);
-          const float4 qq = *reinterpret_cast<const float4*>(&sm.qv[tt][c0 + cc]);
+          const float4 k = *reinterpret_cast<const float4*>(rc + kRk + 4 * cc + c0);
+          const float4 qq = *reinterpret_cast<const float4*>(&sm.qv[tt][4 * cc + c0]);
           Q[cc] = fmaf(al, Q[cc], -ep * k.x);
           Q[cc + 1] = fmaf(al, Q[cc + 1], -ep * k.y);
           Q[cc + 2] = fmaf(al, Q[cc + 2], -ep * k.z);
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(kThreads64, 2) srnl_scan_d64_kernel(const Args
   __syncthreads();
 #pragma unroll
   for (int cc = 0; cc < 16; cc += 4)
-    *reinterpret_cast<float4*>(&sm.Qb[ri][c0 + cc]) = make_float4(Q[cc], Q[cc + 1], Q[cc + 2], Q[cc + 3]);
+    *reinterpret_cast<float4*>(&sm.Qb[ri][4 * cc + c0]) = make_float4(Q[cc], Q[cc + 1], Q[cc + 2], Q[cc + 3]);
   __syncthreads();
   float* fo = A.finals + (size_t)seq * (3 * kD64 * kD64 + 2 * kD64);
   const int nrows = kD64 + kGen64;   // M_mem rows, then the 130 generating rows
