@@ -591,7 +591,7 @@ def main():
                     help="injection cap: the soft cap (the method) or the hard clamp of its ablation")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
     ap.add_argument("--head-dim", type=int, default=0, choices=[0, 4, 8, 16, 32, 64],
-                    help="override the head dim (C = heads x d); 64 runs the fp32-generation path")
+                    help="override the head dim (C = heads x d); 64 defaults to the fp32-generation path")
     ap.add_argument("--seq", action="store_true", help="time the standalone sequence layer instead")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (gradients of x and every parameter) instead")
@@ -606,7 +606,7 @@ def main():
         cfg = cfg.replace(B=args.batch)
     if args.head_dim > 0:
         cfg = cfg.replace(d=args.head_dim, C=cfg.heads * args.head_dim)
-        if args.head_dim == 64:
+        if args.head_dim == 64 and args.gen is None:
             args.gen = "f32"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

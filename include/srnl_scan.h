@@ -100,9 +100,9 @@ typedef enum { SRNL_CAP_SOFT = 0, SRNL_CAP_HARD = 1 } srnl_cap;
 typedef struct {
   int B, H, W, C; /* batch, height, width, channels (C = heads * d) */
   int heads, d;   /* heads and head dim: 4, 8, 16, 32 or 64 (below 32 the heads run zero-padded
-                     to 32 lanes, which is exact; 64 runs 64-wide fp32 SIMT kernels and needs
-                     gen_dtype SRNL_F32, and has no backward; the no-allocation forward takes 32
-                     only) */
+                     to 32 lanes, which is exact; 64 runs a 64-wide SIMT kernel, fp32 products
+                     with the bf16 path's roundings when gen_dtype is SRNL_BF16, and has no
+                     backward; the no-allocation forward takes 32 only) */
   float alpha;    /* retention cap, 0 < alpha < 1 (0.95 hierarchical, 0.9 plain) */
   float eps;      /* key normalisation epsilon, > 0 (1e-6) */
   int chunk_row;  /* chunk length on routes 0/1; 0 means W (full rows) */

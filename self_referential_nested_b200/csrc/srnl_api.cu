@@ -112,8 +112,6 @@ srnl_status validate_config(const srnl_scan_config* c) {
     return fail(nullptr, SRNL_E_INVAL, "C must equal heads * d");
   if (c->d != 4 && c->d != 8 && c->d != 16 && c->d != srnl::kD && c->d != 64)
     return fail(nullptr, SRNL_E_UNSUPPORTED, "head dim d must be 4, 8, 16, 32 or 64");
-  if (c->d == 64 && c->gen_dtype == SRNL_BF16)
-    return fail(nullptr, SRNL_E_UNSUPPORTED, "head dim 64 is built for gen_dtype SRNL_F32");
   if (!(c->alpha > 0.f && c->alpha < 1.f))
     return fail(nullptr, SRNL_E_INVAL, "alpha must lie in (0, 1)");
   if (!(c->eps > 0.f) || !std::isfinite(c->eps))

@@ -101,7 +101,7 @@ cudaError_t launch_backward_seq_combine(const ScanGeom& g, int ud, float* ws, vo
 inline size_t backward_free_region(const ScanGeom& g) { BwdLayout l; backward_workspace_floats(g, &l); return l.dq; }
 cudaError_t prepare_backward_kernel();
 
-// Head dim 64, fp32 generation (SIMT); launch_scan dispatches to it when g.hd == 64.
+// Head dim 64 (SIMT, both precision paths); launch_scan dispatches to it when g.hd == 64.
 // finals: [routes][B][heads][3*64*64 + 2*64] or nullptr.
 cudaError_t launch_scan_d64(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q, float* yr,
                             float* finals, unsigned long long* binds, cudaStream_t s);

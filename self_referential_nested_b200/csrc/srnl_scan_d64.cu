@@ -1,4 +1,4 @@
-// SRNL four-direction chunked scan for head dim 64, fp32-generation path (sm_100a).
+// SRNL four-direction chunked scan for head dim 64 (sm_100a), both precision paths.
 //
 // Method sources (web pages on VisionHOPE; no page prints an equation): "VisionHOPE" README,
 // "SRNL and VisionHOPE operator" (head_dim up to 64); "VisionHOPE: Visual Backbones as
@@ -19,7 +19,10 @@
 // generation and the vector reductions with a warp per token; the scalar gates with a lane
 // per token; the token loop (which also forms z_t = Q_t q_t); then the readout
 // y_t = M_mem0 z_t with a warp per token, scaled by the route's fusion scales and stored
-// at the token's raster position.  All arithmetic is fp32 (SIMT).
+// at the token's raster position.  All arithmetic is fp32 (SIMT).  With bf16 generation the
+// kernel applies that path's roundings: x, the boundary products w = Q_b x and G are rounded
+// to bf16 before the generation product, and q arrives in bf16; the write and the readout
+// stay fp32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -56,7 +59,7 @@ static_assert(sizeof(Smem64) <= 112 * 1024, "two CTAs per SM");
 
 struct Args64 {
   const void* x;     // [B][N][C] act dtype (C = heads * 64)
-  const float* q;    // [B][N][C] fp32
+  const void* q;     // [B][N][C] fp32, or bf16 with bf16 generation
   float* yr;         // [routes][B*N][C] scaled route partials at raster positions
   float* finals;     // [routes][B][heads][3*64*64 + 2*64] or nullptr
   unsigned long long* binds;
@@ -65,7 +68,7 @@ struct Args64 {
   const float* scales;
   int B, H, W, C, heads, Lrow, Lcol;
   float alpha, eps;
-  bool act_bf16, hard_cap;
+  bool act_bf16, gen_bf16, hard_cap;
 };
 
 // Dot product of a 16-byte-aligned shared row with a broadcast shared vector, n a multiple of
@@ -116,7 +119,10 @@ __global__ void __launch_bounds__(kThreads64, 2) srnl_scan_d64_kernel(const Args
   const int rh = r * A.heads + hh;
 
   for (int i = tid; i < kD64 * kD64; i += kThreads64) sm.Mm[i / kD64][i % kD64] = A.Mm[(size_t)rh * kD64 * kD64 + i];
-  for (int i = tid; i < kGen64 * kD64; i += kThreads64) sm.Gm[i / kD64][i % kD64] = A.G[(size_t)rh * kGen64 * kD64 + i];
+  for (int i = tid; i < kGen64 * kD64; i += kThreads64) {
+    const float gv = A.G[(size_t)rh * kGen64 * kD64 + i];
+    sm.Gm[i / kD64][i % kD64] = A.gen_bf16 ? round_bf16(gv) : gv;
+  }
   const float sc0 = A.scales[(size_t)r * C + ch0 + lane], sc1 = A.scales[(size_t)r * C + ch0 + 32 + lane];
 
   float Q[16];   // Q[4 m + e] = Q[ri][16 m + c0 + e]
@@ -136,14 +142,17 @@ __global__ void __launch_bounds__(kThreads64, 2) srnl_scan_d64_kernel(const Args
       for (int idx = tid; idx < T * kD64; idx += kThreads64) {
         const int tt = idx / kD64, j = idx % kD64;
         const int64_t o = (tokbase + route_pos(r, t0 + tt, A.H, A.W)) * C + ch0 + j;
-        sm.xs[tt][j] = load_act64(A.x, o, A.act_bf16);
-        sm.qv[tt][j] = A.q[o];
+        const float xv = load_act64(A.x, o, A.act_bf16);
+        sm.xs[tt][j] = A.gen_bf16 ? round_bf16(xv) : xv;
+        sm.qv[tt][j] = load_act64(A.q, o, A.gen_bf16);
       }
       __syncthreads();
       // generation and the vector reductions (warp per token; lane covers j and 32 + j)
       for (int tt = warp; tt < T; tt += kWarps64) {
-        sm.wh[warp][lane] = dot64<kD64>(sm.Qb[lane], sm.xs[tt]);           // w = Q_b x
-        sm.wh[warp][32 + lane] = dot64<kD64>(sm.Qb[32 + lane], sm.xs[tt]);
+        const float w0 = dot64<kD64>(sm.Qb[lane], sm.xs[tt]);              // w = Q_b x
+        const float w1 = dot64<kD64>(sm.Qb[32 + lane], sm.xs[tt]);
+        sm.wh[warp][lane] = A.gen_bf16 ? round_bf16(w0) : w0;
+        sm.wh[warp][32 + lane] = A.gen_bf16 ? round_bf16(w1) : w1;
         __syncwarp();
         const float k0 = dot64<kD64>(sm.Gm[lane], sm.wh[warp]);
         const float k1 = dot64<kD64>(sm.Gm[32 + lane], sm.wh[warp]);
@@ -254,10 +263,10 @@ cudaError_t prepare_scan_d64_kernel() {
 cudaError_t launch_scan_d64(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q, float* yr,
                             float* finals, unsigned long long* binds, cudaStream_t s) {
   Args64 a;
-  a.x = x; a.q = static_cast<const float*>(q); a.yr = yr; a.finals = finals; a.binds = binds;
+  a.x = x; a.q = q; a.yr = yr; a.finals = finals; a.binds = binds;
   a.G = p.G; a.Mm = p.Mm; a.scales = p.scales;
   a.B = g.B; a.H = g.H; a.W = g.W; a.C = g.C; a.heads = g.heads; a.Lrow = g.Lrow; a.Lcol = g.Lcol;
-  a.alpha = g.alpha; a.eps = g.eps; a.act_bf16 = g.act_bf16; a.hard_cap = g.hard_cap;
+  a.alpha = g.alpha; a.eps = g.eps; a.act_bf16 = g.act_bf16; a.gen_bf16 = g.gen_bf16; a.hard_cap = g.hard_cap;
   const unsigned nseq = (unsigned)g.routes * (unsigned)g.B * (unsigned)g.heads;
   srnl_scan_d64_kernel<<<nseq, kThreads64, sizeof(Smem64), s>>>(a);
   return cudaGetLastError();

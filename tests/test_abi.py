@@ -62,7 +62,6 @@ def _cfg_dict(cfg, **kw):
     (dict(eps=float("inf")), S.SRNL_E_INVAL),
     (dict(chunk_row=-2), S.SRNL_E_INVAL),
     (dict(act_dtype=7), S.SRNL_E_INVAL),
-    (dict(C=128, heads=2, d=64, act_dtype="bf16", gen_dtype="bf16"), S.SRNL_E_UNSUPPORTED),
     (dict(C=256, heads=2, d=128), S.SRNL_E_UNSUPPORTED),
     (dict(C=24, heads=2, d=12), S.SRNL_E_UNSUPPORTED),
 ])
@@ -117,7 +116,6 @@ def _seq_cfg(**kw):
     (dict(eps=0.0), S.SRNL_E_INVAL),
     (dict(chunk=-1), S.SRNL_E_INVAL),
     (dict(gen_dtype=5), S.SRNL_E_INVAL),
-    (dict(D=128, heads=2, d=64, gen_dtype="bf16"), S.SRNL_E_UNSUPPORTED),
     (dict(D=256, heads=2, d=128), S.SRNL_E_UNSUPPORTED),
 ])
 def test_seq_create_rejects_bad_config_before_cuda(lib, bad, status):

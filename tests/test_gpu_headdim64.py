@@ -1,6 +1,6 @@
-"""GPU parity at head dim 64 (the fp32-generation path, 64-wide SIMT kernel) through both ABIs
-against the float64 oracle.  Tolerances: 1e-4 relative Frobenius error with fp32 activations,
-2e-2 when x and y are bf16 (as for the other paths)."""
+"""GPU parity at head dim 64 (64-wide SIMT kernel) through both ABIs against the float64
+oracle.  Tolerances as for the other paths: 1e-4 relative Frobenius error on the fp32 path,
+2e-2 whenever bf16 enters (bf16 activations or the bf16 generation path's roundings)."""
 import numpy as np
 import pytest
 import torch
@@ -33,12 +33,12 @@ def _cfg(name, **kw):
     return ScanConfig(**base)
 
 
-def run_operator(cfg, cap="soft", seed=0, mem_scale=0.02, vec_scale=0.1, finals=True):
+def run_operator(cfg, cap="soft", seed=0, mem_scale=0.02, vec_scale=0.1, finals=True, gen="f32"):
     inp = make_inputs(cfg, seed=seed, mem_scale=mem_scale, vec_scale=vec_scale)
     act = cfg.act_dtype
     h = S.srnl_scan_create(dict(B=cfg.B, H=cfg.H, W=cfg.W, C=cfg.C, heads=cfg.heads, d=cfg.d, alpha=cfg.alpha,
                                 eps=cfg.eps, chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, act_dtype=act,
-                                gen_dtype="f32", injection_cap=cap), inp.params())
+                                gen_dtype=gen, injection_cap=cap), inp.params())
     try:
         x = _dev(inp.x32, act)
         y = torch.full_like(x, float("nan"))
@@ -53,12 +53,12 @@ def run_operator(cfg, cap="soft", seed=0, mem_scale=0.02, vec_scale=0.1, finals=
     ref, ref_fin, _ = O.operator_forward(inp.x32, inp.params(), alpha_max=cfg.alpha, eps=cfg.eps,
                                          chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, heads=cfg.heads,
                                          cap=cap, counter=counter)
-    tol = 1e-4 if act == "f32" else 2e-2
+    tol = 1e-4 if (act == "f32" and gen == "f32") else 2e-2
     err = O.rel_fro(y.float().cpu().numpy(), ref)
     assert err <= tol, f"y: relative Frobenius error {err:.3e} > {tol:.0e}"
     if finals:
         ferr = O.rel_fro(fin.cpu().numpy(), ref_fin)
-        assert ferr <= 1e-4, f"final states: relative Frobenius error {ferr:.3e}"
+        assert ferr <= (1e-4 if gen == "f32" else 2e-2), f"final states: relative Frobenius error {ferr:.3e}"
     return count, counter[0]
 
 
@@ -68,6 +68,11 @@ def test_d64_operator_f32_ragged_chunks():
 
 def test_d64_operator_bf16_activations():
     run_operator(_cfg("d64b", B=2, H=7, W=9, act_dtype="bf16"), seed=2)
+
+
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+def test_d64_operator_bf16_generation(act):
+    run_operator(_cfg("d64g", B=2, H=7, W=11, chunk_row=4, act_dtype=act), seed=8, gen="bf16")
 
 
 def test_d64_operator_long_chunks_span_segments():
@@ -91,15 +96,16 @@ def test_d64_operator_56x56_shape():
     run_operator(_cfg("d64s1", B=2, H=56, W=56), seed=6, finals=False)
 
 
-@pytest.mark.parametrize("queries", [True, False])
-def test_d64_sequence_layer(queries):
+@pytest.mark.parametrize("queries,gen", [(True, "f32"), (False, "f32"), (True, "bf16")])
+def test_d64_sequence_layer(queries, gen):
     B, T, D, heads = 2, 130, 128, 2
-    si = make_seq_inputs(B, T, D, heads, "f32", seed=7)
-    h = S.srnl_seq_create(dict(B=B, T=T, D=D, heads=heads, d=64, alpha=0.95, eps=1e-6, chunk=0, act_dtype="f32",
-                               gen_dtype="f32"), si.params())
+    act = gen
+    si = make_seq_inputs(B, T, D, heads, act, seed=7)
+    h = S.srnl_seq_create(dict(B=B, T=T, D=D, heads=heads, d=64, alpha=0.95, eps=1e-6, chunk=0, act_dtype=act,
+                               gen_dtype=gen), si.params())
     try:
-        x = _dev(si.x32, "f32")
-        q = _dev(si.q32, "f32") if queries else None
+        x = _dev(si.x32, act)
+        q = _dev(si.q32, act) if queries else None
         y = torch.full_like(x, float("nan"))
         S.srnl_seq_forward(h, x, y, q=q)
         torch.cuda.synchronize()
@@ -107,8 +113,9 @@ def test_d64_sequence_layer(queries):
         h.close()
     ref, _ = O.sequence_forward(si.x32, si.params(), alpha_max=0.95, chunk=64, heads=heads,
                                 queries=si.q32 if queries else None)
-    err = O.rel_fro(y.cpu().numpy(), ref)
-    assert err <= 1e-4, f"relative Frobenius error {err:.3e}"
+    err = O.rel_fro(y.float().cpu().numpy(), ref)
+    tol = 1e-4 if gen == "f32" else 2e-2
+    assert err <= tol, f"relative Frobenius error {err:.3e}"
 
 
 def test_d64_backward_is_unsupported():
