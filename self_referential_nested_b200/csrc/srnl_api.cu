@@ -350,7 +350,6 @@ srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void
   srnl_status st = check_device(h);
   if (st != SRNL_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (h->cfg.d == 64) return fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for head dims up to 32");
   const bool padded = h->cfg.d < srnl::kD;
   const int elt = h->geom.act_bf16 ? 2 : 4;
   const int64_t tokens = (int64_t)h->geom.B * h->geom.H * h->geom.W;

@@ -195,6 +195,7 @@ cudaError_t prepare_kernels() {
   cudaError_t e = prepare_scan_kernels();
   if (e != cudaSuccess) return e;
   if ((e = prepare_backward_kernel()) != cudaSuccess) return e;
+  if ((e = prepare_backward64_kernel()) != cudaSuccess) return e;
   if ((e = prepare_scan_d64_kernel()) != cudaSuccess) return e;
   return prepare_projection_kernel();
 }

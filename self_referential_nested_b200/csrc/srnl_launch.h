@@ -76,6 +76,9 @@ struct BwdGrads {      // device outputs in the caller's (unpadded) layouts; nul
 struct BwdLayout {     // float offsets of the backward workspace
   size_t dxr, dqr, dq, parts, ckpt, qs, grec, dwq, total;
   int max_chunks, Lmax, nsplit;
+  int hd;              // head width of the kernels (32 or 64)
+  int rec;             // floats per token gate record (2 hd + 8)
+  size_t seq_part;     // floats of parameter partials per sequence: hd^2 + (2 hd + 2) hd + hd
 };
 // Floats of backward workspace for the geometry (and the layout when lay != nullptr).
 size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay);
@@ -100,6 +103,10 @@ cudaError_t launch_backward_seq_combine(const ScanGeom& g, int ud, float* ws, vo
 // layer stages fp32 queries there).
 inline size_t backward_free_region(const ScanGeom& g) { BwdLayout l; backward_workspace_floats(g, &l); return l.dq; }
 cudaError_t prepare_backward_kernel();
+// The 64-wide reverse scan (head dim 64); launch_backward_scan dispatches to it when g.hd == 64.
+cudaError_t launch_backward_scan64(const ScanGeom& g, const ScanParamsDev& p, const void* x, const float* q,
+                                   const void* dy, float* ws, const BwdLayout& l, cudaStream_t s);
+cudaError_t prepare_backward64_kernel();
 
 // Head dim 64 (SIMT, both precision paths); launch_scan dispatches to it when g.hd == 64.
 // finals: [routes][B][heads][3*64*64 + 2*64] or nullptr.

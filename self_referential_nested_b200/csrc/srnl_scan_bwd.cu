@@ -39,11 +39,14 @@
 
 #include <algorithm>
 
+#include "srnl_bwd_common.cuh"
 #include "srnl_common.cuh"
 #include "srnl_launch.h"
 
 namespace srnl {
 namespace {
+
+using bwd::load_act;
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -98,32 +101,6 @@ struct BwdArgs {
   float alpha, eps;
   bool act_bf16, hard_cap;
 };
-
-__device__ __forceinline__ float load_act(const void* base, int64_t idx, bool bf16) {
-  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
-  return reinterpret_cast<const float*>(base)[idx];
-}
-
-__device__ __forceinline__ float sigmoid_f(float z) {
-  const float e = expf(-fabsf(z));
-  return z >= 0.f ? 1.f / (1.f + e) : e / (1.f + e);
-}
-
-__device__ __forceinline__ float softplus_f(float z) { return fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))); }
-
-// phi(z) = tanh(z) / z, by 1 - z^2/3 below 1e-4.
-__device__ __forceinline__ float phi_f(float z) { return z < 1e-4f ? 1.f - z * z * (1.f / 3.f) : tanhf(z) / z; }
-
-// phi'(z): the Taylor series -2z/3 + 8z^3/15 - 102z^5/315 + 496z^7/2835 of the derivative of
-// tanh(z)/z below 0.25 (where the closed form cancels in fp32), else (z (1 - tanh^2 z) - tanh z) / z^2.
-__device__ __forceinline__ float dphi_f(float z) {
-  if (z < 0.25f) {
-    const float z2 = z * z;
-    return z * (-2.f / 3.f + z2 * (8.f / 15.f + z2 * (-102.f / 315.f + z2 * (496.f / 2835.f))));
-  }
-  const float t = tanhf(z);
-  return (z * (1.f - t * t) - t) / (z * z);
-}
 
 __device__ __forceinline__ float row8_sum(float v) {   // sum over the 8 lanes of a matrix row
   v += __shfl_xor_sync(0xffffffffu, v, 1);
@@ -183,20 +160,6 @@ __device__ __forceinline__ void block_copy4(float* dst, const float* src, int n4
     reinterpret_cast<float4*>(dst)[i] = reinterpret_cast<const float4*>(src)[i];
 }
 
-// Scalar gates of one token from |k|^2, |k - v|^2, a and beta (accurate math functions; the
-// forward's clamp decisions): alpha_t and eta.
-__device__ __forceinline__ void gate_scalars_f(float kn2, float ne2, float a, float beta, const BwdArgs& A,
-                                               float& al, float& eta) {
-  const float gain = sqrtf(ne2) * sqrtf(kn2);
-  al = fminf(sigmoid_f(beta), A.alpha);
-  const float eta0 = softplus_f(a);
-  const float m = 1.f - al;
-  float eta1;
-  if (A.hard_cap) eta1 = (eta0 * gain > m) ? m / gain : eta0;
-  else eta1 = eta0 * phi_f(eta0 * gain / m);
-  eta = (eta1 * kn2 > 2.f) ? 2.f / kn2 : eta1;
-}
-
 // Gates of tokens [t0, t0 + T) of the sequence into sm.rec (T <= kSeg), by all threads:
 // the segment's x staged block-wide (over sx and sq), generation and the vector reductions
 // with a warp per token, the scalar gates with a lane per token, then u = (1 + alpha) k - v.
@@ -233,7 +196,7 @@ __device__ void gates_segment(BwdSmem& sm, const BwdArgs& A, int r, int64_t tokb
   if (tid < T) {
     float* rc = sm.rec[tid];
     float al, eta;
-    gate_scalars_f(rc[kRkn2], rc[kRne2], rc[kRa], rc[kRb], A, al, eta);
+    bwd::gate_scalars_f(rc[kRkn2], rc[kRne2], rc[kRa], rc[kRb], A.alpha, A.hard_cap, al, eta);
     rc[kRal] = al;
     rc[kReta] = eta;
   }
@@ -243,43 +206,6 @@ __device__ void gates_segment(BwdSmem& sm, const BwdArgs& A, int r, int64_t tokb
     rc[kRu + lane] = (1.f + rc[kRal]) * rc[kRk + lane] - rc[kRu + lane];
   }
   __syncthreads();
-}
-
-// Scalar part of the gate backward for one token (one lane per token).  In: sc[0] = dL/dalpha_t
-// so far, sc[1] = dL/deta_t, sc[2] = |k|^2, sc[3] = |k - v|^2; the token's record.  Out:
-// sc[4] = c_e, sc[5] = c_k with dk += c_e (k - v) + c_k k and dv -= c_e (k - v) (the gain and
-// spectral-clamp paths), sc[6] = dL/da, sc[7] = dL/dbeta.
-__device__ __forceinline__ void gate_backward_scalars(float* sc, const float* rc, const BwdArgs& A) {
-  float dal = sc[0];
-  const float deta = sc[1], kn2 = sc[2];
-  const float ne = sqrtf(sc[3]), kn = sqrtf(kn2), gain = ne * kn;
-  const float al = rc[kRal], a = rc[kRa], beta = rc[kRb];
-  const float sg = sigmoid_f(beta);
-  const float eta0 = softplus_f(a);
-  const float m = 1.f - al;
-  float eta1;
-  if (A.hard_cap) eta1 = (eta0 * gain > m) ? m / gain : eta0;
-  else eta1 = eta0 * phi_f(eta0 * gain / m);
-  const bool over = eta1 * kn2 > 2.f;                        // spectral clamp eta = 2 / |k|^2
-  const float deta1 = over ? 0.f : deta;
-  const float dkn2 = over ? -2.f * deta / (kn2 * kn2) : 0.f;
-  float deta0, dgain;
-  if (A.hard_cap) {                                          // eta1 = min(eta0, (1 - alpha_t) / g)
-    const bool binds = eta0 * gain > m;
-    deta0 = binds ? 0.f : deta1;
-    dgain = binds ? -deta1 * m / (gain * gain) : 0.f;
-    if (binds) dal -= deta1 / gain;
-  } else {                                                   // eta1 = eta0 phi(eta0 g / (1 - alpha_t))
-    const float z = eta0 * gain / m;
-    const float dz = deta1 * eta0 * dphi_f(z);
-    deta0 = deta1 * phi_f(z) + dz * gain / m;
-    dgain = dz * eta0 / m;
-    dal += dz * eta0 * gain / (m * m);
-  }
-  sc[4] = (ne > 0.f) ? dgain * kn / ne : 0.f;                // g = |k - v| |k|
-  sc[5] = 2.f * dkn2 + (kn > 0.f ? dgain * ne / kn : 0.f);
-  sc[6] = deta0 * sigmoid_f(a);                              // eta0 = softplus(a)
-  sc[7] = (sg > A.alpha) ? 0.f : dal * sg * (1.f - sg);      // alpha_t = min(sigmoid(beta), alpha)
 }
 
 __device__ __forceinline__ void load_row4(const float* m, int i, int j0, float (&v)[4]) {
@@ -513,7 +439,10 @@ __global__ void __launch_bounds__(kThreads, 2) srnl_scan_backward_kernel(const B
           A.dqr[((int64_t)r * A.B * N + tokbase_b + route_pos(r, t, A.H, A.W)) * C + ch0 + lane] = dq;
         }
         __syncthreads();
-        if (tid < nsb) gate_backward_scalars(sm.sc[tid], sm.rec[sb0 + tid], A);   // lane per token
+        if (tid < nsb) {   // lane per token
+          const float* rc = sm.rec[sb0 + tid];
+          bwd::gate_backward_scalars_f(sm.sc[tid], rc[kRal], rc[kRa], rc[kRb], A.alpha, A.hard_cap);
+        }
         __syncthreads();
         // per token, the rest (warp per token): dk~, then the generation and readout adjoints
         for (int tt = warp; tt < nsb; tt += kWarps) {
@@ -694,13 +623,13 @@ __global__ void __launch_bounds__(256) dwq_partial_kernel(const float* __restric
 }
 
 // Sum the split-K partials in split order and unpad to the caller's [C][C].
-__global__ void dwq_reduce_kernel(const float* __restrict__ part, int nsplit, int Cp, int heads, int ud,
+__global__ void dwq_reduce_kernel(const float* __restrict__ part, int nsplit, int Cp, int heads, int ud, int hd,
                                   float* __restrict__ out) {
   const int Cu = heads * ud;
   const int64_t n = (int64_t)Cu * Cu;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int o = (int)(i / Cu), c = (int)(i % Cu);
-    const int op = (o / ud) * kD + o % ud, cp = (c / ud) * kD + c % ud;
+    const int op = (o / ud) * hd + o % ud, cp = (c / ud) * hd + c % ud;
     float s = 0.f;
     for (int k = 0; k < nsplit; ++k) s += part[(size_t)k * Cp * Cp + (size_t)op * Cp + cp];
     out[i] = s;
@@ -708,31 +637,33 @@ __global__ void dwq_reduce_kernel(const float* __restrict__ part, int nsplit, in
 }
 
 // Sum the per-sequence partials over the batch (in batch order) and unpad: one thread per
-// output element of dM_mem0, dM_k0, dM_v0, dm_eta0, dm_alpha0 and dscales.
-__global__ void param_reduce_kernel(const float* __restrict__ parts, int routes, int B, int heads, int ud,
-                                    BwdGrads out) {
+// output element of dM_mem0, dM_k0, dM_v0, dm_eta0, dm_alpha0 and dscales.  A sequence's partials
+// (stride seq_part) are dM0 [hd][hd], dG [2 hd + 2][hd] (M_k, M_v, m_eta, m_alpha rows) and ds [hd].
+__global__ void param_reduce_kernel(const float* __restrict__ parts, int routes, int B, int heads, int ud, int hd,
+                                    size_t seq_part, BwdGrads out) {
   const int nm = ud * ud;
   const int per_rh = 3 * nm + 2 * ud + ud;      // M_mem, M_k, M_v, m_eta, m_alpha, scales
   const int64_t total = (int64_t)routes * heads * per_rh;
+  const int hh2 = hd * hd;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int rh = (int)(i / per_rh), e = (int)(i % per_rh);
     const int r = rh / heads, hh = rh % heads;
     int src;      // offset inside a sequence's partial block
     float* dst;
-    if (e < nm) { src = (e / ud) * kD + e % ud; dst = out.M_mem0 ? out.M_mem0 + (size_t)rh * nm + e : nullptr; }
-    else if (e < 2 * nm) { const int f = e - nm; src = kD * kD + (f / ud) * kD + f % ud;
+    if (e < nm) { src = (e / ud) * hd + e % ud; dst = out.M_mem0 ? out.M_mem0 + (size_t)rh * nm + e : nullptr; }
+    else if (e < 2 * nm) { const int f = e - nm; src = hh2 + (f / ud) * hd + f % ud;
       dst = out.M_k0 ? out.M_k0 + (size_t)rh * nm + f : nullptr; }
-    else if (e < 3 * nm) { const int f = e - 2 * nm; src = kD * kD + (kD + f / ud) * kD + f % ud;
+    else if (e < 3 * nm) { const int f = e - 2 * nm; src = hh2 + (hd + f / ud) * hd + f % ud;
       dst = out.M_v0 ? out.M_v0 + (size_t)rh * nm + f : nullptr; }
-    else if (e < 3 * nm + ud) { const int f = e - 3 * nm; src = kD * kD + 2 * kD * kD + f;
+    else if (e < 3 * nm + ud) { const int f = e - 3 * nm; src = hh2 + 2 * hh2 + f;
       dst = out.m_eta0 ? out.m_eta0 + (size_t)rh * ud + f : nullptr; }
-    else if (e < 3 * nm + 2 * ud) { const int f = e - 3 * nm - ud; src = kD * kD + 2 * kD * kD + kD + f;
+    else if (e < 3 * nm + 2 * ud) { const int f = e - 3 * nm - ud; src = hh2 + 2 * hh2 + hd + f;
       dst = out.m_alpha0 ? out.m_alpha0 + (size_t)rh * ud + f : nullptr; }
-    else { const int f = e - 3 * nm - 2 * ud; src = kD * kD + kGen * kD + f;
+    else { const int f = e - 3 * nm - 2 * ud; src = hh2 + (2 * hd + 2) * hd + f;
       dst = out.scales ? out.scales + (size_t)r * heads * ud + hh * ud + f : nullptr; }
     if (dst == nullptr) continue;
     float s = 0.f;
-    for (int b = 0; b < B; ++b) s += parts[((size_t)(r * B + b) * heads + hh) * kSeqPart + src];
+    for (int b = 0; b < B; ++b) s += parts[((size_t)(r * B + b) * heads + hh) * seq_part + src];
     *dst = s;
   }
 }
@@ -758,6 +689,8 @@ __global__ void seq_combine_kernel(const float* __restrict__ dxr, const float* _
 size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay) {
   const int N = g.H * g.W;
   const int nseq = g.routes * g.B * g.heads;
+  const int hd = g.hd;
+  const size_t hd2 = (size_t)hd * hd;
   int maxc = 0, Lmax = 0;
   for (int r = 0; r < g.routes; ++r) {
     const int L = r < 2 ? g.Lrow : g.Lcol;
@@ -768,7 +701,9 @@ size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay) {
   BwdLayout l;
   l.max_chunks = maxc;
   l.Lmax = Lmax;
-  l.nsplit = 0;
+  l.hd = hd;
+  l.rec = 2 * hd + 8;
+  l.seq_part = hd2 + (size_t)(2 * hd + 2) * hd + hd;
   const int tiles = ((g.C + kGT - 1) / kGT) * ((g.C + kGT - 1) / kGT);
   const int64_t M = (int64_t)g.B * N;
   l.nsplit = (int)std::min<int64_t>(std::max<int64_t>(1, 296 / tiles), (M + kGK - 1) / kGK);
@@ -776,10 +711,10 @@ size_t backward_workspace_floats(const ScanGeom& g, BwdLayout* lay) {
   l.dxr = off;  off += (size_t)g.routes * act;
   l.dqr = off;  off += (size_t)g.routes * act;
   l.dq = off;   off += act;
-  l.parts = off; off += (size_t)nseq * kSeqPart;
-  l.ckpt = off; off += (size_t)nseq * (maxc + 1) * kD * kD;
-  l.qs = off;   off += (size_t)nseq * Lmax * kD * kD;
-  l.grec = off; off += (size_t)nseq * N * kRec;
+  l.parts = off; off += (size_t)nseq * l.seq_part;
+  l.ckpt = off; off += (size_t)nseq * (maxc + 1) * hd2;
+  l.qs = off;   off += (size_t)nseq * Lmax * hd2;
+  l.grec = off; off += (size_t)nseq * N * l.rec;
   l.dwq = off;  off += (size_t)l.nsplit * g.C * g.C;
   l.total = off;
   if (lay) *lay = l;
@@ -808,6 +743,7 @@ cudaError_t launch_backward_scan(const ScanGeom& g, const ScanParamsDev& p, cons
                                  const void* dy, float* ws, cudaStream_t s) {
   BwdLayout l;
   backward_workspace_floats(g, &l);
+  if (g.hd == 64) return launch_backward_scan64(g, p, x, q, dy, ws, l, s);
   const BwdArgs A = backward_args(g, p, x, q, dy, ws, l);
   const int nseq = g.routes * g.B * g.heads;
   srnl_scan_backward_kernel<<<nseq, kThreads, sizeof(BwdSmem), s>>>(A);
@@ -836,12 +772,12 @@ cudaError_t launch_backward_combine(const ScanGeom& g, const ScanParamsDev& p, i
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t nout = (int64_t)g.heads * ud * g.heads * ud;
     dwq_reduce_kernel<<<(unsigned)std::min<int64_t>((nout + 255) / 256, 4096), 256, 0, s>>>(
-        ws + l.dwq, l.nsplit, g.C, g.heads, ud, dwq_out);
+        ws + l.dwq, l.nsplit, g.C, g.heads, ud, l.hd, dwq_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const int64_t nparam = (int64_t)g.routes * g.heads * (3 * ud * ud + 3 * ud);
   param_reduce_kernel<<<(unsigned)std::min<int64_t>((nparam + 255) / 256, 4096), 256, 0, s>>>(
-      ws + l.parts, g.routes, g.B, g.heads, ud, out);
+      ws + l.parts, g.routes, g.B, g.heads, ud, l.hd, l.seq_part, out);
   return cudaGetLastError();
 }
 
@@ -856,7 +792,7 @@ cudaError_t launch_backward_seq_combine(const ScanGeom& g, int ud, float* ws, vo
   if (e != cudaSuccess) return e;
   const int64_t nparam = (int64_t)g.routes * g.heads * (3 * ud * ud + 3 * ud);
   param_reduce_kernel<<<(unsigned)std::min<int64_t>((nparam + 255) / 256, 4096), 256, 0, s>>>(
-      ws + l.parts, g.routes, g.B, g.heads, ud, out);
+      ws + l.parts, g.routes, g.B, g.heads, ud, l.hd, l.seq_part, out);
   return cudaGetLastError();
 }
 

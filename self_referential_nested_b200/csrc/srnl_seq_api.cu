@@ -244,7 +244,6 @@ srnl_status srnl_seq_backward(srnl_seq* h, const void* x, const void* q, const v
       return seq_fail(h, SRNL_E_INVAL, "dx or dq overlaps an input");
   if (dq != nullptr && overlap(dx, dq, bytes)) return seq_fail(h, SRNL_E_INVAL, "dx and dq overlap");
   if (g.gen_bf16) return seq_fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for gen_dtype SRNL_F32 handles");
-  if (h->cfg.d == 64) return seq_fail(h, SRNL_E_UNSUPPORTED, "the backward pass is built for head dims up to 32");
   int cur = -1;
   cudaError_t e = cudaGetDevice(&cur);
   if (e != cudaSuccess) return seq_cuda_fail(h, e, "cudaGetDevice");

@@ -187,3 +187,24 @@ def test_backward_s1_full_size_bf16():
     got = gpu_backward(inp, dout, "bf16")
     ref = GR.backward_from_inputs(inp, dout)
     check(got, ref, "bf16", "hier_s1_56x56 B=32")
+
+
+# ---------------------------------------------------------------- head dim 64 (64-wide kernel)
+def _cfg64(name, **kw):
+    base = dict(name=name, B=2, H=5, W=9, C=128, heads=2, d=64, alpha=0.95, act_dtype="f32")
+    base.update(kw)
+    return ScanConfig(**base)
+
+
+@pytest.mark.parametrize("act", ["f32", "bf16"])
+def test_backward_d64_ragged_chunks(act):
+    run_case(_cfg64("b64", chunk_row=4, chunk_col=2), act, seed=11)
+
+
+def test_backward_d64_long_chunks_span_segments():
+    """Row chunks of 40 tokens: three gate segments and five sub-blocks per chunk."""
+    run_case(_cfg64("b64l", B=1, H=3, W=40), "f32", seed=12)
+
+
+def test_backward_d64_active_gates_hard_cap():
+    run_case(_cfg64("b64h", B=2, H=4, W=6, chunk_row=3), "f32", "hard", seed=13, mem_scale=0.2, vec_scale=0.6)

@@ -116,17 +116,3 @@ def test_d64_sequence_layer(queries, gen):
     err = O.rel_fro(y.float().cpu().numpy(), ref)
     tol = 1e-4 if gen == "f32" else 2e-2
     assert err <= tol, f"relative Frobenius error {err:.3e}"
-
-
-def test_d64_backward_is_unsupported():
-    cfg = _cfg("d64bwd")
-    inp = make_inputs(cfg, seed=0)
-    h = S.srnl_scan_create(dict(B=2, H=6, W=10, C=128, heads=2, d=64, alpha=0.95, act_dtype="f32",
-                                gen_dtype="f32"), inp.params())
-    try:
-        x = _dev(inp.x32, "f32")
-        with pytest.raises(S.SrnlError) as ei:
-            S.srnl_scan_backward(h, x, x.clone(), torch.empty_like(x))
-        assert ei.value.status == S.SRNL_E_UNSUPPORTED
-    finally:
-        h.close()

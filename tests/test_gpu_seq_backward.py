@@ -90,3 +90,8 @@ def test_seq_backward_rejects_dq_without_queries():
         assert ei.value.status == S.SRNL_E_INVAL
     finally:
         h.close()
+
+
+def test_seq_backward_head_dim_64():
+    run(2, 70, 128, 2, chunk=24, seed=14)
+    run(1, 33, 64, 1, chunk=0, queries=False, seed=15)
