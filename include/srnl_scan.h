@@ -100,9 +100,9 @@ typedef enum { SRNL_CAP_SOFT = 0, SRNL_CAP_HARD = 1 } srnl_cap;
 typedef struct {
   int B, H, W, C; /* batch, height, width, channels (C = heads * d) */
   int heads, d;   /* heads and head dim: 4, 8, 16, 32 or 64 (below 32 the heads run zero-padded
-                     to 32 lanes, which is exact; 64 runs a 64-wide SIMT kernel, fp32 products
-                     with the bf16 path's roundings when gen_dtype is SRNL_BF16, and has no
-                     backward; the no-allocation forward takes 32 only) */
+                     to 32 lanes, which is exact; 64 runs 64-wide SIMT kernels, fp32 products
+                     with the bf16 path's roundings when gen_dtype is SRNL_BF16; the
+                     no-allocation forward takes 32 only) */
   float alpha;    /* retention cap, 0 < alpha < 1 (0.95 hierarchical, 0.9 plain) */
   float eps;      /* key normalisation epsilon, > 0 (1e-6) */
   int chunk_row;  /* chunk length on routes 0/1; 0 means W (full rows) */
@@ -249,8 +249,9 @@ typedef struct {
  * The forward is recomputed from x (boundary products are kept per chunk and the states
  * inside a chunk recomputed), so no forward state is needed.  The first call allocates the
  * backward workspace (cudaMalloc, synchronous; about 9 fp32 values per activation element,
- * plus per (route, batch, head) sequence 288 bytes per token and 4 KB per chunk and per token
- * of its longest chunk); later calls reuse it.  Asynchronous on `stream`; shares the handle's workspace with the forward. */
+ * plus per (route, batch, head) sequence (2 w + 8) floats per token and w^2 floats per chunk
+ * and per token of its longest chunk, w = 32 or 64 the kernels' head width); later calls
+ * reuse it.  Asynchronous on `stream`; shares the handle's workspace with the forward. */
 SRNL_API srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void* dx,
                                        const srnl_scan_grads* grads, void* stream);
 
