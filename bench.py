@@ -380,7 +380,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                   "note": "scan of one image (each sequence alone on an SM) over the full scan"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * elt),
                 "d2h_bytes_per_step": int(y.numel() * elt), "ms_per_step": e2e_ms / args.steps},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (3 if cfg.d >= 32 else 5) * args.steps,   # + pad x, unpad y below 32
         "clocks": clocks.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -524,7 +524,7 @@ def run_backward(args, cfg):
         "e2e": {"value": route_tokens * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": int(2 * x.numel() * elt), "d2h_bytes_per_step": int(dx.numel() * elt) + grad_bytes,
                 "ms_per_step": e2e_ms / args.steps},
-        "gpu_launches": (7 if cfg.d == 32 else 10) * args.steps,
+        "gpu_launches": (7 if cfg.d >= 32 else 10) * args.steps,   # + pad x, pad dy, unpad dx below 32
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline:
