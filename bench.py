@@ -517,7 +517,8 @@ def run_backward(args, cfg):
                    "heads": cfg.heads, "d": cfg.d, "alpha": cfg.alpha, "act_dtype": act, "gen_dtype": "f32",
                    "injection_cap": args.cap, "l2": "flushed (256 MiB write before each timed step)"},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": fp32_peak_tflops, "unit": "TFLOP/s",
-                     "frac": achieved / fp32_peak_tflops, "traffic": None, "kernel": "srnl_scan_backward_kernel",
+                     "frac": achieved / fp32_peak_tflops, "traffic": None,
+                     "kernel": "srnl_scan_backward64_kernel" if cfg.d == 64 else "srnl_scan_backward_kernel",
                      "kernel_ms": scan_ms, "flops_per_route_head_token": backward_flops_per_token(cfg.d),
                      "peak_note": "fp32 FMA peak 148 SM x 128 lanes x 2 x sm_max_mhz (derived)"},
         "stage_ms": {"query_projection": float(stage[0]), "scan_backward": scan_ms, "combine": float(stage[2])},
