@@ -354,16 +354,25 @@ srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void
   const int elt = h->geom.act_bf16 ? 2 : 4;
   const int64_t tokens = (int64_t)h->geom.B * h->geom.H * h->geom.W;
   cudaError_t e;
-  if (h->bws == nullptr) {
+  if (h->bws == nullptr) {  // all or nothing: a failed allocation leaves none of the three
     const size_t nb = srnl::backward_workspace_floats(h->geom, nullptr) * sizeof(float);
-    if ((e = cudaMalloc(&h->bws, nb)) != cudaSuccess) { h->bws = nullptr; return cuda_fail(h, e, "cudaMalloc (backward workspace)"); }
-    h->ws_bytes += nb;
-    if (padded) {
-      const size_t pb = (size_t)tokens * h->geom.C * elt;
-      if ((e = cudaMalloc(&h->dy_pad, pb)) != cudaSuccess) { h->dy_pad = nullptr; return cuda_fail(h, e, "cudaMalloc (dy padding)"); }
-      if ((e = cudaMalloc(&h->dx_pad, pb)) != cudaSuccess) { h->dx_pad = nullptr; return cuda_fail(h, e, "cudaMalloc (dx padding)"); }
-      h->ws_bytes += 2 * pb;
+    const size_t pb = padded ? (size_t)tokens * h->geom.C * elt : 0;
+    void* ws = nullptr;
+    void* dyp = nullptr;
+    void* dxp = nullptr;
+    e = cudaMalloc(&ws, nb);
+    if (e == cudaSuccess && padded) e = cudaMalloc(&dyp, pb);
+    if (e == cudaSuccess && padded) e = cudaMalloc(&dxp, pb);
+    if (e != cudaSuccess) {
+      void* got[] = {ws, dyp, dxp};
+      for (void* q : got)
+        if (q != nullptr) cudaFree(q);
+      return cuda_fail(h, e, "cudaMalloc (backward workspace)");
     }
+    h->bws = static_cast<float*>(ws);
+    h->dy_pad = dyp;
+    h->dx_pad = dxp;
+    h->ws_bytes += nb + 2 * pb;
   }
   if (padded) {
     e = srnl::launch_pad_heads(x, h->x_pad, tokens, h->geom.heads, h->cfg.d, elt, s);
@@ -430,7 +439,19 @@ static srnl_status pipeline_setup(srnl_scan* h) {
     for (cudaEvent_t* ev : evs)
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
   }
-  if (e != cudaSuccess) return cuda_fail(h, e, "pipeline set-up");
+  if (e != cudaSuccess) {  // all or nothing: release what was created, so a later call starts over
+    if (h->x_stage1 != nullptr) cudaFree(h->x_stage1);
+    if (h->y_stage1 != nullptr) cudaFree(h->y_stage1);
+    h->x_stage1 = h->y_stage1 = nullptr;
+    for (int k = 0; k < 2; ++k) {
+      cudaEvent_t* evs[] = {&h->h2d_done[k], &h->fwd_done[k], &h->d2h_done[k]};
+      for (cudaEvent_t* ev : evs)
+        if (*ev != nullptr) { cudaEventDestroy(*ev); *ev = nullptr; }
+    }
+    if (h->d2h != nullptr) { cudaStreamDestroy(h->d2h); h->d2h = nullptr; }
+    if (h->h2d != nullptr) { cudaStreamDestroy(h->h2d); h->h2d = nullptr; }
+    return cuda_fail(h, e, "pipeline set-up");
+  }
   h->ws_bytes += 2 * n;
   return SRNL_OK;
 }

@@ -253,16 +253,19 @@ srnl_status srnl_seq_backward(srnl_seq* h, const void* x, const void* q, const v
   const int elt = g.act_bf16 ? 2 : 4;
   const int64_t tokens = (int64_t)g.B * g.W;
   const size_t pbytes = (size_t)tokens * g.C * elt;
-  if (h->bws == nullptr) {
-    if ((e = cudaMalloc(&h->bws, srnl::backward_workspace_floats(g, nullptr) * sizeof(float))) != cudaSuccess) {
-      h->bws = nullptr;
+  if (h->bws == nullptr) {  // all or nothing: a failed allocation leaves none of the four
+    void* got[4] = {nullptr, nullptr, nullptr, nullptr};
+    e = cudaMalloc(&got[0], srnl::backward_workspace_floats(g, nullptr) * sizeof(float));
+    for (int i = 1; i < 4 && padded && e == cudaSuccess; ++i) e = cudaMalloc(&got[i], pbytes);
+    if (e != cudaSuccess) {
+      for (void* q : got)
+        if (q != nullptr) cudaFree(q);
       return seq_cuda_fail(h, e, "cudaMalloc (backward workspace)");
     }
-    if (padded) {
-      void** bufs[] = {&h->dy_pad, &h->dx_pad, &h->dq_pad};
-      for (void** b : bufs)
-        if ((e = cudaMalloc(b, pbytes)) != cudaSuccess) { *b = nullptr; return seq_cuda_fail(h, e, "cudaMalloc (padding)"); }
-    }
+    h->bws = static_cast<float*>(got[0]);
+    h->dy_pad = got[1];
+    h->dx_pad = got[2];
+    h->dq_pad = got[3];
   }
   const void* qk = q != nullptr ? q : x;
   if (padded) {
