@@ -1,12 +1,13 @@
 """Python binding of the SRNL four-direction scan C ABI (``include/srnl_scan.h``).
 
-Argument marshalling only: every step of the forward runs in the CUDA kernels of
-``libsrnl_scan.so``.  There is no CPU fallback; importing works without a GPU,
+Argument marshalling only: every step of the forward and the backward runs in the CUDA
+kernels of ``libsrnl_scan.so``.  There is no CPU fallback; importing works without a GPU,
 but creating a handle needs the built library and a CUDA device.
 
     from self_referential_nested_b200 import srnl_scan_create, srnl_scan_forward
     h = srnl_scan_create(cfg_dict, params_dict)      # params: float32 numpy arrays
     srnl_scan_forward(h, x, y)                      # x, y: CUDA tensors [B,H,W,C]
+    srnl_scan_backward(h, x, dy, dx, grads)         # fp32-generation handles; grads: GRAD_KEYS
 """
 from __future__ import annotations
 
