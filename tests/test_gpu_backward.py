@@ -95,6 +95,10 @@ def test_backward_ragged_chunks(act):
     run_case(_cfg("ragged", B=2, H=7, W=13, chunk_row=5, chunk_col=3), act, seed=1)
 
 
+def test_backward_single_token_map():
+    run_case(_cfg("one", B=2, H=1, W=1), "f32", seed=9)
+
+
 def test_backward_long_chunks_span_segments():
     """Row chunks of 150 tokens: several gate segments and sub-blocks per chunk."""
     run_case(_cfg("long", B=1, H=3, W=150), "f32", seed=2)

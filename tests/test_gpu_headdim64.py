@@ -81,6 +81,10 @@ def test_d64_operator_long_chunks_span_segments():
     run_operator(_cfg("d64l", B=1, H=2, W=100), seed=3, finals=False)
 
 
+def test_d64_operator_single_token_map():
+    run_operator(_cfg("d64one", B=2, H=1, W=1), seed=9)
+
+
 def test_d64_operator_one_head():
     run_operator(_cfg("d64h1", C=64, heads=1, H=5, W=8), seed=4)
 

@@ -159,6 +159,7 @@ ACTIVE = dict(mem_scale=0.3, vec_scale=1.0)
 
 RAGGED = [
     # (H, W, B, heads, chunk_row, chunk_col, alpha)
+    (1, 1, 2, 2, 0, 0, 0.95),       # a single token on every route
     (3, 5, 2, 1, 0, 0, 0.95),
     (5, 3, 1, 3, 0, 0, 0.9),
     (1, 9, 2, 2, 0, 0, 0.95),

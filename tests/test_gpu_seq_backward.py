@@ -95,3 +95,7 @@ def test_seq_backward_rejects_dq_without_queries():
 def test_seq_backward_head_dim_64():
     run(2, 70, 128, 2, chunk=24, seed=14)
     run(1, 33, 64, 1, chunk=0, queries=False, seed=15)
+
+
+def test_seq_backward_single_token():
+    run(3, 1, 64, 2, seed=16)
