@@ -82,7 +82,7 @@ typedef struct srnl_scan srnl_scan; /* opaque; owned by the library */
 typedef enum {
   SRNL_OK = 0,
   SRNL_E_INVAL = -1,       /* bad argument: NULL, shape, alignment, range */
-  SRNL_E_UNSUPPORTED = -2, /* valid but not built (e.g. head dim other than 32) */
+  SRNL_E_UNSUPPORTED = -2, /* valid but not built (e.g. a head dim other than 4, 8, 16, 32, 64) */
   SRNL_E_CUDA = -3,        /* a CUDA runtime call failed */
   SRNL_E_NOMEM = -4,       /* device or pinned allocation failed */
   SRNL_E_TIMEOUT = -5      /* a bounded in-kernel wait gave up (see srnl_scan_device_status) */
