@@ -215,3 +215,27 @@ def test_sequence_backward_matches_finite_differences(with_queries, cap):
     for key in keys:
         fd, an = _directional_check(loss, base, grads[key], rng, key)
         assert abs(fd - an) <= FD_TOL * max(abs(an), 1e-3), (key, fd, an)
+
+
+def test_sequence_backward_is_route_zero_of_the_operator():
+    """The sequence layer is route 0 of the operator on a 1 x T map with W_q = I and scales one on
+    route 0, zero elsewhere (the forward pin); so are its gradients: dx (including the query
+    path) and the initial-state gradients equal the operator's route-0 gradients, and the other
+    routes' initial states get none."""
+    B, T, D, heads = 2, 11, 8, 2
+    d = D // heads
+    rng = np.random.default_rng(31)
+    x = rng.normal(0, 1, (B, T, D))
+    dy = rng.normal(0, 1, (B, T, D))
+    seq_p = {"M_mem0": rng.normal(0, .3, (heads, d, d)), "M_k0": rng.normal(0, .3, (heads, d, d)),
+             "M_v0": rng.normal(0, .4, (heads, d, d)), "m_eta0": rng.normal(0, .8, (heads, d)),
+             "m_alpha0": rng.normal(0, 1.5, (heads, d))}
+    op_p = {k: np.concatenate([v[None], 0.5 * np.ones((3,) + v.shape)], axis=0) for k, v in seq_p.items()}
+    op_p["W_q"] = np.eye(D)
+    op_p["scales"] = np.concatenate([np.ones((1, D)), np.zeros((3, D))], axis=0)
+    gs = GR.sequence_backward(x, seq_p, dy, alpha_max=0.95, chunk=4, heads=heads)
+    go = GR.operator_backward(x[:, None], op_p, dy[:, None], alpha_max=0.95, chunk_row=4, heads=heads)
+    np.testing.assert_allclose(go["x"][:, 0], gs["x"], rtol=1e-12, atol=1e-14)
+    for key in ("M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0"):
+        np.testing.assert_allclose(go[key][0], gs[key], rtol=1e-12, atol=1e-14)
+        assert np.all(go[key][1:] == 0.0), key
