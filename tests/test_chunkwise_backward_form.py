@@ -120,3 +120,65 @@ def test_chunkwise_stage_reverse_equals_token_recurrence(T, retention):
     for key in ("Qe", "z", "w", "deta", "du", "dk", "dq", "dal", "dQs"):
         scale = max(np.max(np.abs(ref[key])), 1e-300)
         np.testing.assert_allclose(got[key], ref[key], rtol=1e-9, atol=1e-10 * scale, err_msg=key)
+
+
+def test_chunkwise_scan_backward_equals_oracle():
+    """The whole scan's backward assembled from the chunkwise stage reverse: per chunk in
+    reverse, the stage reverse above, then the gate backward, the generation adjoint and the
+    boundary gradient joining the carried dQ; against the gradient oracle."""
+    from oracle import srnl_grad as GR
+    from oracle import srnl_oracle as O
+
+    rng = np.random.default_rng(52)
+    S_, N, d, chunk = 2, 19, 4, 6
+    xs, qs, dy = rng.normal(0, 1, (S_, N, d)), rng.normal(0, 1, (S_, N, d)), rng.normal(0, 1, (S_, N, d))
+    inits = dict(M_mem=rng.normal(0, .3, (S_, d, d)), M_k=rng.normal(0, .3, (S_, d, d)),
+                 M_v=rng.normal(0, .4, (S_, d, d)), m_eta=rng.normal(0, .8, (S_, d)),
+                 m_alpha=rng.normal(0, 1.5, (S_, d)))
+    ref_x, ref_q, ref_init, _ = GR.scan_five_memory_backward(xs, qs, inits, chunk, 0.95, 1e-6, dy)
+    for s in range(S_):
+        M0 = inits["M_mem"][s]
+        G = np.concatenate([inits["M_k"][s], inits["M_v"][s], inits["m_eta"][s][None], inits["m_alpha"][s][None]])
+        bounds = list(range(0, N, chunk))
+        Q, ckpt = np.eye(d), []
+        for c0 in bounds:                                   # checkpoint pass (token loop is fine here)
+            c1 = min(c0 + chunk, N)
+            ckpt.append(Q.copy())
+            gen = (G @ (Q @ xs[s, c0:c1].T)).T
+            gt = O.gates(gen[:, :d], gen[:, d:2 * d], gen[:, 2 * d], gen[:, 2 * d + 1], 0.95, 1e-6)
+            for j in range(c1 - c0):
+                u = (1 + gt["alpha_t"][j]) * gt["k"][j] - gen[j, d:2 * d]
+                Q = gt["alpha_t"][j] * Q - gt["eta"][j] * np.outer(Q @ u, gt["k"][j])
+        dQ = np.zeros((d, d))
+        dx, dq = np.zeros((N, d)), np.zeros((N, d))
+        dM0, dG = np.zeros((d, d)), np.zeros_like(G)
+        for c0, Qb in reversed(list(zip(bounds, ckpt))):
+            c1 = min(c0 + chunk, N)
+            X = xs[s, c0:c1]
+            h = (Qb @ X.T).T
+            gen = h @ G.T
+            kt, vv, av, bv = gen[:, :d], gen[:, d:2 * d], gen[:, 2 * d], gen[:, 2 * d + 1]
+            gt = O.gates(kt, vv, av, bv, 0.95, 1e-6)
+            k, al, et = gt["k"], gt["alpha_t"], gt["eta"]
+            u = (1 + al)[:, None] * k - vv
+            a = dy[s, c0:c1] @ M0                            # a_t = M0^T dy_t
+            st = chunkwise_reverse(Qb, k, u, qs[s, c0:c1], al, et, a, dQ)
+            dq[c0:c1] = st["dq"]
+            dM0 += dy[s, c0:c1].T @ st["z"]
+            # through u = (1 + alpha) k - v
+            dk_w = st["dk"] + (1 + al)[:, None] * st["du"]
+            dal_w = st["dal"] + np.sum(k * st["du"], axis=1)
+            dkt, dvv, da, db = GR.gates_backward(kt, vv, av, bv, 0.95, 1e-6, "soft", dk_w, -st["du"], dal_w,
+                                                 st["deta"])
+            dgen = np.concatenate([dkt, dvv, da[:, None], db[:, None]], axis=1)
+            dG += dgen.T @ h
+            dh = dgen @ G
+            dx[c0:c1] = dh @ Qb
+            dQ = st["dQs"] + dh.T @ X                        # the boundary joins the carried gradient
+        np.testing.assert_allclose(dx, ref_x[s], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(dq, ref_q[s], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(dM0, ref_init["M_mem"][s], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(dG[:d], ref_init["M_k"][s], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(dG[d:2 * d], ref_init["M_v"][s], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(dG[2 * d], ref_init["m_eta"][s], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(dG[2 * d + 1], ref_init["m_alpha"][s], rtol=1e-9, atol=1e-12)
