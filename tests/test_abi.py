@@ -156,3 +156,16 @@ def test_selftest_rejects_out_of_range_limits_before_cuda(lib):
 def test_backward_null_arguments_fail_cleanly(lib):
     assert lib.srnl_scan_backward(None, None, None, None, None, None) == S.SRNL_E_INVAL
     assert lib.srnl_seq_backward(None, None, None, None, None, None, None, None) == S.SRNL_E_INVAL
+
+
+def test_committed_code_never_uses_the_scratch_directory():
+    """Nothing in the product, the tests or the bench may read or run files from _work/."""
+    pat = re.compile(r"\b_work/")
+    for dirpath, dirnames, files in os.walk(ROOT):
+        dirnames[:] = [d for d in dirnames if d not in ("_work", ".git", "gpurun_out", "__pycache__", ".pytest_cache")]
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".sh")):
+                path = os.path.join(dirpath, f)
+                if os.path.samefile(path, __file__):
+                    continue
+                assert not pat.search(open(path, errors="ignore").read()), path
