@@ -113,6 +113,65 @@ def test_soft_cap_limits():
     np.testing.assert_allclose(big * 1.0, 0.1, rtol=1e-12)
 
 
+def test_sigmoid_closed_forms():
+    """The logistic function: sigma(0) = 1/2, sigma(ln 3) = 3/4, sigma(-z) = 1 - sigma(z), and its
+    asymptotes (1 - e^-z above, e^z below), without overflow at |z| = 800."""
+    z = np.array([0.0, np.log(3.0), -np.log(3.0), np.log(99.0)])
+    np.testing.assert_allclose(O.sigmoid(z), [0.5, 0.75, 0.25, 0.99], rtol=1e-15)
+    rng = np.random.default_rng(31)
+    w = rng.normal(0, 6, 1000)
+    np.testing.assert_allclose(O.sigmoid(-w), 1.0 - O.sigmoid(w), atol=1e-15)
+    np.testing.assert_allclose(O.sigmoid(np.array([40.0, -40.0])), [1.0 - np.exp(-40.0), np.exp(-40.0)],
+                               rtol=1e-14)
+    with np.errstate(over="raise"):
+        big = O.sigmoid(np.array([800.0, -800.0]))
+    assert big[0] == 1.0 and 0.0 <= big[1] < 1e-300
+
+
+def test_softplus_closed_forms():
+    """softplus(z) = log(1 + e^z): softplus(0) = ln 2, softplus(ln(e - 1)) = 1,
+    softplus(z) - softplus(-z) = z, and softplus(z) -> z above, e^z below."""
+    np.testing.assert_allclose(O.softplus(np.array([0.0, np.log(np.e - 1.0)])), [np.log(2.0), 1.0], rtol=1e-15)
+    rng = np.random.default_rng(32)
+    w = rng.normal(0, 8, 1000)
+    np.testing.assert_allclose(O.softplus(w) - O.softplus(-w), w, atol=1e-13)
+    np.testing.assert_allclose(O.softplus(np.array([50.0, -50.0])), [50.0, np.exp(-50.0)], rtol=1e-15)
+
+
+def test_retention_clamp_values():
+    """alpha_t = min(sigmoid(beta), alpha): below the cap it is the logistic of beta, above it the cap."""
+    beta = np.array([np.log(3.0), -np.log(3.0), np.log(99.0), 0.0])
+    np.testing.assert_allclose(O.retention(beta, 0.95), [0.75, 0.25, 0.95, 0.5], rtol=1e-15)
+
+
+def test_gates_hand_computed_token():
+    """One token worked by hand (d = 2, eps = 0): k~ = (3, 4), v = 0, a = 0, beta = ln 3.
+    k = (3, 4) / 5; alpha_t = sigmoid(ln 3) = 3/4; eta0 = softplus(0) = ln 2; gain
+    g = ||k - v|| ||k|| = 1; the soft cap's z = eta0 g / (1 - alpha_t) = 4 ln 2, and
+    tanh(4 ln 2) = (16 - 1/16) / (16 + 1/16) = 255/257, so eta1 = eta0 tanh(z) / z = 255/1028;
+    the spectral clamp (eta ||k||^2 <= 2) leaves it."""
+    gt = O.gates(np.array([[3.0, 4.0]]), np.zeros((1, 2)), np.array([0.0]), np.array([np.log(3.0)]),
+                 0.95, 0.0)
+    np.testing.assert_allclose(gt["k"], [[0.6, 0.8]], rtol=1e-15)
+    np.testing.assert_allclose(gt["alpha_t"], [0.75], rtol=1e-15)
+    np.testing.assert_allclose(gt["eta0"], [np.log(2.0)], rtol=1e-15)
+    np.testing.assert_allclose(gt["gain"], [1.0], rtol=1e-15)
+    np.testing.assert_allclose(gt["eta"], [255.0 / 1028.0], rtol=1e-14)
+    # a value that is not a rescaled key: v = (0, 1) gives ||k - v|| = sqrt(0.36 + 0.04)
+    gt = O.gates(np.array([[3.0, 4.0]]), np.array([[0.0, 1.0]]), np.array([0.0]), np.array([np.log(3.0)]),
+                 0.95, 0.0)
+    np.testing.assert_allclose(gt["gain"], [np.sqrt(0.4)], rtol=1e-15)
+
+
+def test_query_projection_orientation_hand_computed():
+    """q = x W_q^T with W_q[o][c] (output channel o, input channel c): x = (1, 10) and
+    W_q = [[1, 2], [3, 4]] give q = (1 + 20, 3 + 40) = (21, 43)."""
+    x = np.array([1.0, 10.0]).reshape(1, 1, 1, 2)
+    q = O.query_projection(x, np.array([[1.0, 2.0], [3.0, 4.0]]))
+    assert q.shape == (1, 1, 1, 2)
+    np.testing.assert_array_equal(q.reshape(2), [21.0, 43.0])
+
+
 def test_spectral_clamp_bound():
     e1 = np.array([0.5, 3.0, 10.0, 0.0])
     kn2 = np.array([1.0, 1.0, 0.5, 0.0])
