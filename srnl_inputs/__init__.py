@@ -19,6 +19,14 @@ Draw order for one config with seed s (numpy ``default_rng(s)``):
   5. W_q ~ N(0, 1 / C), shape [C, C]
 Channel scales are the constant 0.25 ([4, C]).  For bf16 configs x is rounded
 to bfloat16 (round to nearest even) and both sides receive those same values.
+
+Long-sequence parity cases add a ``Sustain`` knob after the draws (it draws nothing and
+changes the draw order of nothing): channel 0 of every head of x becomes the constant
+``feature`` and ``retention_bias`` / ``step_bias`` are added to channel 0 of m_alpha0 /
+m_eta0.  A retention logit that stays far above the clamp keeps alpha_t = alpha on every
+token, so a retention cap close to 1 holds the memories inside fp32 range over thousands of
+tokens; with the workload's own initials the memories halve every token and every chunk
+after the first few is zero in fp32.
 """
 from __future__ import annotations
 
@@ -105,9 +113,25 @@ class ScanInputs:
                     m_alpha0=self.m_alpha0)
 
 
+@dataclasses.dataclass(frozen=True)
+class Sustain:
+    """A constant feature on channel 0 of every head of x, and biases on channel 0 of the
+    retention and step initials (parity cases on long sequences only)."""
+    feature: float = 1.0
+    retention_bias: float = 300.0
+    step_bias: float = -7.0
+
+
+def _apply_sustain(x: np.ndarray, m_eta0: np.ndarray, m_alpha0: np.ndarray, d: int, sus: Sustain) -> None:
+    x.reshape(x.shape[:-1] + (x.shape[-1] // d, d))[..., 0] = np.float32(sus.feature)
+    m_alpha0[..., 0] += np.float32(sus.retention_bias)
+    m_eta0[..., 0] += np.float32(sus.step_bias)
+
+
 def make_inputs(cfg: ScanConfig, seed: int = 0, *, x_scale: float = 1.0,
-                mem_scale: float = 0.02, vec_scale: float = 0.1) -> ScanInputs:
-    """Draw one workload.  ``*_scale`` knobs exist for extra parity cases only."""
+                mem_scale: float = 0.02, vec_scale: float = 0.1,
+                sustain: Optional[Sustain] = None) -> ScanInputs:
+    """Draw one workload.  ``*_scale`` and ``sustain`` knobs exist for extra parity cases only."""
     rng = np.random.default_rng(seed)
     B, H, W, C, nh, d = cfg.B, cfg.H, cfg.W, cfg.C, cfg.heads, cfg.d
     x = rng.standard_normal((B, H, W, C), dtype=np.float32) * np.float32(x_scale)
@@ -126,6 +150,8 @@ def make_inputs(cfg: ScanConfig, seed: int = 0, *, x_scale: float = 1.0,
     m_alpha0 = (rng.standard_normal((4, nh, d)) * vec_scale).astype(np.float32)
     W_q = (rng.standard_normal((C, C)) / np.sqrt(C)).astype(np.float32)
     scales = np.full((4, C), 0.25, dtype=np.float32)
+    if sustain is not None:
+        _apply_sustain(x, m_eta0, m_alpha0, d, sustain)
     x_bits = None
     if cfg.act_dtype == BF16:
         x_bits = bf16_round_bits(x)
@@ -163,9 +189,11 @@ class SeqInputs:
 
 
 def make_seq_inputs(B: int, T: int, D: int, heads: int, act_dtype: str = F32, seed: int = 0, *,
-                    mem_scale: float = 0.02, vec_scale: float = 0.1) -> SeqInputs:
+                    mem_scale: float = 0.02, vec_scale: float = 0.1,
+                    sustain: Optional[Sustain] = None) -> SeqInputs:
     """Draw x, queries ~ N(0, 1) [B, T, D], then M_mem0, M_k0, M_v0 ~ N(0, mem_scale^2)
-    [heads, d, d] and m_eta0, m_alpha0 ~ N(0, vec_scale^2) [heads, d], in that order."""
+    [heads, d, d] and m_eta0, m_alpha0 ~ N(0, vec_scale^2) [heads, d], in that order; then
+    apply ``sustain`` (to x only, not to the queries)."""
     rng = np.random.default_rng(seed)
     d = D // heads
     x = rng.standard_normal((B, T, D), dtype=np.float32)
@@ -175,6 +203,8 @@ def make_seq_inputs(B: int, T: int, D: int, heads: int, act_dtype: str = F32, se
     M_v0 = (rng.standard_normal((heads, d, d)) * mem_scale).astype(np.float32)
     m_eta0 = (rng.standard_normal((heads, d)) * vec_scale).astype(np.float32)
     m_alpha0 = (rng.standard_normal((heads, d)) * vec_scale).astype(np.float32)
+    if sustain is not None:
+        _apply_sustain(x, m_eta0, m_alpha0, d, sustain)
     x_bits = q_bits = None
     if act_dtype == BF16:
         x_bits, q_bits = bf16_round_bits(x), bf16_round_bits(q)

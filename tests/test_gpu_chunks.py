@@ -1,0 +1,209 @@
+"""GPU parity chunk by chunk, at the workloads' full sizes, on inputs that keep every chunk alive.
+
+With the workloads' own initials the memories halve every token (the retention gate sits near
+sigmoid(0) = 1/2), so after the first chunk of a route the outputs fall below fp32 range and a
+whole-tensor error only checks the first chunk.  These cases use the ``Sustain`` knob of the
+input generator (a constant feature channel and a retention bias that keeps alpha_t = alpha on
+every token) with a retention cap close to 1, so that the last chunk of every route still
+carries a few percent of the first chunk's norm.  The test asserts that before it compares.
+
+Each route is isolated with one-hot fusion scales ("VisionHOPE" README, "Overview" item 3: the
+four scans are fused with learned channel-wise scales), gathered back to route order and split
+into its chunks ("VisionHOPE Model Overview", "Four-Directional Scanning and Spatial Chunking":
+full rows on the row routes, full columns on the column routes, the boundary states of each
+chunk generating the next).  Every chunk must match the float64 oracle on its own: 1e-4 on the
+fp32 path, 2e-2 on the bf16 path (relative Frobenius error of the chunk).  The worst chunk of
+each case is printed (run pytest with -s to see it).
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import self_referential_nested_b200 as S
+from oracle import srnl_grad as GR
+from oracle import srnl_oracle as O
+from srnl_inputs import CONFIGS, Sustain, bf16_round_bits, make_cotangent, make_inputs, make_seq_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {("f32", "f32"): 1e-4, ("bf16", "bf16"): 2e-2, ("bf16", "f32"): 2e-2}
+ALIVE_FLOOR = 1e-3     # every reference chunk keeps at least this share of the first chunk's norm
+
+# (config, retention cap, retention bias, images compared)
+S1 = (CONFIGS["hier_s1_56x56"].replace(alpha=0.999), Sustain(), (0, 31))
+HIRES = (CONFIGS["hires_200x304"].replace(alpha=0.99995), Sustain(retention_bias=1000.0), (1,))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from self_referential_nested_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+
+
+def _dev(a32, act):
+    if act == "bf16":
+        return torch.from_numpy(bf16_round_bits(a32).view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a32, dtype=np.float32)).cuda()
+
+
+def _cfg_dict(cfg, act, gen):
+    return dict(B=cfg.B, H=cfg.H, W=cfg.W, C=cfg.C, heads=cfg.heads, d=cfg.d, alpha=cfg.alpha, eps=cfg.eps,
+                chunk_row=cfg.chunk_row, chunk_col=cfg.chunk_col, act_dtype=act, gen_dtype=gen)
+
+
+def one_hot(params, route):
+    p = dict(params)
+    p["scales"] = np.zeros_like(params["scales"])
+    p["scales"][route] = 1.0
+    return p
+
+
+@functools.lru_cache(maxsize=None)
+def _inputs(case, act):
+    cfg, sus, _ = case
+    return make_inputs(cfg.replace(act_dtype=act), seed=0, mem_scale=0.3, vec_scale=0.05, sustain=sus)
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_routes(case, act):
+    """Route-order outputs [4][n, N, C] and final states [4, n, heads, 3 d^2 + 2 d] of the
+    sampled images, one route at a time through the oracle's scan."""
+    cfg, _, images = case
+    inp = _inputs(case, act)
+    x = inp.x32[list(images)].astype(np.float64)
+    n, N, d, nh = x.shape[0], cfg.H * cfg.W, cfg.d, cfg.heads
+    q = O.query_projection(x, inp.W_q.astype(np.float64))
+
+    def per_head(a, r):
+        return O.gather(a, r).reshape(n, N, nh, d).transpose(0, 2, 1, 3).reshape(n * nh, N, d)
+
+    outs, fins = [], []
+    for r in range(4):
+        inits = {}
+        for key, name in (("M_mem0", "M_mem"), ("M_k0", "M_k"), ("M_v0", "M_v"), ("m_eta0", "m_eta"),
+                          ("m_alpha0", "m_alpha")):
+            arr = np.asarray(getattr(inp, key), np.float64)[r]
+            inits[name] = np.broadcast_to(arr[None], (n,) + arr.shape).reshape((-1,) + arr.shape[1:]).copy()
+        L = O.default_chunk(cfg.H, cfg.W, r, cfg.chunk_row, cfg.chunk_col)
+        y, fin, _ = O.scan_five_memory(per_head(x, r), per_head(q, r), inits, L, cfg.alpha, cfg.eps)
+        outs.append(y.reshape(n, nh, N, d).transpose(0, 2, 1, 3).reshape(n, N, cfg.C))
+        fins.append(np.concatenate([fin[k].reshape(n * nh, -1) for k in ("M_mem", "M_k", "M_v", "m_eta", "m_alpha")],
+                                   axis=1).reshape(n, nh, -1))
+    return outs, np.stack(fins)
+
+
+def chunk_errors(got, ref, L):
+    """Relative Frobenius error of every chunk of a route ([n, N, C], route order); asserts that
+    every reference chunk is alive first."""
+    N = ref.shape[1]
+    norms = [np.linalg.norm(ref[:, c0:c0 + L]) for c0 in range(0, N, L)]
+    assert min(norms) >= ALIVE_FLOOR * norms[0], f"reference chunk norms fall to {min(norms) / norms[0]:.2e}"
+    return np.array([O.rel_fro(got[:, c0:c0 + L], ref[:, c0:c0 + L]) for c0 in range(0, N, L)])
+
+
+def run_routes(case, act, gen):
+    cfg, _, images = case
+    inp = _inputs(case, act)
+    x = _dev(inp.x32, act)
+    ref, ref_fin = oracle_routes(case, act)
+    worst = []
+    fin = None
+    for r in range(4):
+        h = S.srnl_scan_create(_cfg_dict(inp.cfg, act, gen), one_hot(inp.params(), r))
+        try:
+            y = torch.empty_like(x)
+            f = torch.full((4, cfg.B, cfg.heads, S.STATE_FLOATS_D32), float("nan"), device="cuda") if r == 0 else None
+            S.srnl_scan_forward(h, x, y, f)
+            torch.cuda.synchronize()
+            S.srnl_scan_device_status(h)
+        finally:
+            h.close()
+        if f is not None:
+            fin = f.cpu().numpy()[:, list(images)]
+        got = O.gather(y.float().cpu().numpy()[list(images)], r)
+        assert np.all(np.isfinite(got))
+        L = O.default_chunk(cfg.H, cfg.W, r, cfg.chunk_row, cfg.chunk_col)
+        err = chunk_errors(got, ref[r], L)
+        worst.append((float(err.max()), int(err.argmax()), len(err)))
+        assert err.max() <= TOL[(act, gen)], f"route {r}: chunk {err.argmax()} of {len(err)} err {err.max():.3e}"
+    fin_err = O.rel_fro(fin, ref_fin)
+    print(f"\n[chunks] {cfg.name} alpha={cfg.alpha} {act}/{gen}: worst chunk per route "
+          + ", ".join(f"r{r}: {e:.2e} (chunk {c} of {n})" for r, (e, c, n) in enumerate(worst))
+          + f"; final states {fin_err:.2e}")
+    assert fin_err <= TOL[(act, gen)], f"final states: {fin_err:.3e}"
+
+
+@pytest.mark.parametrize("path", [("bf16", "bf16"), ("f32", "f32"), ("bf16", "f32")])
+def test_s1_every_chunk_of_every_route(path):
+    """hier_s1_56x56 launch (B = 32, 56 x 56, chunk 56: 56 chunks per route), images 0 and 31."""
+    run_routes(S1, *path)
+
+
+@pytest.mark.parametrize("path", [("bf16", "bf16"), ("f32", "f32")])
+def test_hires_every_chunk_of_every_route(path):
+    """hires_200x304 launch (B = 2): 200 row chunks of 304 tokens (five stages each) and 304
+    column chunks of 200 tokens (four stages each), image 1."""
+    run_routes(HIRES, *path)
+
+
+@pytest.mark.parametrize("path", [("bf16", "bf16"), ("f32", "f32")])
+def test_sequence_layer_every_chunk(path):
+    """Standalone layer, T = 3136 in 64-token chunks (49 chunks), separate queries."""
+    act, gen = path
+    alpha = 0.999
+    inp = make_seq_inputs(2, 3136, 64, 2, act, seed=5, mem_scale=0.3, vec_scale=0.05, sustain=Sustain())
+    h = S.srnl_seq_create(dict(B=2, T=3136, D=64, heads=2, d=32, alpha=alpha, eps=1e-6, chunk=64, act_dtype=act,
+                               gen_dtype=gen), inp.params())
+    try:
+        x = _dev(inp.x32, act)
+        q = _dev(inp.q32, act)
+        y = torch.empty_like(x)
+        fin = torch.full((2, 2, S.STATE_FLOATS_D32), float("nan"), device="cuda")
+        S.srnl_seq_forward(h, x, y, q=q, final_states=fin)
+        torch.cuda.synchronize()
+        S.srnl_seq_device_status(h)
+    finally:
+        h.close()
+    ref, ref_fin = O.sequence_forward(inp.x32, inp.params(), alpha_max=alpha, chunk=64, heads=2, queries=inp.q32)
+    err = chunk_errors(y.float().cpu().numpy(), ref, 64)
+    fin_err = O.rel_fro(fin.cpu().numpy(), ref_fin)
+    print(f"\n[chunks] sequence T=3136 {act}/{gen}: worst chunk {err.max():.2e} (chunk {err.argmax()} of "
+          f"{len(err)}); final states {fin_err:.2e}")
+    assert err.max() <= TOL[path], f"chunk {err.argmax()}: {err.max():.3e}"
+    assert fin_err <= TOL[path]
+
+
+def test_backward_every_chunk_s1_image():
+    """Backward on one sustained hier_s1_56x56 image (fp32 arithmetic, fp32 x and dy): dL/dx of
+    each route (one-hot scales) chunk by chunk in route order, and every parameter gradient,
+    against the gradient oracle at 1e-4."""
+    cfg = S1[0].replace(B=1, act_dtype="f32")
+    inp = make_inputs(cfg, seed=0, mem_scale=0.3, vec_scale=0.05, sustain=S1[1])
+    dout = make_cotangent(inp.x32.shape, seed=0)
+    worst = []
+    for r in range(4):
+        params = one_hot(inp.params(), r)
+        h = S.srnl_scan_create(_cfg_dict(cfg, "f32", "f32"), params)
+        try:
+            x, dy = _dev(inp.x32, "f32"), _dev(dout, "f32")
+            dx = torch.full_like(x, float("nan"))
+            grads = {k: torch.full(np.shape(params[k]), float("nan"), device="cuda") for k in S.GRAD_KEYS}
+            S.srnl_scan_backward(h, x, dy, dx, grads)
+            torch.cuda.synchronize()
+        finally:
+            h.close()
+        ref = GR.operator_backward(inp.x32, params, dout, alpha_max=cfg.alpha, eps=cfg.eps, heads=cfg.heads)
+        L = O.default_chunk(cfg.H, cfg.W, r)
+        err = chunk_errors(O.gather(dx.cpu().numpy(), r), O.gather(ref["x"], r), L)
+        worst.append(float(err.max()))
+        assert err.max() <= 1e-4, f"route {r}: dx chunk {err.argmax()} err {err.max():.3e}"
+        for k in S.GRAD_KEYS:
+            ek = O.rel_fro(grads[k].cpu().numpy(), ref[k])
+            assert ek <= 1e-4, f"route {r}: d{k} err {ek:.3e}"
+    print(f"\n[chunks] backward hier_s1 image alpha={cfg.alpha}: worst dx chunk per route "
+          + ", ".join(f"{e:.2e}" for e in worst))
