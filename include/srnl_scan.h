@@ -153,26 +153,39 @@ SRNL_API srnl_status srnl_scan_forward_host(srnl_scan* h, const void* x_host, vo
  * memory through its own pool, where a raw allocation bypasses its accounting,
  * and latency-critical loops where an allocation may synchronise the device.
  * No handle is created and nothing is allocated or freed; the scratch (packed
- * parameters, projected queries, route partials) is a file-scope device array
- * of SRNL_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds
- * until the process exits.
- *   cfg    : same rules as srnl_scan_create.
- *   params : DEVICE pointers on the current device, same layouts as
- *            srnl_scan_params; W_q 16-byte aligned.
- *   x, y   : DEVICE pointers as in srnl_scan_forward.
- * A workload needing more than SRNL_NOALLOC_SCRATCH_BYTES of scratch
- * (about 18 bytes per activation element on the bf16 path, 20 on fp32, plus
- * the parameters) is rejected with SRNL_E_INVAL and a message giving both
- * sizes.  The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the array and it keeps the last
- * call's contents (nothing in it needs to start at zero); calls that overlap
- * on the GPU race.  Errors are reported through srnl_scan_last_error(NULL).
+ * parameters, projected queries, route partials, a status word) is a
+ * file-scope device array of SRNL_NOALLOC_SCRATCH_BYTES that every GPU loading
+ * this library holds until the process exits.
+ *   cfg    : same rules as srnl_scan_create; head dim d = 32 only.
+ *   params : DEVICE (or managed) pointers on the current device, same layouts
+ *            as srnl_scan_params, each 4-byte aligned (fp32 arrays).
+ *   x, y   : DEVICE (or managed) pointers on the current device as in
+ *            srnl_scan_forward, 16-byte aligned, not overlapping.
+ * Host pointers, pointers of another device, misaligned pointers and a
+ * workload needing more than SRNL_NOALLOC_SCRATCH_BYTES of scratch (about
+ * 18 bytes per activation element on the bf16 path, 20 on fp32, plus the
+ * parameters) are rejected with SRNL_E_INVAL before anything is launched;
+ * the message gives the reason (and both sizes).  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress) and sets
+ * the kernels' function attributes with that device current; make that first
+ * call before any stream capture.  All calls share the array and it keeps the
+ * last call's contents: each call first clears the status word (an
+ * asynchronous memset on `stream`), and everything else it reads it writes
+ * itself; calls that overlap on the GPU race.  Argument and launch errors come
+ * back as the status and through srnl_scan_last_error(NULL); a bounded
+ * in-kernel wait that gives up is reported by srnl_scan_noalloc_status.
  * Asynchronous on `stream`. */
 #define SRNL_NOALLOC_SCRATCH_BYTES (32u << 20)
 SRNL_API srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
                                                const srnl_scan_params* params,
                                                const void* x, void* y, void* stream);
+
+/* Device status of the last srnl_scan_forward_noalloc on the current device (no
+ * counterpart on the pages either): waits for `stream`, then reads the status word of the
+ * shared scratch array.  Returns SRNL_OK, or SRNL_E_TIMEOUT when a bounded in-kernel wait of
+ * that forward gave up (its y is then unspecified).  The next no-allocation forward clears
+ * the word.  Allocates nothing. */
+SRNL_API srnl_status srnl_scan_noalloc_status(void* stream);
 
 /* Test hook: the device computes the route map the scan kernels use and
  * writes out[t] = raster index of the t-th token of `route`, t < H*W, into the
@@ -262,6 +275,13 @@ SRNL_API srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void*
  * SRNL_OK if the wait wrongly completed, SRNL_E_INVAL for wait_ms out of range (no device
  * work), SRNL_E_CUDA on a CUDA error.  Synchronous; the message is srnl_scan_last_error(NULL). */
 SRNL_API srnl_status srnl_selftest_wait_timeout(int wait_ms);
+
+/* The same bounded wait on a barrier nothing completes, run asynchronously on `stream`
+ * with the no-allocation forward's status word as its status (1 <= wait_ms <= 5000): after
+ * it, srnl_scan_noalloc_status returns SRNL_E_TIMEOUT until the next no-allocation forward
+ * clears the word.  Tests the no-allocation forward's failure report without a fault.
+ * Allocates nothing. */
+SRNL_API srnl_status srnl_selftest_noalloc_wait_timeout(int wait_ms, void* stream);
 
 /* Bytes of device workspace the handle holds (packed params excluded). */
 SRNL_API size_t srnl_scan_workspace_bytes(const srnl_scan* h);

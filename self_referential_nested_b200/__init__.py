@@ -35,7 +35,8 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_seq_create", "srnl_seq_forward", "srnl_seq_device_status", "srnl_seq_last_error",
             "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count",
             "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
-            "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout")
+            "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout",
+            "srnl_scan_noalloc_status", "srnl_selftest_noalloc_wait_timeout")
 
 
 class SrnlError(RuntimeError):
@@ -125,12 +126,15 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_scan_backward.argtypes = [vp, vp, vp, vp, ctypes.POINTER(_Grads), vp]
     lib.srnl_seq_backward.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_SeqGrads), vp]
     lib.srnl_selftest_wait_timeout.argtypes = [i]
+    lib.srnl_scan_noalloc_status.argtypes = [vp]
+    lib.srnl_selftest_noalloc_wait_timeout.argtypes = [i, vp]
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
                  "srnl_scan_stage_times", "srnl_scan_device_status", "srnl_seq_create", "srnl_seq_forward",
                  "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count",
                  "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
-                 "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout"):
+                 "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout",
+            "srnl_scan_noalloc_status", "srnl_selftest_noalloc_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -272,6 +276,24 @@ def srnl_scan_forward_noalloc(cfg: Dict, params_dev: Dict, x, y, stream=None) ->
     st = lib.srnl_scan_forward_noalloc(ctypes.byref(c), ctypes.byref(p), _ptr(x), _ptr(y), _stream(stream))
     if st != SRNL_OK:
         raise SrnlError(st, "srnl_scan_forward_noalloc", lib.srnl_scan_last_error(None).decode())
+
+
+def srnl_scan_noalloc_status(stream=None) -> None:
+    """Raise SrnlError if a bounded in-kernel wait of the last allocation-free forward on the
+    current device gave up (waits for ``stream`` first)."""
+    lib = load_library()
+    st = lib.srnl_scan_noalloc_status(_stream(stream))
+    if st != SRNL_OK:
+        raise SrnlError(st, "srnl_scan_noalloc_status", lib.srnl_scan_last_error(None).decode())
+
+
+def srnl_selftest_noalloc_wait_timeout(wait_ms: int = 50, stream=None) -> None:
+    """Run a bounded wait that must give up, recording its status where the allocation-free
+    forward records its own (asynchronous)."""
+    lib = load_library()
+    st = lib.srnl_selftest_noalloc_wait_timeout(int(wait_ms), _stream(stream))
+    if st != SRNL_OK:
+        raise SrnlError(st, "srnl_selftest_noalloc_wait_timeout", lib.srnl_scan_last_error(None).decode())
 
 
 def srnl_scan_route_index(h: SrnlScan, route: int, out, stream=None) -> None:

@@ -12,9 +12,11 @@
 // stand-in, so its device address is looked up with cudaGetSymbolAddress once
 // per device, on the first call made with that device current, and cached.
 //
-// All calls share the array and it keeps the last call's contents.  Nothing in
-// it has to start at zero: every byte a call reads is written earlier in the
-// same call (pack, projection, scan in that order on the caller's stream).
+// All calls share the array and it keeps the last call's contents.  Only the
+// status word at its start must begin at zero, and every call clears it first
+// (an asynchronous memset on the caller's stream); every other byte a call
+// reads is written earlier in the same call (pack, projection, scan in that
+// order on the caller's stream).  srnl_scan_noalloc_status reads the word back.
 // Calls that overlap on the GPU (for example on two streams) race on the array.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -38,7 +40,8 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the scratch array for the current device (set up once per device).
+// Device address of the scratch array for the current device.  Set up once per device, with
+// that device current: the array's address, and the kernels' one-time function attributes.
 srnl_status scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -58,6 +61,11 @@ srnl_status scratch_address(void** out) {
       srnl::set_thread_error(std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(e));
       return SRNL_E_CUDA;
     }
+    e = srnl::prepare_kernels();
+    if (e != cudaSuccess) {
+      srnl::set_thread_error(std::string("kernel attributes: ") + cudaGetErrorString(e));
+      return SRNL_E_CUDA;
+    }
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -65,6 +73,18 @@ srnl_status scratch_address(void** out) {
 }
 
 size_t round_up(size_t n) { return (n + 255) & ~size_t(255); }
+
+// A pointer the kernels may read or write on the current device: device memory of this
+// device, or managed memory.  Host memory (pageable, pinned or mapped) is refused.
+bool on_this_device(const void* p, int dev) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();   // reset the runtime's last error after the failed query
+    return false;
+  }
+  if (a.type == cudaMemoryTypeManaged) return true;
+  return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
 
 // W_q copy (bf16-rounded on the bf16 path, plus a bf16 copy for the tensor-core projection)
 // and G = [M_k0; M_v0; m_eta0; m_alpha0] per (route, head), the layouts the kernels read.
@@ -119,10 +139,19 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
     srnl::set_thread_error("x or y is NULL");
     return SRNL_E_INVAL;
   }
-  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u) ||
-      (reinterpret_cast<uintptr_t>(p->W_q) & 15u)) {
-    srnl::set_thread_error("x, y and W_q must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u)) {
+    srnl::set_thread_error("x and y must be 16-byte aligned");
     return SRNL_E_INVAL;
+  }
+  {
+    // the kernels read every parameter array as fp32 scalars or float4 rows of 4-aligned
+    // starts; a pointer that is not 4-byte aligned would fault on the device
+    const void* ps[7] = {p->W_q, p->scales, p->M_mem0, p->M_k0, p->M_v0, p->m_eta0, p->m_alpha0};
+    for (const void* q : ps)
+      if (reinterpret_cast<uintptr_t>(q) & 3u) {
+        srnl::set_thread_error("every parameter pointer must be 4-byte aligned (fp32 arrays)");
+        return SRNL_E_INVAL;
+      }
   }
   const bool act_bf16 = cfg->act_dtype == SRNL_BF16, gen_bf16 = cfg->gen_dtype == SRNL_BF16;
   const size_t tokens = (size_t)cfg->B * cfg->H * cfg->W;
@@ -148,6 +177,20 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
                            std::to_string(kNoallocScratchBytes));
     return SRNL_E_INVAL;
   }
+  {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      srnl::set_thread_error("cudaGetDevice failed");
+      return SRNL_E_CUDA;
+    }
+    const void* ps[9] = {x, y, p->W_q, p->scales, p->M_mem0, p->M_k0, p->M_v0, p->m_eta0, p->m_alpha0};
+    const char* names[9] = {"x", "y", "W_q", "scales", "M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0"};
+    for (int i = 0; i < 9; ++i)
+      if (!on_this_device(ps[i], dev)) {
+        srnl::set_thread_error(std::string(names[i]) + " is not device (or managed) memory of the current device");
+        return SRNL_E_INVAL;
+      }
+  }
   void* base = nullptr;
   st = scratch_address(&base);
   if (st != SRNL_OK) return st;
@@ -162,11 +205,13 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   float* yr = reinterpret_cast<float*>(s8 + g_b + q_b);
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(dev_err, 0, sizeof(int), cs);   // status of this call
   const size_t n_pack = n_wq > n_g ? n_wq : n_g;
-  noalloc_pack_kernel<<<(unsigned)((n_pack + 255) / 256), 256, 0, cs>>>(
-      p->W_q, Wq, Wqb, (int64_t)n_wq, gen_bf16, p->M_k0, p->M_v0, p->m_eta0, p->m_alpha0, G, (int64_t)n_g);
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) e = srnl::prepare_kernels();
+  if (e == cudaSuccess) {
+    noalloc_pack_kernel<<<(unsigned)((n_pack + 255) / 256), 256, 0, cs>>>(
+        p->W_q, Wq, Wqb, (int64_t)n_wq, gen_bf16, p->M_k0, p->M_v0, p->m_eta0, p->m_alpha0, G, (int64_t)n_g);
+    e = cudaGetLastError();
+  }
 
   srnl::ScanGeom g{};
   g.B = cfg->B; g.H = cfg->H; g.W = cfg->W; g.C = cfg->C; g.heads = cfg->heads;
@@ -181,6 +226,44 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   if (e == cudaSuccess) e = srnl::launch_fuse(g, yr, y, cs);
   if (e != cudaSuccess) {
     srnl::set_thread_error(std::string("no-allocation forward launch: ") + cudaGetErrorString(e));
+    return SRNL_E_CUDA;
+  }
+  return SRNL_OK;
+}
+
+extern "C" srnl_status srnl_scan_noalloc_status(void* stream) {
+  srnl::set_thread_error("");
+  void* base = nullptr;
+  const srnl_status st = scratch_address(&base);
+  if (st != SRNL_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_noalloc_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) {
+    srnl::set_thread_error(std::string("no-allocation status read: ") + cudaGetErrorString(e));
+    return SRNL_E_CUDA;
+  }
+  if (v != 0) {
+    srnl::set_thread_error("a bounded in-kernel wait of the last no-allocation forward gave up");
+    return static_cast<srnl_status>(v);
+  }
+  return SRNL_OK;
+}
+
+extern "C" srnl_status srnl_selftest_noalloc_wait_timeout(int wait_ms, void* stream) {
+  srnl::set_thread_error("");
+  if (wait_ms < 1 || wait_ms > 5000) {
+    srnl::set_thread_error("wait_ms must lie in [1, 5000]");
+    return SRNL_E_INVAL;
+  }
+  void* base = nullptr;
+  const srnl_status st = scratch_address(&base);
+  if (st != SRNL_OK) return st;
+  const cudaError_t e = srnl::launch_wait_probe((unsigned long long)wait_ms * 1000000ull,
+                                                static_cast<int*>(base), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    srnl::set_thread_error(std::string("self-test launch: ") + cudaGetErrorString(e));
     return SRNL_E_CUDA;
   }
   return SRNL_OK;

@@ -32,6 +32,13 @@ __global__ void bounded_wait_probe_kernel(unsigned long long limit_ns, int* stat
 
 }  // namespace
 
+namespace srnl {
+cudaError_t launch_wait_probe(unsigned long long limit_ns, int* status, cudaStream_t s) {
+  bounded_wait_probe_kernel<<<1, 32, 0, s>>>(limit_ns, status);
+  return cudaGetLastError();
+}
+}  // namespace srnl
+
 extern "C" srnl_status srnl_selftest_wait_timeout(int wait_ms) {
   if (wait_ms < 1 || wait_ms > 5000) {
     srnl::set_thread_error("wait_ms must lie in [1, 5000]");
