@@ -24,15 +24,22 @@ __device__ __forceinline__ float softplus_f(float z) { return fmaxf(z, 0.f) + lo
 // phi(z) = tanh(z) / z, by 1 - z^2/3 below 1e-4.
 __device__ __forceinline__ float phi_f(float z) { return z < 1e-4f ? 1.f - z * z * (1.f / 3.f) : tanhf(z) / z; }
 
-// phi'(z): the Taylor series -2z/3 + 8z^3/15 - 102z^5/315 + 496z^7/2835 of the derivative of
-// tanh(z)/z below 0.25 (where the closed form cancels in fp32), else (z (1 - tanh^2 z) - tanh z) / z^2.
-__device__ __forceinline__ float dphi_f(float z) {
+// phi'(z) for z >= 0: below 0.25 the Taylor series -2z/3 + 8z^3/15 - 102z^5/315 + 496z^7/2835
+// of the derivative of tanh(z)/z (the closed form cancels there in fp32), else
+// (z sech^2 z - tanh z) / z^2, with sech^2 z = 4e / (1 + e)^2 and e = exp(-2z) returned in
+// sech2 (0 below 0.25, where it is not used).  1 - tanh^2 z would lose the small value once
+// tanh z rounds near 1: its relative error reaches 1e-3 around z = 5.
+__device__ __forceinline__ float dphi_f(float z, float& sech2) {
   if (z < 0.25f) {
     const float z2 = z * z;
+    sech2 = 0.f;
     return z * (-2.f / 3.f + z2 * (8.f / 15.f + z2 * (-102.f / 315.f + z2 * (496.f / 2835.f))));
   }
-  const float t = tanhf(z);
-  return (z * (1.f - t * t) - t) / (z * z);
+  const float e = expf(-2.f * z);
+  const float inv = 1.f / (1.f + e);
+  const float t = (1.f - e) * inv;
+  sech2 = 4.f * e * inv * inv;
+  return (z * sech2 - t) / (z * z);
 }
 
 // Scalar gates of one token from |k|^2, |k - v|^2, a and beta (the forward's clamp decisions):
@@ -75,8 +82,12 @@ __device__ __forceinline__ void gate_backward_scalars_f(float* sc, float al, flo
     if (binds) dal -= deta1 / gain;
   } else {                                                   // eta1 = eta0 phi(eta0 g / (1 - alpha_t))
     const float z = eta0 * gain / m;
-    const float dz = deta1 * eta0 * dphi_f(z);
-    deta0 = deta1 * phi_f(z) + dz * gain / m;
+    float sech2;
+    const float dph = dphi_f(z, sech2);
+    const float dz = deta1 * eta0 * dph;
+    // d(eta0 phi(eta0 g / m)) / d eta0 = phi(z) + z phi'(z) = sech^2 z: taken directly above the
+    // series range, where the sum of the two would cancel
+    deta0 = (z < 0.25f) ? deta1 * phi_f(z) + dz * gain / m : deta1 * sech2;
     dgain = dz * eta0 / m;
     dal += dz * eta0 * gain / (m * m);
   }
