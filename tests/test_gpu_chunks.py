@@ -14,6 +14,10 @@ full rows on the row routes, full columns on the column routes, the boundary sta
 chunk generating the next).  Every chunk must match the float64 oracle on its own: 1e-4 on the
 fp32 path, 2e-2 on the bf16 path (relative Frobenius error of the chunk).  The worst chunk of
 each case is printed (run pytest with -s to see it).
+
+The oracle receives the retention cap and the key stabiliser as the library does, as fp32
+values: with alpha_t = alpha on every token, a cap of 0.99995 that differs from its fp32
+value by 3e-8 would otherwise drift the two apart by 60800 x 3e-8 = 2e-3 over a HiRes route.
 """
 import functools
 
@@ -49,6 +53,11 @@ def _dev(a32, act):
     if act == "bf16":
         return torch.from_numpy(bf16_round_bits(a32).view(np.int16)).cuda().view(torch.bfloat16)
     return torch.from_numpy(np.ascontiguousarray(a32, dtype=np.float32)).cuda()
+
+
+def f32(v):
+    """The value a float field of the C config struct holds."""
+    return float(np.float32(v))
 
 
 def _cfg_dict(cfg, act, gen):
@@ -90,7 +99,7 @@ def oracle_routes(case, act):
             arr = np.asarray(getattr(inp, key), np.float64)[r]
             inits[name] = np.broadcast_to(arr[None], (n,) + arr.shape).reshape((-1,) + arr.shape[1:]).copy()
         L = O.default_chunk(cfg.H, cfg.W, r, cfg.chunk_row, cfg.chunk_col)
-        y, fin, _ = O.scan_five_memory(per_head(x, r), per_head(q, r), inits, L, cfg.alpha, cfg.eps)
+        y, fin, _ = O.scan_five_memory(per_head(x, r), per_head(q, r), inits, L, f32(cfg.alpha), f32(cfg.eps))
         outs.append(y.reshape(n, nh, N, d).transpose(0, 2, 1, 3).reshape(n, N, cfg.C))
         fins.append(np.concatenate([fin[k].reshape(n * nh, -1) for k in ("M_mem", "M_k", "M_v", "m_eta", "m_alpha")],
                                    axis=1).reshape(n, nh, -1))
@@ -169,7 +178,8 @@ def test_sequence_layer_every_chunk(path):
         S.srnl_seq_device_status(h)
     finally:
         h.close()
-    ref, ref_fin = O.sequence_forward(inp.x32, inp.params(), alpha_max=alpha, chunk=64, heads=2, queries=inp.q32)
+    ref, ref_fin = O.sequence_forward(inp.x32, inp.params(), alpha_max=f32(alpha), eps=f32(1e-6), chunk=64, heads=2,
+                                      queries=inp.q32)
     err = chunk_errors(y.float().cpu().numpy(), ref, 64)
     fin_err = O.rel_fro(fin.cpu().numpy(), ref_fin)
     print(f"\n[chunks] sequence T=3136 {act}/{gen}: worst chunk {err.max():.2e} (chunk {err.argmax()} of "
@@ -197,7 +207,8 @@ def test_backward_every_chunk_s1_image():
             torch.cuda.synchronize()
         finally:
             h.close()
-        ref = GR.operator_backward(inp.x32, params, dout, alpha_max=cfg.alpha, eps=cfg.eps, heads=cfg.heads)
+        ref = GR.operator_backward(inp.x32, params, dout, alpha_max=f32(cfg.alpha), eps=f32(cfg.eps),
+                                   heads=cfg.heads)
         L = O.default_chunk(cfg.H, cfg.W, r)
         err = chunk_errors(O.gather(dx.cpu().numpy(), r), O.gather(ref["x"], r), L)
         worst.append(float(err.max()))
