@@ -60,6 +60,11 @@ namespace {
 
 constexpr int kThreadsTc = 192;
 constexpr int kTile = kUmmaM * 64;      // 128 rows x 32 bf16: one K = 32 operand tile
+// The Z product's A operand tiles space their K-adjacent core matrices 144 B apart (not 128):
+// the scalar column stores of Kd^T (lanes = consecutive K) then fall in distinct banks.
+constexpr uint32_t kZCore = 144;                       // LBO: K-adjacent core matrices
+constexpr uint32_t kZGroup = 4 * kZCore;               // SBO: 8-row groups (576 B)
+constexpr int kTileZ = (kUmmaM / 8) * kZGroup;         // 9216 B per K = 32 sub-tile
 constexpr int kB1Rows = 96;             // M1 B operand: 64 keys + 32 rows of Q_s
 constexpr uint32_t kTmemColsTc = 256;   // two halves of 128 columns
 constexpr uint32_t kColM1 = 0;          // W, Gen, M1 and Y accumulate from column 0 of a half
@@ -77,8 +82,8 @@ struct alignas(128) TcSmem {
   alignas(128) unsigned char b1l[kB1Rows * 64];
   // Z A operand, K halves j < 32 and j >= 32: rows 0..31 Kd^T, rows 32..63 free,
   // rows 64..127 Mz^T.  Rows 32..63 hold the right-hand sides b^T during the solve.
-  alignas(128) unsigned char zah[2][kTile];
-  alignas(128) unsigned char zal[2][kTile];
+  alignas(128) unsigned char zah[2][kTileZ];
+  alignas(128) unsigned char zal[2][kTileZ];
   // Z B operand: -S (row r, K = token j)
   alignas(128) unsigned char zbh[2][kD * 64];
   alignas(128) unsigned char zbl[2][kD * 64];
@@ -93,11 +98,12 @@ struct alignas(128) TcSmem {
   alignas(16) float qsT[kD][kD + 1];            // Q_s transposed, fp32 (column c in row c)
   alignas(16) float lam[kStage];                // Lambda_t (log2 retention prefix)
   alignas(16) float eta[kStage];
+  alignas(16) float cf32[32];                   // 2^(Lambda_31 - Lambda_j) eta_j for j < 32
   alignas(16) float scale[kD];
   alignas(16) float4 gpart[kStage];            // readout-warp halves of ||k~||^2, k~.v, ||v||^2
   alignas(16) float4 gpar[kStage];             // gate scalars: 1/||k~||, alpha, g(t, T-1) eta, live
   float wsum;                                   // prefix of the first token warp
-  alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y;
+  alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y, mbar_c;
   uint32_t tmem_base;
   int wait_failed;
 };
@@ -106,7 +112,7 @@ static_assert(offsetof(TcSmem, yal) + 2 * 64 * 64 <= sizeof(TcSmem), "Y operand 
 static_assert(offsetof(TcSmem, a1l) == offsetof(TcSmem, a1h) + kTile, "A pieces");
 static_assert(offsetof(TcSmem, b1h) == offsetof(TcSmem, a1h) + 2 * kTile, "A pieces");
 static_assert(offsetof(TcSmem, b1l) == offsetof(TcSmem, b1h) + kB1Rows * 64, "A pieces");
-static_assert(offsetof(TcSmem, zal) == offsetof(TcSmem, zah) + 2 * kTile, "b pieces");
+static_assert(offsetof(TcSmem, zal) == offsetof(TcSmem, zah) + 2 * kTileZ, "b pieces");
 
 struct TcArgs {
   const void* x;
@@ -132,10 +138,27 @@ __device__ __forceinline__ float* neg_a_row(TcSmem& sm, int j) {
   return reinterpret_cast<float*>(base) + (j & 15) * kStage;
 }
 
-// b^T[r][t] (right-hand sides) in rows 32..63 of the four Z A sub-tiles.
-__device__ __forceinline__ float* rhs_row(TcSmem& sm, int r) {
-  return reinterpret_cast<float*>(&sm.zah[0][0] + (r >> 3) * kTile + 2048) + (r & 7) * kStage;
+__device__ __forceinline__ const float* neg_a_col(const TcSmem& sm, int j) {
+  const int p = j >> 4;
+  const unsigned char* base = p < 2 ? sm.a1h + p * kTile : sm.b1h + (p - 2) * (kB1Rows * 64);
+  return reinterpret_cast<const float*>(base) + (j & 15) * kStage;
 }
+
+// b^T[r][t] (right-hand sides) in rows 32..63 of the four Z A sub-tiles, 64 floats per row r.
+// The 16-byte chunks of a row are permuted by r & 7 (rhs_chunk), so that the solve warp's
+// lanes r reading the same chunk index hit distinct banks.
+__device__ __forceinline__ float* rhs_row(TcSmem& sm, int r) {
+  return reinterpret_cast<float*>(&sm.zah[0][0] + (r >> 3) * kTileZ + 4 * kZGroup) + (r & 7) * kStage;
+}
+static_assert(8 * kStage * 4 <= 4 * (int)kZGroup, "right-hand sides fit in rows 32..63 of a Z A sub-tile");
+
+// Byte offset of element (row, k) of a Z A sub-tile (the padded layout above).
+__device__ __forceinline__ uint32_t zoff(int row, int k) {
+  return (uint32_t)((row >> 3) * kZGroup + (k >> 3) * kZCore + (row & 7) * 16 + (k & 7) * 2);
+}
+
+// Offset in floats of chunk i (tokens 4i .. 4i + 3) in row r of the right-hand sides.
+__device__ __forceinline__ int rhs_chunk(int r, int i) { return (i ^ (r & 7)) << 2; }
 
 // 8 fp32 values -> bf16 hi and lo, each one 16-byte core-matrix row.
 __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
@@ -201,6 +224,129 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Forward substitution of one row of the stage's shared unit lower-triangular system over the
+// tokens [BASE, BASE + TB), on the lane that owns the row: b[i] holds the right-hand side of
+// token BASE + i, already reduced by every earlier token's contribution, and leaves as its
+// solution s.  No value crosses lanes: the columns of -A are read with broadcast loads (every
+// lane of the warp reads the same address).  Blocks of 4 columns J:
+//   - the 4 x 4 diagonal block is solved in registers (s_j = b_j, then the later b of the block);
+//   - the next block's 4 right-hand sides take block J's contribution first (the chain);
+//   - the remaining rows take it afterwards, off the chain.
+// The -A values the chain needs (the next block's diagonal block and its coupling to block J)
+// are loaded one block ahead.  TB is a multiple of 8; past the stage's tokens the right-hand
+// sides and the columns of A are zero, so those s stay zero.
+template <int BASE, int TB>
+__device__ __forceinline__ void solve_block(const TcSmem& sm, float (&b)[TB]) {
+  constexpr int NB = TB / 4;
+  // dg[i] = -A[j0 .. j0 + 3][j0 + i] (i = 0..2): the diagonal block of block J (rows as a float4)
+  // cp[i] = -A[j0 + 4 .. j0 + 7][j0 + i] (i = 0..3): block J's columns on the next block's rows
+  float4 dg[3], cp[4];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) dg[i] = *reinterpret_cast<const float4*>(neg_a_col(sm, BASE + i) + BASE);
+  if (NB > 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cp[i] = *reinterpret_cast<const float4*>(neg_a_col(sm, BASE + i) + BASE + 4);
+  }
+#pragma unroll
+  for (int J = 0; J < NB; ++J) {
+    const int j0 = 4 * J;   // local index; the token is BASE + j0
+    b[j0 + 1] = fmaf(dg[0].y, b[j0], b[j0 + 1]);
+    b[j0 + 2] = fmaf(dg[0].z, b[j0], b[j0 + 2]);
+    b[j0 + 3] = fmaf(dg[0].w, b[j0], b[j0 + 3]);
+    b[j0 + 2] = fmaf(dg[1].z, b[j0 + 1], b[j0 + 2]);
+    b[j0 + 3] = fmaf(dg[1].w, b[j0 + 1], b[j0 + 3]);
+    b[j0 + 3] = fmaf(dg[2].w, b[j0 + 2], b[j0 + 3]);
+    if (J + 1 < NB) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 s2 = f2(b[j0 + i], b[j0 + i]);
+        const float2 lo = __ffma2_rn(f2(cp[i].x, cp[i].y), s2, f2(b[j0 + 4], b[j0 + 5]));
+        const float2 hi = __ffma2_rn(f2(cp[i].z, cp[i].w), s2, f2(b[j0 + 6], b[j0 + 7]));
+        b[j0 + 4] = lo.x; b[j0 + 5] = lo.y; b[j0 + 6] = hi.x; b[j0 + 7] = hi.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 3; ++i)
+        dg[i] = *reinterpret_cast<const float4*>(neg_a_col(sm, BASE + j0 + 4 + i) + BASE + j0 + 4);
+      if (J + 2 < NB) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          cp[i] = *reinterpret_cast<const float4*>(neg_a_col(sm, BASE + j0 + 4 + i) + BASE + j0 + 8);
+      }
+#pragma unroll
+      for (int t4 = J + 2; t4 < NB; ++t4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 av = *reinterpret_cast<const float4*>(neg_a_col(sm, BASE + j0 + i) + BASE + 4 * t4);
+          const float2 s2 = f2(b[j0 + i], b[j0 + i]);
+          const float2 lo = __ffma2_rn(f2(av.x, av.y), s2, f2(b[4 * t4], b[4 * t4 + 1]));
+          const float2 hi = __ffma2_rn(f2(av.z, av.w), s2, f2(b[4 * t4 + 2], b[4 * t4 + 3]));
+          b[4 * t4] = lo.x; b[4 * t4 + 1] = lo.y; b[4 * t4 + 2] = hi.x; b[4 * t4 + 3] = hi.y;
+        }
+      }
+    }
+  }
+}
+
+// Right-hand sides of tokens [BASE, BASE + TB) of row r from shared memory.
+template <int BASE, int TB>
+__device__ __forceinline__ void load_rhs(TcSmem& sm, int r, float (&b)[TB]) {
+  const float* src = rhs_row(sm, r);
+#pragma unroll
+  for (int i = 0; i < TB / 4; ++i) {
+    const float4 v = *reinterpret_cast<const float4*>(src + rhs_chunk(r, BASE / 4 + i));
+    b[4 * i] = v.x; b[4 * i + 1] = v.y; b[4 * i + 2] = v.z; b[4 * i + 3] = v.w;
+  }
+}
+
+// -S of tokens [BASE, BASE + 32) of row r into the Z B operand (row r, K = token), one
+// core-matrix row per 8 tokens, hi and lo; zeros past TB (the Z product contracts over all 64).
+template <int BASE, int TB>
+__device__ __forceinline__ void store_neg_s(TcSmem& sm, int r, const float (&b)[TB]) {
+#pragma unroll
+  for (int g8 = 0; g8 < 4; ++g8) {
+    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+    if (8 * g8 < TB) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = -b[8 * g8 + i];
+      split8(v, hi, lo);
+    }
+    *reinterpret_cast<uint4*>(sm.zbh[BASE / 32] + umma_off(r, 8 * g8)) = hi;
+    *reinterpret_cast<uint4*>(sm.zbl[BASE / 32] + umma_off(r, 8 * g8)) = lo;
+  }
+}
+
+// Zeros for -S of tokens [BASE, BASE + 32) of row r (tokens past the stage).
+template <int BASE>
+__device__ __forceinline__ void store_neg_s_zero(TcSmem& sm, int r) {
+#pragma unroll
+  for (int g8 = 0; g8 < 4; ++g8) {
+    *reinterpret_cast<uint4*>(sm.zbh[BASE / 32] + umma_off(r, 8 * g8)) = make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(sm.zbl[BASE / 32] + umma_off(r, 8 * g8)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Tokens [0, min(T, 32)) of row r: right-hand sides, solve, -S.
+template <int TB>
+__device__ __forceinline__ void solve_first(TcSmem& sm, int r) {
+  float b[TB];
+  load_rhs<0, TB>(sm, r, b);
+  solve_block<0, TB>(sm, b);
+  store_neg_s<0, TB>(sm, r, b);
+}
+
+// Tokens [32, T) of row r: right-hand sides reduced by the coupling c[t - 32] of the first 32
+// tokens (from TMEM), solve, -S.
+template <int TB>
+__device__ __forceinline__ void solve_second(TcSmem& sm, int r, const float (&c)[32]) {
+  float b[TB];
+  load_rhs<32, TB>(sm, r, b);
+#pragma unroll
+  for (int i = 0; i < TB; ++i) b[i] -= c[i];
+  solve_block<32, TB>(sm, b);
+  store_neg_s<32, TB>(sm, r, b);
 }
 
 // Number of stages that hold tokens: only the last chunk can be short.
@@ -282,6 +428,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_1)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_z)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_y)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_c)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -325,6 +472,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
   const uint32_t wb_lo = qb_is_qs ? smem_u32(sm.b1l) + 64 * 64 : smem_u32(sm.qbl);
 
   // readout warps: the stage whose z / y is still to be produced
+  uint32_t cpar = 0;   // phase of mbar_c (warp 0)
   bool pend = false;
   StageInfo pst{0, 0, 0};
   uint32_t phb = 0;
@@ -445,6 +593,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         tok_bar();
         const float gk = live ? exp2_fast(sm.lam[T - 1] - pre) * et : 0.f;
         sm.gpar[t] = make_float4(inv, al, gk, live ? 1.f : 0.f);
+        if (t < 32) sm.cf32[t] = exp2_fast(sm.lam[31] - pre) * et;   // 2^(Lambda_31 - Lambda_t) eta_t
       }
       named_bar(7, 128);
       {
@@ -461,7 +610,12 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         unsigned char* zh = sm.zah[t >> 5];
         unsigned char* zl = sm.zal[t >> 5];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) store_split(zh, zl, c0 + c, t & 31, gp.z * kt[c]);
+        for (int c = 0; c < 16; ++c) {
+          const float v = gp.z * kt[c];
+          const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+          *reinterpret_cast<__nv_bfloat16*>(zh + zoff(c0 + c, t & 31)) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(zl + zoff(c0 + c, t & 31)) = __float2bfloat16_rn(v - __bfloat162float(hi));
+        }
       }
       fence_async_smem();
     }
@@ -479,20 +633,45 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     }
     // ---- (D) -A and the right-hand sides (solve and token warps) | readout coefficients
     // (readout warps) | then the token warps copy the next stage and store y of the previous one
-    if (is_s || is_k) {
+    if (is_s) {
+      // -A (warps 0 and 1; thread = token t = TMEM lane).  Columns j < 32 of tokens t >= 32
+      // (warp 1) lie below the split point 31 <= t - 1, so
+      // g(j, t - 1) = 2^(Lambda_{t-1} - Lambda_31) 2^(Lambda_31 - Lambda_j) with both factors <= 1:
+      // one exp2 per thread and the precomputed column factors.  The diagonal 32 x 32 blocks take
+      // one exp2 per element.  Columns j >= 32 of tokens t < 32 are above the diagonal; the solve
+      // never reads them, so nobody writes them.
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
-      const int t = is_k ? tid - 128 : tid;  // TMEM lane = token
+      const int t = tid;
       const bool live = t < T;
-      const int j0 = is_k ? 32 : 0;          // this thread's columns j of A: [j0, j0 + 32)
-      float g[32], bv[kD];
+      const float lp = (t > 0 && live) ? sm.lam[t - 1] : 0.f;  // Lambda_{t-1}
+      float g[32];
+      if (warp == 1) {
+        SRNL_LD16(g, tmem_lane + hb + kColM1);
+        SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + 16);
+        tmem_wait_ld();
+        const float rf = live ? exp2_fast(lp - sm.lam[31]) : 0.f;
+#pragma unroll
+        for (int jb = 0; jb < 32; jb += 16) {
+          float cv[16];
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(&sm.cf32[jb + i]);
+            cv[i] = c4.x; cv[i + 1] = c4.y; cv[i + 2] = c4.z; cv[i + 3] = c4.w;
+          }
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = -rf * cv[i] * g[jb + i];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) neg_a_row(sm, jb + i)[t] = v[i];
+          // the same block as the coupling product's B operand: row t - 32, K = j, bf16 hi + lo
+          store_half_split(sm.b1h, sm.b1l, 64 + (t - 32), jb, v);
+        }
+        fence_async_smem();
+      }
+      const int j0 = 32 * warp;   // the diagonal block: columns [32 w, 32 w + 32)
       SRNL_LD16(g, tmem_lane + hb + kColM1 + j0);
       SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + j0 + 16);
-      if (is_k) {
-        SRNL_LD16(bv, tmem_lane + hb + kColZ0);
-        SRNL_LD16(bv + 16, tmem_lane + hb + kColZ0 + 16);
-      }
       tmem_wait_ld();
-      const float lp = (t > 0 && live) ? sm.lam[t - 1] : 0.f;  // Lambda_{t-1}
 #pragma unroll
       for (int jb = 0; jb < 32; jb += 16) {
         // the block's Lambda_j and eta_j first: the stores below may alias them
@@ -510,11 +689,18 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
 #pragma unroll
         for (int i = 0; i < 16; ++i) neg_a_row(sm, j0 + jb + i)[t] = v[i];
       }
-      if (is_k) {
-        const float cp = live ? exp2_fast(lp) : 0.f;
+    } else if (is_k) {
+      // the right-hand sides b^T[r][t] = 2^Lambda_{t-1} (Q_s u_t)[r] (token warps)
+      mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
+      const int t = tid - 128;
+      const bool live = t < T;
+      float bv[kD];
+      SRNL_LD16(bv, tmem_lane + hb + kColZ0);
+      SRNL_LD16(bv + 16, tmem_lane + hb + kColZ0 + 16);
+      tmem_wait_ld();
+      const float cp = (live && t > 0) ? exp2_fast(sm.lam[t - 1]) : (live ? 1.f : 0.f);
 #pragma unroll
-        for (int i = 0; i < kD; ++i) rhs_row(sm, i)[t] = cp * bv[i];
-      }
+      for (int i = 0; i < kD; ++i) rhs_row(sm, i)[rhs_chunk(i, t >> 2) + (t & 3)] = cp * bv[i];
     }
     if (is_k) {
       const int gt = tid - 128;
@@ -549,105 +735,91 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       SRNL_LD16(g + 32, tmem_lane + hb + kColM1 + 32);
       SRNL_LD16(g + 48, tmem_lane + hb + kColM1 + 48);
       tmem_wait_ld();
+      // as for -A: columns j < 32 of tokens t >= 32 (warp 3) factor at the split point 31 <= t;
+      // columns j >= 32 of tokens t < 32 (warp 2) are zero
+      const float rf = (warp == 3 && live) ? exp2_fast(lt - sm.lam[31]) : 0.f;
 #pragma unroll
       for (int jb = 0; jb < kStage; jb += 16) {
-        float lv[16], ev[16], v[16];
+        float v[16];
+        if (warp == 3 && jb < 32) {
 #pragma unroll
-        for (int i = 0; i < 16; i += 4) {
-          const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
-          const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
-          lv[i] = lj.x; lv[i + 1] = lj.y; lv[i + 2] = lj.z; lv[i + 3] = lj.w;
-          ev[i] = ej.x; ev[i + 1] = ej.y; ev[i + 2] = ej.z; ev[i + 3] = ej.w;
+          for (int i = 0; i < 16; i += 4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(&sm.cf32[jb + i]);
+            v[i] = rf * c4.x * g[jb + i]; v[i + 1] = rf * c4.y * g[jb + i + 1];
+            v[i + 2] = rf * c4.z * g[jb + i + 2]; v[i + 3] = rf * c4.w * g[jb + i + 3];
+          }
+        } else if (warp == 2 && jb >= 32) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        } else {
+          float lv[16], ev[16];
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
+            const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
+            lv[i] = lj.x; lv[i + 1] = lj.y; lv[i + 2] = lj.z; lv[i + 3] = lj.w;
+            ev[i] = ej.x; ev[i + 1] = ej.y; ev[i + 2] = ej.z; ev[i + 3] = ej.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            v[i] = (live && jb + i <= t) ? exp2_fast(lt - lv[i]) * ev[i] * g[jb + i] : 0.f;
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          v[i] = (live && jb + i <= t) ? exp2_fast(lt - lv[i]) * ev[i] * g[jb + i] : 0.f;
         unsigned char* th = sm.zah[jb >> 5];
         unsigned char* tl = sm.zal[jb >> 5];
 #pragma unroll
         for (int c = 0; c < 16; c += 8) {
           uint4 hi, lo;
           split8(v + c, hi, lo);
-          *reinterpret_cast<uint4*>(th + umma_off(64 + t, (jb & 31) + c)) = hi;
-          *reinterpret_cast<uint4*>(tl + umma_off(64 + t, (jb & 31) + c)) = lo;
+          *reinterpret_cast<uint4*>(th + zoff(64 + t, (jb & 31) + c)) = hi;
+          *reinterpret_cast<uint4*>(tl + zoff(64 + t, (jb & 31) + c)) = lo;
         }
       }
       fence_async_smem();
       ct_pend = live ? exp2_fast(lt) : 0.f;
     }
-    // ---- forward substitution (solve warps).  Thread: rows rg + 8 m (m = 0..3, rg = 4 warp +
-    // (lane & 3)), tokens [8 kb, 8 kb + 8) (kb = lane >> 2).  Two tokens per broadcast: the
-    // owner lanes of tokens t, t + 1 (kb == t / 8) finish s_{t+1} = b_{t+1} - A[t+1][t] s_t
-    // from their registers, then every lane subtracts A[t'][t] s_t + A[t'][t+1] s_{t+1}
-    // from its tokens t' (A is zero for t' <= t, so finished tokens stay as they are).
-    if (is_s) {
+    // ---- forward substitution (warp 0): lane r owns row r of Q (solve_rows), then writes -S.
+    if (warp == 0) {
       named_bar(5, 128);  // A and the right-hand sides (the token warps arrive without waiting)
-      const int rg = 4 * warp + (lane & 3), kb = lane >> 2;
-      float sv[4][8];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float* src = rhs_row(sm, rg + 8 * m) + 8 * kb;
-        const float4 v0 = *reinterpret_cast<const float4*>(src);
-        const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
-        sv[m][0] = v0.x; sv[m][1] = v0.y; sv[m][2] = v0.z; sv[m][3] = v0.w;
-        sv[m][4] = v1.x; sv[m][5] = v1.y; sv[m][6] = v1.z; sv[m][7] = v1.w;
+      switch ((min(T, 32) + 7) >> 3) {   // the smallest multiple of 8 tokens that covers them
+        case 1: solve_first<8>(sm, lane); break;
+        case 2: solve_first<16>(sm, lane); break;
+        case 3: solve_first<24>(sm, lane); break;
+        default: solve_first<32>(sm, lane); break;
       }
-      const int nblk = (T + 7) >> 3;
-#pragma unroll 1
-      for (int bt = 0; bt < nblk; ++bt) {
-        const int src = (bt << 2) | (lane & 3);
-        const float* abase = neg_a_row(sm, 8 * bt) + 8 * kb;
-#pragma unroll
-        for (int tl = 0; tl < 8; tl += 2) {
-          float a0[8], a1[8];
-          {
-            const float* ar = abase + tl * kStage;
-            const float4 p0 = *reinterpret_cast<const float4*>(ar);
-            const float4 p1 = *reinterpret_cast<const float4*>(ar + 4);
-            const float4 p2 = *reinterpret_cast<const float4*>(ar + kStage);
-            const float4 p3 = *reinterpret_cast<const float4*>(ar + kStage + 4);
-            a0[0] = p0.x; a0[1] = p0.y; a0[2] = p0.z; a0[3] = p0.w; a0[4] = p1.x; a0[5] = p1.y; a0[6] = p1.z; a0[7] = p1.w;
-            a1[0] = p2.x; a1[1] = p2.y; a1[2] = p2.z; a1[3] = p2.w; a1[4] = p3.x; a1[5] = p3.y; a1[6] = p3.z; a1[7] = p3.w;
-          }
-          float xs[4], ys[4];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const float xo = sv[m][tl];
-            const float yo = fmaf(a0[tl + 1], xo, sv[m][tl + 1]);
-            xs[m] = __shfl_sync(0xffffffffu, xo, src);
-            ys[m] = __shfl_sync(0xffffffffu, yo, src);
-          }
-          // the pair of tokens t + 2, t + 3 first: it feeds the next broadcast
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int i = ((tl + 2) & 7) ^ (2 * q);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const float2 r2 = __ffma2_rn(f2(a1[i], a1[i + 1]), f2(ys[m], ys[m]),
-                                           __ffma2_rn(f2(a0[i], a0[i + 1]), f2(xs[m], xs[m]), f2(sv[m][i], sv[m][i + 1])));
-              sv[m][i] = r2.x;
-              sv[m][i + 1] = r2.y;
-            }
-          }
+      if (T > 32) {
+        // the coupling of tokens 32.. to the first 32: C[r][t'] = sum_{j < 32} S[r][j] A[32 + t'][j]
+        // = (-S_1)(-A_21)^T on the tensor cores (A_21 as bf16 hi + lo in rows 64..95 of the M1 B
+        // tiles, written by warp 1), into the Z columns, which the Z product overwrites later
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t sh = smem_u32(sm.zbh[0]), sl = smem_u32(sm.zbl[0]);
+          const uint32_t ah = smem_u32(sm.b1h) + 64 * 64, al = smem_u32(sm.b1l) + 64 * 64;
+          mma_k32(tmem + hb + kColZ, sh, ah, idesc32, false);
+          mma_k32(tmem + hb + kColZ, sh, al, idesc32, true);
+          mma_k32(tmem + hb + kColZ, sl, ah, idesc32, true);
+          mma_commit(&sm.mbar_c);
         }
-      }
-      // -S into the Z B operand (row r, K = token): one core-matrix row per (row, hi/lo)
-      {
-        unsigned char* th = sm.zbh[kb >> 2];
-        unsigned char* tl = sm.zbl[kb >> 2];
-        const int k0 = 8 * (kb & 3);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          float v[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = -sv[m][i];
-          uint4 hi, lo;
-          split8(v, hi, lo);
-          *reinterpret_cast<uint4*>(th + umma_off(rg + 8 * m, k0)) = hi;
-          *reinterpret_cast<uint4*>(tl + umma_off(rg + 8 * m, k0)) = lo;
+        mbar_wait(&sm.mbar_c, cpar, &sm.wait_failed);
+        cpar ^= 1u;
+        float c[32];
+        SRNL_LD16(c, tmem + hb + kColZ);
+        SRNL_LD16(c + 16, tmem + hb + kColZ + 16);
+        tmem_wait_ld();
+        switch ((T - 32 + 7) >> 3) {
+          case 1: solve_second<8>(sm, lane, c); break;
+          case 2: solve_second<16>(sm, lane, c); break;
+          case 3: solve_second<24>(sm, lane, c); break;
+          default: solve_second<32>(sm, lane, c); break;
         }
+      } else {
+        store_neg_s_zero<32>(sm, lane);
       }
       fence_async_smem();
+    } else if (warp == 1) {
+      named_bar(5, 128);
     }
     // ---- (E) Z = [Kd^T; -; Mz^T] (-S)^T
     if (!is_k) {
@@ -657,11 +829,16 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
-          const uint32_t ah = smem_u32(sm.zah[kk]), al = smem_u32(sm.zal[kk]);
-          const uint32_t bh = smem_u32(sm.zbh[kk]), bl = smem_u32(sm.zbl[kk]);
-          mma_k32(tmem + hb + kColZ, ah, bh, idesc32, kk > 0);
-          mma_k32(tmem + hb + kColZ, ah, bl, idesc32, true);
-          mma_k32(tmem + hb + kColZ, al, bh, idesc32, true);
+#pragma unroll
+          for (int k16 = 0; k16 < 2; ++k16) {   // A steps 2 padded core matrices, B 2 plain ones
+            const uint32_t ao = k16 * 2 * kZCore, bo = k16 * 256;
+            const uint64_t ah = umma_desc_strided(smem_u32(sm.zah[kk]) + ao, kZCore, kZGroup);
+            const uint64_t al = umma_desc_strided(smem_u32(sm.zal[kk]) + ao, kZCore, kZGroup);
+            const uint64_t bh = umma_desc(smem_u32(sm.zbh[kk]) + bo), bl = umma_desc(smem_u32(sm.zbl[kk]) + bo);
+            mma_k16_desc(tmem + hb + kColZ, ah, bh, idesc32, kk + k16 > 0);
+            mma_k16_desc(tmem + hb + kColZ, ah, bl, idesc32, true);
+            mma_k16_desc(tmem + hb + kColZ, al, bh, idesc32, true);
+          }
         }
         mma_commit(&sm.mbar_z);
       }

@@ -28,6 +28,13 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
          ((uint64_t)(512u >> 4) << 32) | (1ull << 46);
 }
 
+// The same descriptor with other strides: K-adjacent core matrices lbo bytes apart, 8-row
+// groups sbo bytes apart (both multiples of 16).
+__device__ __forceinline__ uint64_t umma_desc_strided(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
 // Byte offset of element (row, k) of a [rows x 32] bf16 K-major operand tile.
 __host__ __device__ __forceinline__ uint32_t umma_off(int row, int k) {
   return (uint32_t)((row >> 3) * 512 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
@@ -54,6 +61,15 @@ __device__ __forceinline__ void mma_k32(uint32_t tmem, uint32_t a_smem, uint32_t
                                         bool accumulate) {
   mma_k16(tmem, a_smem, b_smem, idesc, accumulate);
   mma_k16(tmem, a_smem + 256, b_smem + 256, idesc, true);
+}
+
+// D[tmem] (+)= A B^T over one K = 16 step, with explicit descriptors.
+__device__ __forceinline__ void mma_k16_desc(uint32_t tmem, uint64_t ad, uint64_t bd, uint32_t idesc, bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
 }
 
 __device__ __forceinline__ void mma_commit(unsigned long long* bar) {
