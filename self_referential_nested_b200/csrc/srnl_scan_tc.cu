@@ -45,10 +45,15 @@
 //   Y    [z] M_mem0^T                   N = 32   y_t
 // TMEM holds two 128-column halves; consecutive stages alternate, so the readout of
 // one stage overlaps the generation of the next.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
+
+#include <cstring>
+#include <mutex>
 
 #include "srnl_common.cuh"
 #include "srnl_launch.h"
@@ -103,7 +108,7 @@ struct alignas(128) TcSmem {
   alignas(16) float4 gpart[kStage];            // readout-warp halves of ||k~||^2, k~.v, ||v||^2
   alignas(16) float4 gpar[kStage];             // gate scalars: 1/||k~||, alpha, g(t, T-1) eta, live
   float wsum;                                   // prefix of the first token warp
-  alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y, mbar_c;
+  alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y, mbar_c, mbar_x;
   uint32_t tmem_base;
   int wait_failed;
 };
@@ -129,6 +134,15 @@ struct TcArgs {
   bool act_bf16;
   bool hard_cap;
 };
+
+// Tensor maps of the bf16 activations and queries, [B][H][W][C]: "row" views tokens as one
+// dimension (B*H*W tokens of C channels; a stage of a row route is consecutive tokens) and
+// "col" as [B*H][W][C] (a stage of a column route is one column j: consecutive i at stride
+// W*C).  Boxes are 32 channels (one head) by 64 tokens.
+struct TcMaps {
+  CUtensorMap xr, xc, qr, qc;
+};
+constexpr uint32_t kBoxBytes = kStage * kD * 2;   // one 64-token x 32-channel bf16 box
 
 // -A[t][j] for j in [16p, 16p + 16) lives in the first 4 KB of a1h, a1l, b1h, b1l
 // (p = 0..3): the u and k rows of M1, dead between M1 and the next stage's gates.
@@ -394,7 +408,67 @@ __device__ __forceinline__ void tc_prefetch(TcSmem& sm, const StageInfo& si, con
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(const TcArgs a) {
+// One thread: the stage's x and q boxes into the staging area (the Y operand tiles, dead
+// between the Y product's completion and the next z), completing on mbar_x.  Row routes load
+// the 64 tokens from the stage's lowest raster index p_lo on; column routes the 64 rows of
+// column j from i_lo on.  Boxes may run past the image or the tensor (the rest is unused; TMA
+// fills what lies outside the tensor with zeros).  Coordinates: channels ch0 (a multiple of
+// 32, so 64-byte aligned), then tokens; never negative.
+__device__ __forceinline__ void tma_stage(TcSmem& sm, const TcMaps& m, const StageInfo& si, int r, int b, int ch0,
+                                          int H, int W) {
+  const uint32_t bar = smem_u32(&sm.mbar_x);
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kBoxBytes) : "memory");
+  const int t_lo = (r & 1) ? si.t0 + si.T - 1 : si.t0;      // route token at the lowest address
+  const int p = route_pos(r, t_lo, H, W);
+  if (r < 2) {
+    const int c1 = b * H * W + p;
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(sm.yah)), "l"(reinterpret_cast<uint64_t>(&m.xr)), "r"(ch0), "r"(c1), "r"(bar)
+        : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(sm.yal)), "l"(reinterpret_cast<uint64_t>(&m.qr)), "r"(ch0), "r"(c1), "r"(bar)
+        : "memory");
+  } else {
+    const int i = p / W, j = p - i * W;
+    const int c2 = b * H + i;
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(sm.yah)), "l"(reinterpret_cast<uint64_t>(&m.xc)), "r"(ch0), "r"(j), "r"(c2), "r"(bar)
+        : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(sm.yal)), "l"(reinterpret_cast<uint64_t>(&m.qc)), "r"(ch0), "r"(j), "r"(c2), "r"(bar)
+        : "memory");
+  }
+}
+
+// Whether a stage's tokens form one box: always on the row routes (consecutive raster
+// indices); on the column routes when they lie in one column (the default chunks are whole
+// columns; an overridden chunk length may cross a column boundary, and such a stage is
+// copied token by token instead).  The reverse column route walks the same columns.
+__device__ __forceinline__ bool stage_is_box(const StageInfo& si, int r, int H) {
+  return r < 2 || si.t0 / H == (si.t0 + si.T - 1) / H;
+}
+
+// Token warps (ht = 0..63): the staged boxes (64-byte rows, ascending raster order) into the
+// operand tiles in route order: x into rows t and 64 + t of the x tile, q into rows 64 + t of
+// the M1 A tile.  Reverse routes read the box backwards over the stage's T tokens.
+__device__ __forceinline__ void unstage(TcSmem& sm, const StageInfo& si, int r, int ht) {
+  for (int idx = ht; idx < kStage * 4; idx += 64) {
+    const int t = idx >> 2, part = idx & 3;
+    const int row = ((r & 1) && t < si.T) ? si.T - 1 - t : t;
+    const uint4 xv = *reinterpret_cast<const uint4*>(sm.yah + row * 64 + part * 16);
+    const uint4 qv = *reinterpret_cast<const uint4*>(sm.yal + row * 64 + part * 16);
+    *reinterpret_cast<uint4*>(sm.xa + umma_off(t, part * 8)) = xv;
+    *reinterpret_cast<uint4*>(sm.xa + umma_off(64 + t, part * 8)) = xv;
+    *reinterpret_cast<uint4*>(sm.a1h + umma_off(64 + t, part * 8)) = qv;
+  }
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(const TcArgs a,
+                                                                       const __grid_constant__ TcMaps maps) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw);
 
@@ -420,6 +494,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     uint4* z = reinterpret_cast<uint4*>(&sm);
     const int n16 = (int)(offsetof(TcSmem, qsT) / 16);
     for (int i = tid; i < n16; i += kThreadsTc) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_async_smem();   // the zeros land before any tensor copy into the same tiles
   }
   if (tid == 0) {
     sm.wait_failed = 0;
@@ -429,6 +504,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_z)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_y)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_c)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_x)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -453,9 +529,18 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
   if (tid < kD) sm.scale[tid] = a.scales[r * a.C + ch0 + tid];
 
   const int nst = live_stages(N, L);
+  uint32_t xpar = 0;   // phase of mbar_x (token warps)
   if (is_k && nst > 0) {
-    tc_prefetch(sm, stage_info(0, N, L), a, r, tok0, ch0, tid - 128);
-    cp_async_wait_all();
+    const StageInfo s0 = stage_info(0, N, L);
+    if (a.act_bf16 && stage_is_box(s0, r, a.H)) {
+      if (tid == 128) tma_stage(sm, maps, s0, r, b, ch0, a.H, a.W);
+      mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
+      xpar ^= 1u;
+      unstage(sm, s0, r, tid - 128);
+    } else {
+      tc_prefetch(sm, s0, a, r, tok0, ch0, tid - 128);
+      cp_async_wait_all();
+    }
   }
   fence_async_smem();
   tc_fence_before();
@@ -705,7 +790,9 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     if (is_k) {
       const int gt = tid - 128;
       named_bar_arrive(5, 128);  // this half of A and the right-hand sides are written
-      if (ne + 1 < nst) tc_prefetch(sm, stage_info(ne + 1, N, L), a, r, tok0, ch0, gt);
+      const StageInfo sn = stage_info(ne + 1 < nst ? ne + 1 : ne, N, L);
+      const bool next_box = a.act_bf16 && ne + 1 < nst && stage_is_box(sn, r, a.H);
+      if (!next_box && ne + 1 < nst) tc_prefetch(sm, sn, a, r, tok0, ch0, gt);
       if (pend) {  // y of the previous stage: the Y product was issued in (A)
         mbar_wait(&sm.mbar_y, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
         float y[kD];
@@ -722,7 +809,16 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
                             sm.scale[i + 3] * y[i + 3]);
         }
       }
-      cp_async_wait_all();
+      if (next_box) {
+        // the next stage's boxes into the staging area, which the Y product has finished reading
+        tok_bar();   // both token warps are past the Y wait
+        if (gt == 0) tma_stage(sm, maps, sn, r, b, ch0, a.H, a.W);
+        mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
+        xpar ^= 1u;
+        unstage(sm, sn, r, gt);
+      } else {
+        cp_async_wait_all();
+      }
       fence_async_smem();
     } else if (is_r) {
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
@@ -940,6 +1036,46 @@ cudaError_t prepare_scan_chunkwise_kernel() {
                               (int)sizeof(TcSmem));
 }
 
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+// The driver's tensor-map encoder, looked up once through the runtime (no link to libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// Row view: [B*H*W][C]; column view: [B*H][W][C].  bf16, box 32 channels x 64 tokens.
+bool encode_maps(const void* base, int B, int H, int W, int C, CUtensorMap* row, CUtensorMap* col) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint64_t rdim[2] = {(cuuint64_t)C, (cuuint64_t)B * H * W};
+  const cuuint64_t rstr[1] = {(cuuint64_t)C * 2};
+  const cuuint32_t rbox[2] = {(cuuint32_t)kD, (cuuint32_t)kStage};
+  CUresult e = enc(row, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), rdim, rstr, rbox, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (e != CUDA_SUCCESS) return false;
+  const cuuint64_t cdim[3] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)B * H};
+  const cuuint64_t cstr[2] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2};
+  const cuuint32_t cbox[3] = {(cuuint32_t)kD, 1, (cuuint32_t)kStage};
+  e = enc(col, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), cdim, cstr, cbox, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return e == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
                                   float* yr, float* finals, int* err, unsigned long long* binds,
                                   cudaStream_t s) {
@@ -951,7 +1087,14 @@ cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, con
   a.act_bf16 = g.act_bf16;
   a.hard_cap = g.hard_cap; a.binds = binds;
   const unsigned nseq = (unsigned)g.routes * (unsigned)g.B * (unsigned)g.heads;
-  srnl_scan_chunkwise_kernel<<<nseq, kThreadsTc, sizeof(TcSmem), s>>>(a);
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (g.act_bf16) {
+    if (!encode_maps(x, g.B, g.H, g.W, g.C, &maps.xr, &maps.xc) ||
+        !encode_maps(q, g.B, g.H, g.W, g.C, &maps.qr, &maps.qc))
+      return cudaErrorInvalidValue;
+  }
+  srnl_scan_chunkwise_kernel<<<nseq, kThreadsTc, sizeof(TcSmem), s>>>(a, maps);
   return cudaGetLastError();
 }
 
