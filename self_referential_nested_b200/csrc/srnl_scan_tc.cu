@@ -251,8 +251,8 @@ __device__ __forceinline__ void tc_fence_after() {
 // The -A values the chain needs (the next block's diagonal block and its coupling to block J)
 // are loaded one block ahead.  TB is a multiple of 8; past the stage's tokens the right-hand
 // sides and the columns of A are zero, so those s stay zero.
-template <int BASE, int TB>
-__device__ __forceinline__ void solve_block(const TcSmem& sm, float (&b)[TB]) {
+template <int TB>
+__device__ __forceinline__ void solve_block(const TcSmem& sm, float (&b)[TB], int BASE) {
   constexpr int NB = TB / 4;
   // dg[i] = -A[j0 .. j0 + 3][j0 + i] (i = 0..2): the diagonal block of block J (rows as a float4)
   // cp[i] = -A[j0 + 4 .. j0 + 7][j0 + i] (i = 0..3): block J's columns on the next block's rows
@@ -304,8 +304,8 @@ __device__ __forceinline__ void solve_block(const TcSmem& sm, float (&b)[TB]) {
 }
 
 // Right-hand sides of tokens [BASE, BASE + TB) of row r from shared memory.
-template <int BASE, int TB>
-__device__ __forceinline__ void load_rhs(TcSmem& sm, int r, float (&b)[TB]) {
+template <int TB>
+__device__ __forceinline__ void load_rhs(TcSmem& sm, int r, float (&b)[TB], int BASE) {
   const float* src = rhs_row(sm, r);
 #pragma unroll
   for (int i = 0; i < TB / 4; ++i) {
@@ -316,8 +316,8 @@ __device__ __forceinline__ void load_rhs(TcSmem& sm, int r, float (&b)[TB]) {
 
 // -S of tokens [BASE, BASE + 32) of row r into the Z B operand (row r, K = token), one
 // core-matrix row per 8 tokens, hi and lo; zeros past TB (the Z product contracts over all 64).
-template <int BASE, int TB>
-__device__ __forceinline__ void store_neg_s(TcSmem& sm, int r, const float (&b)[TB]) {
+template <int TB>
+__device__ __forceinline__ void store_neg_s(TcSmem& sm, int r, const float (&b)[TB], int BASE) {
 #pragma unroll
   for (int g8 = 0; g8 < 4; ++g8) {
     uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
@@ -333,8 +333,7 @@ __device__ __forceinline__ void store_neg_s(TcSmem& sm, int r, const float (&b)[
 }
 
 // Zeros for -S of tokens [BASE, BASE + 32) of row r (tokens past the stage).
-template <int BASE>
-__device__ __forceinline__ void store_neg_s_zero(TcSmem& sm, int r) {
+__device__ __forceinline__ void store_neg_s_zero(TcSmem& sm, int r, int BASE) {
 #pragma unroll
   for (int g8 = 0; g8 < 4; ++g8) {
     *reinterpret_cast<uint4*>(sm.zbh[BASE / 32] + umma_off(r, 8 * g8)) = make_uint4(0u, 0u, 0u, 0u);
@@ -342,25 +341,19 @@ __device__ __forceinline__ void store_neg_s_zero(TcSmem& sm, int r) {
   }
 }
 
-// Tokens [0, min(T, 32)) of row r: right-hand sides, solve, -S.
+// Tokens [BASE, BASE + 32) of row r (BASE = 0 or 32): right-hand sides (reduced by the coupling
+// c of the first 32 tokens when BASE = 32), solve, -S.  Both halves run the same instance, so
+// the code fetched for the first half serves the second.
 template <int TB>
-__device__ __forceinline__ void solve_first(TcSmem& sm, int r) {
+__device__ __forceinline__ void solve_half(TcSmem& sm, int r, int BASE, const float* c) {
   float b[TB];
-  load_rhs<0, TB>(sm, r, b);
-  solve_block<0, TB>(sm, b);
-  store_neg_s<0, TB>(sm, r, b);
-}
-
-// Tokens [32, T) of row r: right-hand sides reduced by the coupling c[t - 32] of the first 32
-// tokens (from TMEM), solve, -S.
-template <int TB>
-__device__ __forceinline__ void solve_second(TcSmem& sm, int r, const float (&c)[32]) {
-  float b[TB];
-  load_rhs<32, TB>(sm, r, b);
+  load_rhs<TB>(sm, r, b, BASE);
+  if (c != nullptr) {
 #pragma unroll
-  for (int i = 0; i < TB; ++i) b[i] -= c[i];
-  solve_block<32, TB>(sm, b);
-  store_neg_s<32, TB>(sm, r, b);
+    for (int i = 0; i < TB; ++i) b[i] -= c[i];
+  }
+  solve_block<TB>(sm, b, BASE);
+  store_neg_s<TB>(sm, r, b, BASE);
 }
 
 // Number of stages that hold tokens: only the last chunk can be short.
@@ -529,6 +522,12 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
   if (tid < kD) sm.scale[tid] = a.scales[r * a.C + ch0 + tid];
 
   const int nst = live_stages(N, L);
+  if (tid == 32 && a.act_bf16) {   // the tensor maps into the descriptor cache before first use
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.xr)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.qr)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.xc)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.qc)) : "memory");
+  }
   uint32_t xpar = 0;   // phase of mbar_x (token warps)
   if (is_k && nst > 0) {
     const StageInfo s0 = stage_info(0, N, L);
@@ -703,6 +702,14 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         }
       }
       fence_async_smem();
+    } else if (tid == 32 && ne + 1 < nst) {
+      // warp 1 is idle here: the next stage's x and q boxes, as soon as the Y product (issued
+      // by the readout warps for the previous stage) has finished reading the staging area
+      const StageInfo sn = stage_info(ne + 1, N, L);
+      if (a.act_bf16 && stage_is_box(sn, r, a.H)) {
+        if (pend) mbar_wait(&sm.mbar_y, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
+        tma_stage(sm, maps, sn, r, b, ch0, a.H, a.W);
+      }
     }
     tc_fence_before();
     __syncthreads();
@@ -810,9 +817,8 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         }
       }
       if (next_box) {
-        // the next stage's boxes into the staging area, which the Y product has finished reading
-        tok_bar();   // both token warps are past the Y wait
-        if (gt == 0) tma_stage(sm, maps, sn, r, b, ch0, a.H, a.W);
+        // the next stage's boxes (issued at the end of the gates) into the operand tiles, which
+        // the Gen and M1 products have finished reading
         mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
         xpar ^= 1u;
         unstage(sm, sn, r, gt);
@@ -825,40 +831,33 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       const int t = tid - 64;
       const bool live = t < T;
       const float lt = live ? sm.lam[t] : 0.f;
-      float g[kStage];
-      SRNL_LD16(g, tmem_lane + hb + kColM1);
-      SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + 16);
-      SRNL_LD16(g + 32, tmem_lane + hb + kColM1 + 32);
-      SRNL_LD16(g + 48, tmem_lane + hb + kColM1 + 48);
-      tmem_wait_ld();
       // as for -A: columns j < 32 of tokens t >= 32 (warp 3) factor at the split point 31 <= t;
-      // columns j >= 32 of tokens t < 32 (warp 2) are zero
+      // columns j >= 32 of tokens t < 32 (warp 2) are zero.  A rolled loop over 16-column
+      // blocks keeps the code small (instruction fetch is shared by every SM on the GPU).
       const float rf = (warp == 3 && live) ? exp2_fast(lt - sm.lam[31]) : 0.f;
-#pragma unroll
+#pragma unroll 1
       for (int jb = 0; jb < kStage; jb += 16) {
         float v[16];
-        if (warp == 3 && jb < 32) {
-#pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float4 c4 = *reinterpret_cast<const float4*>(&sm.cf32[jb + i]);
-            v[i] = rf * c4.x * g[jb + i]; v[i + 1] = rf * c4.y * g[jb + i + 1];
-            v[i + 2] = rf * c4.z * g[jb + i + 2]; v[i + 3] = rf * c4.w * g[jb + i + 3];
-          }
-        } else if (warp == 2 && jb >= 32) {
+        if (warp == 2 && jb >= 32) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = 0.f;
         } else {
-          float lv[16], ev[16];
+          float g[16];
+          SRNL_LD16(g, tmem_lane + hb + kColM1 + jb);
+          tmem_wait_ld();
+          const bool fac = warp == 3 && jb < 32;
 #pragma unroll
           for (int i = 0; i < 16; i += 4) {
             const float4 lj = *reinterpret_cast<const float4*>(&sm.lam[jb + i]);
             const float4 ej = *reinterpret_cast<const float4*>(&sm.eta[jb + i]);
-            lv[i] = lj.x; lv[i + 1] = lj.y; lv[i + 2] = lj.z; lv[i + 3] = lj.w;
-            ev[i] = ej.x; ev[i + 1] = ej.y; ev[i + 2] = ej.z; ev[i + 3] = ej.w;
-          }
+            const float4 c4 = *reinterpret_cast<const float4*>(&sm.cf32[(jb + i) & 31]);
+            const float lv[4] = {lj.x, lj.y, lj.z, lj.w}, ev[4] = {ej.x, ej.y, ej.z, ej.w};
+            const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            v[i] = (live && jb + i <= t) ? exp2_fast(lt - lv[i]) * ev[i] * g[jb + i] : 0.f;
+            for (int e = 0; e < 4; ++e)
+              v[i + e] = fac ? rf * cv[e] * g[i + e]
+                             : ((live && jb + i + e <= t) ? exp2_fast(lt - lv[e]) * ev[e] * g[i + e] : 0.f);
+          }
         }
         unsigned char* th = sm.zah[jb >> 5];
         unsigned char* tl = sm.zal[jb >> 5];
@@ -876,11 +875,15 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     // ---- forward substitution (warp 0): lane r owns row r of Q (solve_rows), then writes -S.
     if (warp == 0) {
       named_bar(5, 128);  // A and the right-hand sides (the token warps arrive without waiting)
-      switch ((min(T, 32) + 7) >> 3) {   // the smallest multiple of 8 tokens that covers them
-        case 1: solve_first<8>(sm, lane); break;
-        case 2: solve_first<16>(sm, lane); break;
-        case 3: solve_first<24>(sm, lane); break;
-        default: solve_first<32>(sm, lane); break;
+      if (T > 32) {
+        solve_half<32>(sm, lane, 0, nullptr);
+      } else {
+        switch ((T + 7) >> 3) {   // the smallest multiple of 8 tokens that covers the stage
+          case 1: solve_half<8>(sm, lane, 0, nullptr); break;
+          case 2: solve_half<16>(sm, lane, 0, nullptr); break;
+          case 3: solve_half<24>(sm, lane, 0, nullptr); break;
+          default: solve_half<32>(sm, lane, 0, nullptr); break;
+        }
       }
       if (T > 32) {
         // the coupling of tokens 32.. to the first 32: C[r][t'] = sum_{j < 32} S[r][j] A[32 + t'][j]
@@ -904,14 +907,9 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         SRNL_LD16(c, tmem + hb + kColZ);
         SRNL_LD16(c + 16, tmem + hb + kColZ + 16);
         tmem_wait_ld();
-        switch ((T - 32 + 7) >> 3) {
-          case 1: solve_second<8>(sm, lane, c); break;
-          case 2: solve_second<16>(sm, lane, c); break;
-          case 3: solve_second<24>(sm, lane, c); break;
-          default: solve_second<32>(sm, lane, c); break;
-        }
+        solve_half<32>(sm, lane, 32, c);
       } else {
-        store_neg_s_zero<32>(sm, lane);
+        store_neg_s_zero(sm, lane, 32);
       }
       fence_async_smem();
     } else if (warp == 1) {
