@@ -229,3 +229,70 @@ def make_cotangent(shape, seed: int = 0, act_dtype: str = F32) -> np.ndarray:
     elif act_dtype != F32:
         raise ValueError(f"unknown act_dtype {act_dtype!r}")
     return np.ascontiguousarray(g)
+
+
+# ------------------------------------------------ residual block around the operator
+@dataclasses.dataclass
+class BlockInputs:
+    """Seeded inputs of one VisionHOPE residual block: x [B, H, W, dim] (fp32 values, bf16-exact
+    when act_dtype is bf16) and the block's parameters (fp32): two LayerNorms, the projection
+    into and out of the mixer width m, the depthwise 3 x 3 convolution, the operator's
+    parameters at width m, and the FFN (hidden width 4 dim)."""
+    B: int
+    H: int
+    W: int
+    dim: int
+    m: int
+    head_dim: int
+    act_dtype: str
+    x32: np.ndarray
+    x_bits: Optional[np.ndarray]
+    p: Dict[str, np.ndarray]
+
+    @property
+    def heads(self) -> int:
+        return self.m // self.head_dim
+
+
+def make_block_inputs(B: int, H: int, W: int, dim: int, m: int, head_dim: int, act_dtype: str = BF16,
+                      seed: int = 0, *, mem_scale: float = 0.02, vec_scale: float = 0.1) -> BlockInputs:
+    """Draw, in this order: x ~ N(0, 1) [B, H, W, dim]; ln1_g = 1 + N(0, 0.1^2), ln1_b ~ N(0, 0.1^2);
+    W_in ~ N(0, 1/dim) [m, dim], b_in ~ N(0, 0.02^2); dw_w ~ N(0, 1/9) [m, 3, 3], dw_b ~ N(0, 0.02^2);
+    the operator at width m as make_inputs draws it (M_mem0, M_k0, M_v0 ~ N(0, mem_scale^2),
+    m_eta0, m_alpha0 ~ N(0, vec_scale^2), W_q ~ N(0, 1/m), scales 0.25); W_out ~ N(0, 1/m)
+    [dim, m], b_out ~ N(0, 0.02^2); ln2_g, ln2_b as ln1; W_1 ~ N(0, 1/dim) [4 dim, dim],
+    b_1 ~ N(0, 0.02^2); W_2 ~ N(0, 1/(4 dim)) [dim, 4 dim], b_2 ~ N(0, 0.02^2)."""
+    rng = np.random.default_rng(seed)
+    heads, d, hid = m // head_dim, head_dim, 4 * dim
+    f = lambda a: np.ascontiguousarray(a, dtype=np.float32)
+    x = rng.standard_normal((B, H, W, dim), dtype=np.float32)
+    p = {}
+    p["ln1_g"] = f(1.0 + 0.1 * rng.standard_normal(dim))
+    p["ln1_b"] = f(0.1 * rng.standard_normal(dim))
+    p["W_in"] = f(rng.standard_normal((m, dim)) / np.sqrt(dim))
+    p["b_in"] = f(0.02 * rng.standard_normal(m))
+    p["dw_w"] = f(rng.standard_normal((m, 3, 3)) / 3.0)
+    p["dw_b"] = f(0.02 * rng.standard_normal(m))
+    p["M_mem0"] = f(rng.standard_normal((4, heads, d, d)) * mem_scale)
+    p["M_k0"] = f(rng.standard_normal((4, heads, d, d)) * mem_scale)
+    p["M_v0"] = f(rng.standard_normal((4, heads, d, d)) * mem_scale)
+    p["m_eta0"] = f(rng.standard_normal((4, heads, d)) * vec_scale)
+    p["m_alpha0"] = f(rng.standard_normal((4, heads, d)) * vec_scale)
+    p["W_q"] = f(rng.standard_normal((m, m)) / np.sqrt(m))
+    p["scales"] = np.full((4, m), 0.25, dtype=np.float32)
+    p["W_out"] = f(rng.standard_normal((dim, m)) / np.sqrt(m))
+    p["b_out"] = f(0.02 * rng.standard_normal(dim))
+    p["ln2_g"] = f(1.0 + 0.1 * rng.standard_normal(dim))
+    p["ln2_b"] = f(0.1 * rng.standard_normal(dim))
+    p["W_1"] = f(rng.standard_normal((hid, dim)) / np.sqrt(dim))
+    p["b_1"] = f(0.02 * rng.standard_normal(hid))
+    p["W_2"] = f(rng.standard_normal((dim, hid)) / np.sqrt(hid))
+    p["b_2"] = f(0.02 * rng.standard_normal(dim))
+    x_bits = None
+    if act_dtype == BF16:
+        x_bits = bf16_round_bits(x)
+        x = bf16_bits_to_f32(x_bits).reshape(x.shape)
+    elif act_dtype != F32:
+        raise ValueError(f"unknown act_dtype {act_dtype!r}")
+    return BlockInputs(B=B, H=H, W=W, dim=dim, m=m, head_dim=head_dim, act_dtype=act_dtype,
+                       x32=np.ascontiguousarray(x), x_bits=x_bits, p=p)
