@@ -603,6 +603,52 @@ def run_seq(args):
                       "clocks": clocks.summary()}), flush=True)
 
 
+def run_block(args):
+    """Time the residual block around the operator on the S1 map (B = 32, 56 x 56, dim 64,
+    mixer_dim 64, head_dim 32, bf16): LayerNorm, four tensor-core projections, depthwise
+    convolution, the operator and the FFN per forward."""
+    import torch
+    import self_referential_nested_b200 as S
+    from self_referential_nested_b200 import build as Bld
+    from srnl_inputs import make_block_inputs
+
+    Bld.build()
+    B, H, W, dim, m, hd = args.batch or 32, 56, 56, 64, 64, 32
+    inp = make_block_inputs(B, H, W, dim, m, hd, "bf16", seed=0)
+    h = S.srnl_block_create(dict(B=B, H=H, W=W, dim=dim, mixer_dim=m, head_dim=hd, alpha=0.95, gen_dtype="bf16"),
+                            inp.p)
+    x = torch.from_numpy(inp.x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        S.srnl_block_forward(h, x, y, stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    ts = []
+    for i in range(args.steps):
+        flush.fill_((i + 1) & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        S.srnl_block_forward(h, x, y, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    clocks.stop()
+    S.srnl_block_device_status(h)
+    h.close()
+    ms = float(np.mean(ts))
+    print(json.dumps({"metric": "VisionHOPE block tokens/s (fwd, 1xB200)", "value": B * H * W / (ms * 1e-3),
+                      "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": f"block_b{B}_56x56_dim{dim}_mixer{m}", "B": B, "H": H, "W": W,
+                                 "dim": dim, "mixer_dim": m, "head_dim": hd, "l2": "flushed before each step"},
+                      "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -618,6 +664,7 @@ def main():
     ap.add_argument("--head-dim", type=int, default=0, choices=[0, 4, 8, 16, 32, 64],
                     help="override the head dim (C = heads x d); 64 defaults to the fp32-generation path")
     ap.add_argument("--seq", action="store_true", help="time the standalone sequence layer instead")
+    ap.add_argument("--block", action="store_true", help="time the residual block around the operator instead")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (gradients of x and every parameter) instead")
     ap.add_argument("--sustain", action="store_true",
@@ -628,6 +675,9 @@ def main():
     args = ap.parse_args()
     if args.seq:
         run_seq(args)
+        return
+    if args.block:
+        run_block(args)
         return
     cfg = CONFIGS[args.config]
     if args.batch > 0:

@@ -268,6 +268,64 @@ typedef struct {
 SRNL_API srnl_status srnl_scan_backward(srnl_scan* h, const void* x, const void* dy, void* dx,
                                        const srnl_scan_grads* grads, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The VisionHOPE residual block around the operator ("VisionHOPE: Visual Backbones as
+ * Self-Modifying Learning Systems", 2D-maps paragraph: a standard two-branch residual,
+ * depthwise conv for local context, SRNL for long range, then an FFN; "VisionHOPE Model
+ * Overview", "Four-Directional Scanning and Spatial Chunking": projections, normalization,
+ * depthwise convolution and a feed-forward network; "VisionHOPE" README, "SRNL and VisionHOPE
+ * operator": shape-preserving, mixer_dim sets the internal width).  The pages do not print
+ * the wiring; this library reads it as (channels-last, m = mixer_dim)
+ *   u   = LN1(x) W_in^T + b_in
+ *   mix = DWConv3x3(u) + operator(u)          (3 x 3 per channel, zero padding, bias)
+ *   y   = x + mix W_out^T + b_out
+ *   out = y + GELU(LN2(y) W_1^T + b_1) W_2^T + b_2      (hidden width 4 dim, GELU v Phi(v))
+ * with LayerNorm over channels (scale and shift, epsilon ln_eps).  bf16 activations; the
+ * projections run as bf16 tensor-core products with fp32 accumulation and bf16 outputs, the
+ * normalisations and the convolution in fp32 arithmetic.
+ * ---------------------------------------------------------------------- */
+typedef struct srnl_block srnl_block; /* opaque; owned by the library */
+
+typedef struct {
+  int B, H, W;        /* batch, height, width                                     */
+  int dim;            /* channels of x and y: a multiple of 32, at most 512      */
+  int mixer_dim;      /* width of the mixer and the operator: a multiple of 32, at most 512 */
+  int head_dim;       /* the operator's head dim (4, 8, 16, 32 or 64)             */
+  float alpha, eps;   /* the operator's retention cap and key epsilon              */
+  int chunk_row, chunk_col; /* the operator's chunks (0: full rows / columns)    */
+  int act_dtype;      /* SRNL_BF16                                                */
+  int gen_dtype;      /* the operator's generation dtype                          */
+  int injection_cap;  /* srnl_cap of the operator                                 */
+  float ln_eps;       /* LayerNorm epsilon, > 0 (1e-6)                            */
+} srnl_block_config;
+
+/* HOST pointers to dense fp32 arrays, copied (weights rounded to bf16) at create. */
+typedef struct {
+  const float *ln1_g, *ln1_b;   /* [dim]                      */
+  const float *W_in, *b_in;     /* [m][dim], [m]              */
+  const float *dw_w, *dw_b;     /* [m][3][3], [m]             */
+  srnl_scan_params op;          /* the operator at width m (C = m, heads = m / head_dim) */
+  const float *W_out, *b_out;   /* [dim][m], [dim]            */
+  const float *ln2_g, *ln2_b;   /* [dim]                      */
+  const float *W_1, *b_1;       /* [4 dim][dim], [4 dim]      */
+  const float *W_2, *b_2;       /* [dim][4 dim], [dim]        */
+} srnl_block_params;
+
+/* Validate, pack the parameters and allocate the block's workspace (six bf16 buffers of
+ * B*H*W rows: dim, m, m, m, dim and 4 dim wide) and its operator handle on the CURRENT
+ * device.  cudaMalloc; synchronous.  *out is NULL on failure. */
+SRNL_API srnl_status srnl_block_create(srnl_block** out, const srnl_block_config* cfg,
+                                       const srnl_block_params* params);
+/* out = block(x): DEVICE pointers, bf16 [B][H][W][dim], 16-byte aligned, not overlapping.
+ * Asynchronous on `stream` (eight kernels plus the operator's); calls on one handle must not
+ * overlap on the device. */
+SRNL_API srnl_status srnl_block_forward(srnl_block* h, const void* x, void* y, void* stream);
+/* Synchronously reads the status words of the block's and its operator's kernels: SRNL_OK,
+ * or SRNL_E_TIMEOUT once a bounded in-kernel wait gave up. */
+SRNL_API srnl_status srnl_block_device_status(srnl_block* h);
+SRNL_API const char* srnl_block_last_error(const srnl_block* h);
+SRNL_API void srnl_block_destroy(srnl_block* h);
+
 /* Self-test of the failure path of the bounded in-kernel waits: on the CURRENT device, runs
  * the scan kernels' bounded mbarrier wait on a barrier that nothing completes, with a
  * wall-time limit of wait_ms milliseconds (1..5000).  Returns SRNL_E_TIMEOUT when the wait

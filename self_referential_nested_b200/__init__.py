@@ -36,13 +36,28 @@ EXPORTED = ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host",
             "srnl_seq_destroy", "srnl_scan_cap_count", "srnl_seq_cap_count",
             "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
             "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout",
-            "srnl_scan_noalloc_status", "srnl_selftest_noalloc_wait_timeout")
+            "srnl_scan_noalloc_status", "srnl_selftest_noalloc_wait_timeout",
+            "srnl_block_create", "srnl_block_forward", "srnl_block_device_status", "srnl_block_last_error",
+            "srnl_block_destroy")
 
 
 class SrnlError(RuntimeError):
     def __init__(self, status: int, where: str, message: str):
         self.status = status
         super().__init__(f"{where}: {message} [status {status}]")
+
+
+BLOCK_KEYS = ("ln1_g", "ln1_b", "W_in", "b_in", "dw_w", "dw_b", "W_out", "b_out", "ln2_g", "ln2_b",
+              "W_1", "b_1", "W_2", "b_2")
+OP_KEYS = ("W_q", "scales", "M_mem0", "M_k0", "M_v0", "m_eta0", "m_alpha0")
+
+
+class _BlockConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int), ("dim", ctypes.c_int),
+                ("mixer_dim", ctypes.c_int), ("head_dim", ctypes.c_int), ("alpha", ctypes.c_float),
+                ("eps", ctypes.c_float), ("chunk_row", ctypes.c_int), ("chunk_col", ctypes.c_int),
+                ("act_dtype", ctypes.c_int), ("gen_dtype", ctypes.c_int), ("injection_cap", ctypes.c_int),
+                ("ln_eps", ctypes.c_float)]
 
 
 class _Config(ctypes.Structure):
@@ -55,6 +70,12 @@ class _Config(ctypes.Structure):
 class _Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("W_q", "scales", "M_mem0", "M_k0", "M_v0",
                                                 "m_eta0", "m_alpha0")]
+
+
+class _BlockParams(ctypes.Structure):
+    _fields_ = ([(n, ctypes.c_void_p) for n in ("ln1_g", "ln1_b", "W_in", "b_in", "dw_w", "dw_b")]
+                + [("op", _Params)]
+                + [(n, ctypes.c_void_p) for n in ("W_out", "b_out", "ln2_g", "ln2_b", "W_1", "b_1", "W_2", "b_2")])
 
 
 class _Grads(ctypes.Structure):
@@ -127,6 +148,13 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.srnl_seq_backward.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_SeqGrads), vp]
     lib.srnl_selftest_wait_timeout.argtypes = [i]
     lib.srnl_scan_noalloc_status.argtypes = [vp]
+    lib.srnl_block_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(_BlockConfig), ctypes.POINTER(_BlockParams)]
+    lib.srnl_block_forward.argtypes = [vp, vp, vp, vp]
+    lib.srnl_block_device_status.argtypes = [vp]
+    lib.srnl_block_last_error.argtypes = [vp]
+    lib.srnl_block_last_error.restype = ctypes.c_char_p
+    lib.srnl_block_destroy.argtypes = [vp]
+    lib.srnl_block_destroy.restype = None
     lib.srnl_selftest_noalloc_wait_timeout.argtypes = [i, vp]
     for name in ("srnl_scan_create", "srnl_scan_forward", "srnl_scan_forward_host", "srnl_scan_forward_noalloc",
                  "srnl_scan_route_index", "srnl_scan_gather", "srnl_scan_enable_stage_timing",
@@ -134,7 +162,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                  "srnl_seq_device_status", "srnl_scan_cap_count", "srnl_seq_cap_count",
                  "srnl_scan_forward_host_async", "srnl_scan_host_join", "srnl_scan_host_sync",
                  "srnl_scan_backward", "srnl_seq_backward", "srnl_selftest_wait_timeout",
-            "srnl_scan_noalloc_status", "srnl_selftest_noalloc_wait_timeout"):
+                 "srnl_scan_noalloc_status", "srnl_selftest_noalloc_wait_timeout", "srnl_block_create",
+                 "srnl_block_forward", "srnl_block_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -431,4 +460,72 @@ def srnl_seq_cap_count(h: SrnlSeq) -> int:
 
 
 def srnl_seq_destroy(h: SrnlSeq) -> None:
+    h.close()
+
+
+# ------------------------------------------------ residual block around the operator
+class SrnlBlock:
+    """Owns one ``srnl_block*`` handle (the VisionHOPE residual block, bf16 [B, H, W, dim])."""
+
+    def __init__(self, handle: int, cfg: Dict):
+        self._h = handle
+        self.cfg = dict(cfg)
+
+    @property
+    def handle(self) -> int:
+        if not self._h:
+            raise RuntimeError("srnl_block handle is closed")
+        return self._h
+
+    def _check(self, status: int, where: str):
+        if status != SRNL_OK:
+            raise SrnlError(status, where, load_library().srnl_block_last_error(self._h).decode())
+
+    def close(self):
+        if self._h:
+            load_library().srnl_block_destroy(self._h)
+            self._h = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def srnl_block_create(cfg: Dict, params: Dict[str, np.ndarray]) -> SrnlBlock:
+    """cfg keys: B, H, W, dim, mixer_dim, head_dim, alpha, eps, chunk_row, chunk_col, gen_dtype,
+    injection_cap, ln_eps (act_dtype is bf16).  params: float32 host arrays BLOCK_KEYS and the
+    operator's OP_KEYS at width mixer_dim."""
+    lib = load_library()
+
+    def dt(v):
+        return {"f32": SRNL_F32, "bf16": SRNL_BF16}.get(v, v)
+
+    c = _BlockConfig(B=cfg["B"], H=cfg["H"], W=cfg["W"], dim=cfg["dim"], mixer_dim=cfg["mixer_dim"],
+                     head_dim=cfg["head_dim"], alpha=cfg["alpha"], eps=cfg.get("eps", 1e-6),
+                     chunk_row=cfg.get("chunk_row", 0), chunk_col=cfg.get("chunk_col", 0),
+                     act_dtype=dt(cfg.get("act_dtype", "bf16")), gen_dtype=dt(cfg.get("gen_dtype", "bf16")),
+                     injection_cap=_cap(cfg.get("injection_cap", "soft")), ln_eps=cfg.get("ln_eps", 1e-6))
+    keep = {k: np.ascontiguousarray(params[k], dtype=np.float32) for k in BLOCK_KEYS + OP_KEYS}
+    op = _Params(**{k: keep[k].ctypes.data for k in OP_KEYS})
+    p = _BlockParams(op=op, **{k: keep[k].ctypes.data for k in BLOCK_KEYS})
+    h = ctypes.c_void_p()
+    st = lib.srnl_block_create(ctypes.byref(h), ctypes.byref(c), ctypes.byref(p))
+    if st != SRNL_OK:
+        raise SrnlError(st, "srnl_block_create", lib.srnl_block_last_error(None).decode())
+    return SrnlBlock(h.value, cfg)
+
+
+def srnl_block_forward(h: SrnlBlock, x, y, stream=None) -> None:
+    """y <- block(x): bf16 CUDA tensors [B, H, W, dim], 16-byte aligned, not overlapping."""
+    h._check(load_library().srnl_block_forward(h.handle, _ptr(x), _ptr(y), _stream(stream)), "srnl_block_forward")
+
+
+def srnl_block_device_status(h: SrnlBlock) -> None:
+    """Raise SrnlError if a bounded in-kernel wait of the block or its operator gave up."""
+    h._check(load_library().srnl_block_device_status(h.handle), "srnl_block_device_status")
+
+
+def srnl_block_destroy(h: SrnlBlock) -> None:
     h.close()

@@ -114,6 +114,7 @@ cudaError_t launch_scan_d64(const ScanGeom& g, const ScanParamsDev& p, const voi
                             float* finals, unsigned long long* binds, cudaStream_t s);
 cudaError_t prepare_scan_d64_kernel();
 
+cudaError_t prepare_block_kernels();  // the residual block's GEMM (dynamic smem)
 cudaError_t prepare_kernels();       // one-time function attributes (dynamic smem)
 cudaError_t prepare_scan_kernels();
 cudaError_t prepare_scan_chunkwise_kernel();
