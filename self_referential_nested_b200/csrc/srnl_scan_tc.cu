@@ -52,6 +52,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -141,8 +142,8 @@ struct TcArgs {
 // W*C).  Boxes are 32 channels (one head) by 64 tokens.
 struct TcMaps {
   CUtensorMap xr, xc, qr, qc;
+  uint32_t box_bytes_r, box_bytes_c;   // bytes of one x box (= one q box) per orientation
 };
-constexpr uint32_t kBoxBytes = kStage * kD * 2;   // one 64-token x 32-channel bf16 box
 
 // -A[t][j] for j in [16p, 16p + 16) lives in the first 4 KB of a1h, a1l, b1h, b1l
 // (p = 0..3): the u and k rows of M1, dead between M1 and the next stage's gates.
@@ -402,15 +403,16 @@ __device__ __forceinline__ void tc_prefetch(TcSmem& sm, const StageInfo& si, con
 }
 
 // One thread: the stage's x and q boxes into the staging area (the Y operand tiles, dead
-// between the Y product's completion and the next z), completing on mbar_x.  Row routes load
-// the 64 tokens from the stage's lowest raster index p_lo on; column routes the 64 rows of
-// column j from i_lo on.  Boxes may run past the image or the tensor (the rest is unused; TMA
+// between the Y product's completion and the next z), completing on mbar_x.  A box holds the
+// orientation's chunk length rounded up to 8 tokens, at most 64.  Row routes load from the
+// stage's lowest raster index p_lo on; column routes the rows of column j from i_lo on.  Boxes may run past the image or the tensor (the rest is unused; TMA
 // fills what lies outside the tensor with zeros).  Coordinates: channels ch0 (a multiple of
 // 32, so 64-byte aligned), then tokens; never negative.
 __device__ __forceinline__ void tma_stage(TcSmem& sm, const TcMaps& m, const StageInfo& si, int r, int b, int ch0,
                                           int H, int W) {
   const uint32_t bar = smem_u32(&sm.mbar_x);
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kBoxBytes) : "memory");
+  const uint32_t box = r < 2 ? m.box_bytes_r : m.box_bytes_c;
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * box) : "memory");
   const int t_lo = (r & 1) ? si.t0 + si.T - 1 : si.t0;      // route token at the lowest address
   const int p = route_pos(r, t_lo, H, W);
   if (r < 2) {
@@ -447,11 +449,12 @@ __device__ __forceinline__ bool stage_is_box(const StageInfo& si, int r, int H) 
 
 // Token warps (ht = 0..63): the staged boxes (64-byte rows, ascending raster order) into the
 // operand tiles in route order: x into rows t and 64 + t of the x tile, q into rows 64 + t of
-// the M1 A tile.  Reverse routes read the box backwards over the stage's T tokens.
+// the M1 A tile, for the stage's T tokens (the rows past them keep earlier tokens, which every
+// consumer masks).  Reverse routes read the box backwards.
 __device__ __forceinline__ void unstage(TcSmem& sm, const StageInfo& si, int r, int ht) {
-  for (int idx = ht; idx < kStage * 4; idx += 64) {
+  for (int idx = ht; idx < si.T * 4; idx += 64) {
     const int t = idx >> 2, part = idx & 3;
-    const int row = ((r & 1) && t < si.T) ? si.T - 1 - t : t;
+    const int row = (r & 1) ? si.T - 1 - t : t;
     const uint4 xv = *reinterpret_cast<const uint4*>(sm.yah + row * 64 + part * 16);
     const uint4 qv = *reinterpret_cast<const uint4*>(sm.yal + row * 64 + part * 16);
     *reinterpret_cast<uint4*>(sm.xa + umma_off(t, part * 8)) = xv;
@@ -1051,21 +1054,23 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return g_encode;
 }
 
-// Row view: [B*H*W][C]; column view: [B*H][W][C].  bf16, box 32 channels x 64 tokens.
-bool encode_maps(const void* base, int B, int H, int W, int C, CUtensorMap* row, CUtensorMap* col) {
+// Row view: [B*H*W][C]; column view: [B*H][W][C].  bf16, boxes of 32 channels x box_r (row
+// view) or box_c (column view) tokens.
+bool encode_maps(const void* base, int B, int H, int W, int C, int box_r, int box_c, CUtensorMap* row,
+                 CUtensorMap* col) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint32_t estr[3] = {1, 1, 1};
   const cuuint64_t rdim[2] = {(cuuint64_t)C, (cuuint64_t)B * H * W};
   const cuuint64_t rstr[1] = {(cuuint64_t)C * 2};
-  const cuuint32_t rbox[2] = {(cuuint32_t)kD, (cuuint32_t)kStage};
+  const cuuint32_t rbox[2] = {(cuuint32_t)kD, (cuuint32_t)box_r};
   CUresult e = enc(row, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), rdim, rstr, rbox, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (e != CUDA_SUCCESS) return false;
   const cuuint64_t cdim[3] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)B * H};
   const cuuint64_t cstr[2] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2};
-  const cuuint32_t cbox[3] = {(cuuint32_t)kD, 1, (cuuint32_t)kStage};
+  const cuuint32_t cbox[3] = {(cuuint32_t)kD, 1, (cuuint32_t)box_c};
   e = enc(col, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), cdim, cstr, cbox, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1088,8 +1093,12 @@ cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, con
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
   if (g.act_bf16) {
-    if (!encode_maps(x, g.B, g.H, g.W, g.C, &maps.xr, &maps.xc) ||
-        !encode_maps(q, g.B, g.H, g.W, g.C, &maps.qr, &maps.qc))
+    // a stage holds at most min(L, 64) tokens: the box covers that, rounded up to 8
+    const int box_r = std::min(kStage, (g.Lrow + 7) / 8 * 8), box_c = std::min(kStage, (g.Lcol + 7) / 8 * 8);
+    maps.box_bytes_r = (uint32_t)box_r * kD * 2;
+    maps.box_bytes_c = (uint32_t)box_c * kD * 2;
+    if (!encode_maps(x, g.B, g.H, g.W, g.C, box_r, box_c, &maps.xr, &maps.xc) ||
+        !encode_maps(q, g.B, g.H, g.W, g.C, box_r, box_c, &maps.qr, &maps.qc))
       return cudaErrorInvalidValue;
   }
   srnl_scan_chunkwise_kernel<<<nseq, kThreadsTc, sizeof(TcSmem), s>>>(a, maps);
