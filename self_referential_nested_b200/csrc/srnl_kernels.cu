@@ -135,23 +135,30 @@ __global__ void convert_kernel(const void* __restrict__ src, bool src_bf16, void
 }
 
 __global__ void fuse_kernel(const float* __restrict__ yr, void* __restrict__ y, int64_t total,
-                            int routes, bool act_bf16) {
+                            int routes, bool act_bf16, bool part_bf16) {
   const int64_t i8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (i8 >= total) return;
   float acc[8];
-  {
-    const float4 a = *reinterpret_cast<const float4*>(yr + i8);
-    const float4 b = *reinterpret_cast<const float4*>(yr + i8 + 4);
-    acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
-    acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
-  }
 #pragma unroll
-  for (int r = 1; r < 4; ++r) {
+  for (int r = 0; r < 4; ++r) {   // fixed order r0 + r1 + r2 + r3
     if (r >= routes) break;
-    const float4 a = *reinterpret_cast<const float4*>(yr + r * total + i8);
-    const float4 b = *reinterpret_cast<const float4*>(yr + r * total + i8 + 4);
-    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    float v[8];
+    if (part_bf16) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(yr) + r * total + i8);
+      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+        v[2 * e] = f.x;
+        v[2 * e + 1] = f.y;
+      }
+    } else {
+      const float4 a = *reinterpret_cast<const float4*>(yr + r * total + i8);
+      const float4 b = *reinterpret_cast<const float4*>(yr + r * total + i8 + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = r == 0 ? v[e] : acc[e] + v[e];
   }
   if (act_bf16) {
     uint4 raw;
@@ -213,7 +220,8 @@ cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_
   const int64_t total = (int64_t)g.B * g.H * g.W * g.C;
   const int64_t threads = total / 8;
   const int bs = 256;
-  fuse_kernel<<<(unsigned)((threads + bs - 1) / bs), bs, 0, s>>>(yr, y, total, g.routes, g.act_bf16);
+  fuse_kernel<<<(unsigned)((threads + bs - 1) / bs), bs, 0, s>>>(yr, y, total, g.routes, g.act_bf16,
+                                                                partials_bf16(g));
   return cudaGetLastError();
 }
 

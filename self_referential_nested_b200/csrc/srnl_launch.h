@@ -37,14 +37,20 @@ bool query_projection_tc_supported(const ScanGeom& g);
 cudaError_t launch_query_projection_tc(const ScanGeom& g, const ScanParamsDev& p, const void* x, void* q,
                                        int* err, cudaStream_t s);
 
-// Route partials yr[4][B*N][C] (fp32, already scaled by the fusion scales),
+// Route partials yr[4][B*N][C] (already scaled by the fusion scales; fp32, or bf16 when
+// partials_bf16(g)),
 // optional final states.
 // `err` (device int) receives SRNL_E_TIMEOUT if a bounded in-kernel wait gives up.
 // `binds` (device counter or nullptr) accumulates the tokens on which the hard clamp acts.
 cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
                         float* yr, float* finals, int* err, unsigned long long* binds, cudaStream_t s);
 
-// y = yr[0] + ... + yr[routes - 1] in act dtype, summed in route order.
+// Whether launch_scan writes the route partials in bf16: the chunkwise kernel (bf16 generation,
+// 32-wide heads) with bf16 activations writes them in the output's precision; every other
+// path writes fp32.  The buffer is sized for fp32 either way.
+inline bool partials_bf16(const ScanGeom& g) { return g.gen_bf16 && g.act_bf16 && g.hd == 32; }
+
+// y = yr[0] + ... + yr[routes - 1] in act dtype, summed in fp32 in route order.
 cudaError_t launch_fuse(const ScanGeom& g, const float* yr, void* y, cudaStream_t s);
 
 cudaError_t launch_route_index(int route, int H, int W, int32_t* out, cudaStream_t s);

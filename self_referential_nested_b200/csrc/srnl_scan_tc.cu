@@ -357,6 +357,31 @@ __device__ __forceinline__ void solve_half(TcSmem& sm, int r, int BASE, const fl
   store_neg_s<TB>(sm, r, b, BASE);
 }
 
+// One token's scaled route partial (32 channels of one head) at element offset `off` of the
+// partial buffer: bf16 when the activations are bf16 (the fusion's output precision), else fp32.
+__device__ __forceinline__ void store_partial(float* yr, int64_t off, const float* scale, const float (&y)[kD],
+                                              bool bf16) {
+  if (bf16) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(yr) + off);
+#pragma unroll
+    for (int i = 0; i < kD; i += 8) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(scale[i + 2 * e] * y[i + 2 * e], scale[i + 2 * e + 1] * y[i + 2 * e + 1]);
+        w4[e] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+      dst[i / 8] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  } else {
+    float* dst = yr + off;
+#pragma unroll
+    for (int i = 0; i < kD; i += 4)
+      *reinterpret_cast<float4*>(dst + i) =
+          make_float4(scale[i] * y[i], scale[i + 1] * y[i + 1], scale[i + 2] * y[i + 2], scale[i + 3] * y[i + 3]);
+  }
+}
+
 // Number of stages that hold tokens: only the last chunk can be short.
 __device__ __forceinline__ int live_stages(int N, int L) {
   const int per = (L + kStage - 1) / kStage;
@@ -811,12 +836,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         tmem_wait_ld();
         if (gt < pst.T) {
           const int p = route_pos(r, pst.t0 + gt, a.H, a.W);
-          float* dst = a.yr + ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0;
-#pragma unroll
-          for (int i = 0; i < kD; i += 4)
-            *reinterpret_cast<float4*>(dst + i) =
-                make_float4(sm.scale[i] * y[i], sm.scale[i + 1] * y[i + 1], sm.scale[i + 2] * y[i + 2],
-                            sm.scale[i + 3] * y[i + 3]);
+          store_partial(a.yr, ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0, sm.scale, y, a.act_bf16);
         }
       }
       if (next_box) {
@@ -1001,11 +1021,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     tmem_wait_ld();
     if (gt < pst.T) {
       const int p = route_pos(r, pst.t0 + gt, a.H, a.W);
-      float* dst = a.yr + ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0;
-#pragma unroll
-      for (int i = 0; i < kD; i += 4)
-        *reinterpret_cast<float4*>(dst + i) = make_float4(sm.scale[i] * y[i], sm.scale[i + 1] * y[i + 1],
-                                                          sm.scale[i + 2] * y[i + 2], sm.scale[i + 3] * y[i + 3]);
+      store_partial(a.yr, ((int64_t)r * a.B * N + tok0 + p) * a.C + ch0, sm.scale, y, a.act_bf16);
     }
   }
 
