@@ -759,13 +759,15 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       // g(j, t - 1) = 2^(Lambda_{t-1} - Lambda_31) 2^(Lambda_31 - Lambda_j) with both factors <= 1:
       // one exp2 per thread and the precomputed column factors.  The diagonal 32 x 32 blocks take
       // one exp2 per element.  Columns j >= 32 of tokens t < 32 are above the diagonal; the solve
-      // never reads them, so nobody writes them.
+      // never reads them, so nobody writes them.  A short stage (T <= 32) is solved over tokens
+      // below 8 ceil(T / 8) only: warp 1 has nothing to write, and warp 0 skips columns 16..31
+      // when T <= 16 (the rows of dead tokens the solve does read are written as zeros).
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
       const int t = tid;
       const bool live = t < T;
       const float lp = (t > 0 && live) ? sm.lam[t - 1] : 0.f;  // Lambda_{t-1}
       float g[32];
-      if (warp == 1) {
+      if (warp == 1 && T > 32) {
         SRNL_LD16(g, tmem_lane + hb + kColM1);
         SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + 16);
         tmem_wait_ld();
@@ -789,11 +791,15 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         fence_async_smem();
       }
       const int j0 = 32 * warp;   // the diagonal block: columns [32 w, 32 w + 32)
-      SRNL_LD16(g, tmem_lane + hb + kColM1 + j0);
-      SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + j0 + 16);
-      tmem_wait_ld();
+      const int jb_end = (warp == 1) ? (T > 32 ? 32 : 0) : (T > 16 ? 32 : 16);
+      if (jb_end > 0) {
+        SRNL_LD16(g, tmem_lane + hb + kColM1 + j0);
+        SRNL_LD16(g + 16, tmem_lane + hb + kColM1 + j0 + 16);
+        tmem_wait_ld();
+      }
 #pragma unroll
       for (int jb = 0; jb < 32; jb += 16) {
+        if (jb >= jb_end) break;
         // the block's Lambda_j and eta_j first: the stores below may alias them
         float lv[16], ev[16], v[16];
 #pragma unroll
@@ -809,8 +815,9 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
 #pragma unroll
         for (int i = 0; i < 16; ++i) neg_a_row(sm, j0 + jb + i)[t] = v[i];
       }
-    } else if (is_k) {
-      // the right-hand sides b^T[r][t] = 2^Lambda_{t-1} (Q_s u_t)[r] (token warps)
+    } else if (is_k && (warp == 4 || T > 32)) {
+      // the right-hand sides b^T[r][t] = 2^Lambda_{t-1} (Q_s u_t)[r] (token warps; the solve of a
+      // stage of at most 32 tokens reads none of warp 5's)
       mbar_wait(&sm.mbar_1, par, &sm.wait_failed);
       const int t = tid - 128;
       const bool live = t < T;
@@ -861,7 +868,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
 #pragma unroll 1
       for (int jb = 0; jb < kStage; jb += 16) {
         float v[16];
-        if (warp == 2 && jb >= 32) {
+        if ((warp == 2 && jb >= 32) || jb >= T || (warp == 3 && T <= 32)) {   // all zero
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = 0.f;
         } else {
