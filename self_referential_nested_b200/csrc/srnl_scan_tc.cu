@@ -28,19 +28,24 @@
 //
 // One CTA owns one (route, batch, head) sequence; 192 threads.  Warp w runs on SMSP w % 4
 // and reads TMEM lanes 32 (w % 4) .. + 31, which fixes who can drain which accumulator rows:
-//   warps 0-1  solve warps: half of -A from TMEM lanes 0..63, the forward substitution
-//              (four rows x eight tokens per thread); warp 0 also forms the stage-end Q
+//   warps 0-1  solve warps: -A from TMEM lanes 0..63 (warp 0 its diagonal 32 x 32 block; warp 1
+//              its diagonal block and, factored at the split point 31, the columns below 32,
+//              also written as the coupling operand A_21); warp 0 then solves the stage's
+//              triangular system with one row of Q per lane (tokens 0..31, the tensor-core
+//              coupling, tokens 32..) and forms the stage-end Q; warp 1 issues the next
+//              stage's TMA boxes during the gates
 //   warps 2-3  readout warps: half of the gate vector work (tokens repeated in TMEM lanes
-//              64..127), the readout coefficients from lanes 64..127 during the
-//              substitution, z_t and the Y product of the previous stage
+//              64..127), the readout coefficients from lanes 64..127 during -A and the solve,
+//              z_t and the Y product of the previous stage
 //   warps 4-5  token warps: boundary products and generation, the gate scalars, the
-//              retention prefix, the other half of the gate vector work, of -A and the
-//              right-hand sides, the copies of the next stage and y_t from TMEM
+//              retention prefix, the other half of the gate vector work, the right-hand sides,
+//              y_t of the previous stage, and the next stage's x and q out of the TMA staging
 // Tensor-core products per stage (tcgen05, M = 128, fp32 accumulate in TMEM; an fp32
 // operand is split into bf16 hi + lo and a product of two such takes three MMAs):
 //   W    [x] Q_b^T                      N = 32   w_t = Q_b x_t
 //   Gen  [w] G^T                        N = 80   [k~ v a beta]_t
 //   M1   [u; q] [k; Q_s]^T              N = 96   u.k, Q_s u, q.k, Q_s q
+//   C    (-S_1) (-A_21)^T               N = 32   the first 32 tokens' share of the others' solve
 //   Z    [Kd^T; -; Mz^T] (-S)^T         N = 32   stage-end correction and z_t - 2^Lambda_t Q_s q_t
 //   Y    [z] M_mem0^T                   N = 32   y_t
 // TMEM holds two 128-column halves; consecutive stages alternate, so the readout of
