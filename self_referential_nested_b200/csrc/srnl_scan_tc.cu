@@ -956,18 +956,17 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       named_bar(3, 128);
       if (tid == 0) {
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-#pragma unroll
-          for (int k16 = 0; k16 < 2; ++k16) {   // A steps 2 padded core matrices, B 2 plain ones
-            const uint32_t ao = k16 * 2 * kZCore, bo = k16 * 256;
-            const uint64_t ah = umma_desc_strided(smem_u32(sm.zah[kk]) + ao, kZCore, kZGroup);
-            const uint64_t al = umma_desc_strided(smem_u32(sm.zal[kk]) + ao, kZCore, kZGroup);
-            const uint64_t bh = umma_desc(smem_u32(sm.zbh[kk]) + bo), bl = umma_desc(smem_u32(sm.zbl[kk]) + bo);
-            mma_k16_desc(tmem + hb + kColZ, ah, bh, idesc32, kk + k16 > 0);
-            mma_k16_desc(tmem + hb + kColZ, ah, bl, idesc32, true);
-            mma_k16_desc(tmem + hb + kColZ, al, bh, idesc32, true);
-          }
+        // K steps of 16 tokens up to the stage's last token: past it -S is zero
+        const int nk16 = (T + 15) >> 4;
+        for (int st16 = 0; st16 < nk16; ++st16) {
+          const int kk = st16 >> 1, k16 = st16 & 1;   // A steps 2 padded core matrices, B 2 plain ones
+          const uint32_t ao = k16 * 2 * kZCore, bo = k16 * 256;
+          const uint64_t ah = umma_desc_strided(smem_u32(sm.zah[kk]) + ao, kZCore, kZGroup);
+          const uint64_t al = umma_desc_strided(smem_u32(sm.zal[kk]) + ao, kZCore, kZGroup);
+          const uint64_t bh = umma_desc(smem_u32(sm.zbh[kk]) + bo), bl = umma_desc(smem_u32(sm.zbl[kk]) + bo);
+          mma_k16_desc(tmem + hb + kColZ, ah, bh, idesc32, st16 > 0);
+          mma_k16_desc(tmem + hb + kColZ, ah, bl, idesc32, true);
+          mma_k16_desc(tmem + hb + kColZ, al, bh, idesc32, true);
         }
         mma_commit(&sm.mbar_z);
       }
