@@ -49,13 +49,18 @@
  * chunkwise form: within a chunk every row of the state solves one shared
  * triangular system (fp32), and the products around it run on the tensor cores
  * with each fp32 operand split into bf16 high + low parts (about fp32 accuracy).
+ * With bf16 activations as well, each route's scaled output is rounded to
+ * bfloat16 before the four are summed in fp32 (in the order r0..r3) and
+ * rounded once more to y.
  *
  * Errors.  Every entry point returns an srnl_status and never aborts.  On
  * failure the outputs are unspecified and srnl_scan_last_error() describes
  * the cause.  Kernels are asynchronous on the given stream: a CUDA error
  * raised by a kernel surfaces from a later call or a stream synchronisation.
  * No kernel of this library waits on another kernel, rank or flag; the scan
- * kernel's only waits are bounded polls on its own tensor-core completions.
+ * kernel's only waits are bounded polls on its own tensor-core completions and
+ * on its own TMA copies (the stage tiles of bf16 activations arrive by
+ * cp.async.bulk.tensor, without cluster multicast).
  *
  * Threads.  A handle may be used from one host thread at a time; forward
  * calls on one handle must not overlap on the device (they share the
