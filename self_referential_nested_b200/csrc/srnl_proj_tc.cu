@@ -279,14 +279,15 @@ cudaError_t launch_query_projection_tc(const ScanGeom& g, const ScanParamsDev& p
                                        int* err, cudaStream_t s) {
   const int64_t M = (int64_t)g.B * g.H * g.W;
   if (g.C <= 128) {
-    // persistent: TMEM (2 C columns, rounded up to a power of two) and shared memory allow
-    // several CTAs per SM; enough CTAs for every SM to hold a few, each walking several tiles
+    // persistent: TMEM (2 C columns, rounded up to a power of two) and shared memory bound the
+    // CTAs per SM; every SM holds up to two, each walking several tiles
     uint32_t cols = 32;
     while ((int)cols < 2 * g.C) cols <<= 1;
     const int per_sm_tmem = 512 / (int)cols;
     const size_t sm_bytes = pipelined_smem(g.C);
     const int per_sm_smem = (int)((size_t)(228 * 1024) / (sm_bytes + 1024));
-    const int per_sm = std::max(1, std::min(std::min(per_sm_tmem, per_sm_smem), 4));
+    // two per SM measured best at S1 (20.9 us, against 22.4 with three and 24.7 with one)
+    const int per_sm = std::max(1, std::min(std::min(per_sm_tmem, per_sm_smem), 2));
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
