@@ -278,8 +278,10 @@ static srnl_status run_forward(srnl_scan* h, const void* x, void* y, float* fina
   }
   float* fk = padded && finals != nullptr ? h->fin_pad : finals;
   void* yk = padded ? h->y_pad : y;
-  e = srnl::launch_query_projection(h->geom, p, x, h->q, h->dev_err, s);
-  if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
+  if (!srnl::scan_fuses_query(h->geom, p)) {   // otherwise the scan forms q itself
+    e = srnl::launch_query_projection(h->geom, p, x, h->q, h->dev_err, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "query projection launch");
+  }
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(h, e, "event record");
   if (h->geom.hard_cap && (e = cudaMemsetAsync(h->binds, 0, sizeof(unsigned long long), s)) != cudaSuccess)
     return cuda_fail(h, e, "counter reset");

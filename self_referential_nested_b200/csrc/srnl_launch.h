@@ -45,6 +45,16 @@ cudaError_t launch_query_projection_tc(const ScanGeom& g, const ScanParamsDev& p
 cudaError_t launch_scan(const ScanGeom& g, const ScanParamsDev& p, const void* x, const void* q,
                         float* yr, float* finals, int* err, unsigned long long* binds, cudaStream_t s);
 
+// Whether launch_scan computes the queries itself (the chunkwise kernel on bf16 activations
+// and generation, two 32-wide heads (C = 64), the operator's four routes, chunks that fit one
+// stage and column chunks that stay inside a column): each stage's full-width x rows arrive by
+// TMA and one tensor-core product gives q, so launch_query_projection is skipped and its q
+// buffer is not read.
+inline bool scan_fuses_query(const ScanGeom& g, const ScanParamsDev& p) {
+  return g.act_bf16 && g.gen_bf16 && g.hd == 32 && g.C == 64 && g.routes == 4 && p.Wqb != nullptr &&
+         g.Lrow <= 64 && g.Lcol <= 64 && g.Lcol <= g.H && g.H % g.Lcol == 0;
+}
+
 // Whether launch_scan writes the route partials in bf16: the chunkwise kernel (bf16 generation,
 // 32-wide heads) with bf16 activations writes them in the output's precision; every other
 // path writes fp32.  The buffer is sized for fp32 either way.

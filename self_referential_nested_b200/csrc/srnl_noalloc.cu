@@ -221,7 +221,7 @@ extern "C" srnl_status srnl_scan_forward_noalloc(const srnl_scan_config* cfg,
   g.act_bf16 = act_bf16; g.gen_bf16 = gen_bf16;
   g.hard_cap = cfg->injection_cap == SRNL_CAP_HARD;
   const srnl::ScanParamsDev dp{Wq, Wqb, G, p->M_mem0, p->scales};
-  if (e == cudaSuccess) e = srnl::launch_query_projection(g, dp, x, q, dev_err, cs);
+  if (e == cudaSuccess && !srnl::scan_fuses_query(g, dp)) e = srnl::launch_query_projection(g, dp, x, q, dev_err, cs);
   if (e == cudaSuccess) e = srnl::launch_scan(g, dp, x, q, yr, nullptr, dev_err, nullptr, cs);
   if (e == cudaSuccess) e = srnl::launch_fuse(g, yr, y, cs);
   if (e != cudaSuccess) {

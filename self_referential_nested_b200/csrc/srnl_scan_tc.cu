@@ -101,11 +101,17 @@ struct alignas(128) TcSmem {
   // Y A operand: z_t rows 0..63; the MMA's rows 64..127 read the next 4 KB (unused lanes)
   alignas(128) unsigned char yah[64 * 64];
   alignas(128) unsigned char yal[64 * 64];
+  // the other head's 32 channels of the stage's x rows (rows 0..63), the second K half of the
+  // in-kernel query product when it is fused (its M = 128 read continues into mh / ml)
+  alignas(128) unsigned char xo[64 * 64];
   alignas(128) unsigned char mh[kD * 64];      // M_mem0 hi (row = output channel)
   alignas(128) unsigned char ml[kD * 64];      // M_mem0 lo
   alignas(128) unsigned char gb[80 * 64];      // G in bf16 (rows 66..79 zero)
-  alignas(128) unsigned char qbh[kD * 64];     // Q_b hi (W product B operand)
-  alignas(128) unsigned char qbl[kD * 64];     // Q_b lo
+  // Q_b hi and lo (the W product's B operand when a chunk spans several stages); when every
+  // chunk fits one stage they are unused and, with the query product fused, hold this head's
+  // 32 rows of W_q in bf16 (K = channels 0..31 in qbh, 32..63 in qbl)
+  alignas(128) unsigned char qbh[kD * 64];
+  alignas(128) unsigned char qbl[kD * 64];
   alignas(16) float qsT[kD][kD + 1];            // Q_s transposed, fp32 (column c in row c)
   alignas(16) float lam[kStage];                // Lambda_t (log2 retention prefix)
   alignas(16) float eta[kStage];
@@ -114,12 +120,14 @@ struct alignas(128) TcSmem {
   alignas(16) float4 gpart[kStage];            // readout-warp halves of ||k~||^2, k~.v, ||v||^2
   alignas(16) float4 gpar[kStage];             // gate scalars: 1/||k~||, alpha, g(t, T-1) eta, live
   float wsum;                                   // prefix of the first token warp
-  alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y, mbar_c, mbar_x;
+  alignas(8) unsigned long long mbar_w, mbar_g, mbar_1, mbar_z, mbar_y, mbar_c, mbar_x, mbar_q;
   uint32_t tmem_base;
   int wait_failed;
 };
 static_assert(sizeof(TcSmem) <= 113 * 1024, "two CTAs per SM");
 static_assert(offsetof(TcSmem, yal) + 2 * 64 * 64 <= sizeof(TcSmem), "Y operand rows 64..127 stay in bounds");
+static_assert(offsetof(TcSmem, xo) + 2 * 64 * 64 <= sizeof(TcSmem), "query operand rows 64..127 stay in bounds");
+static_assert(offsetof(TcSmem, qbl) == offsetof(TcSmem, qbh) + kD * 64, "W_q slice halves");
 static_assert(offsetof(TcSmem, a1l) == offsetof(TcSmem, a1h) + kTile, "A pieces");
 static_assert(offsetof(TcSmem, b1h) == offsetof(TcSmem, a1h) + 2 * kTile, "A pieces");
 static_assert(offsetof(TcSmem, b1l) == offsetof(TcSmem, b1h) + kB1Rows * 64, "A pieces");
@@ -139,6 +147,8 @@ struct TcArgs {
   float alpha, eps;
   bool act_bf16;
   bool hard_cap;
+  const __nv_bfloat16* Wqb;   // W_q [C][C] in bf16 (read when fuse_q)
+  bool fuse_q;                // q computed here from full-width x rows (C = 64, chunks <= 64)
 };
 
 // Tensor maps of the bf16 activations and queries, [B][H][W][C]: "row" views tokens as one
@@ -148,6 +158,7 @@ struct TcArgs {
 struct TcMaps {
   CUtensorMap xr, xc, qr, qc;
   uint32_t box_bytes_r, box_bytes_c;   // bytes of one x box (= one q box) per orientation
+  int box_ch;                          // channels per x box: 32 (one head), or C with the fused query
 };
 
 // -A[t][j] for j in [16p, 16p + 16) lives in the first 4 KB of a1h, a1l, b1h, b1l
@@ -442,7 +453,10 @@ __device__ __forceinline__ void tma_stage(TcSmem& sm, const TcMaps& m, const Sta
                                           int H, int W) {
   const uint32_t bar = smem_u32(&sm.mbar_x);
   const uint32_t box = r < 2 ? m.box_bytes_r : m.box_bytes_c;
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * box) : "memory");
+  const bool full = m.box_ch != kD;   // the fused query: full-width x rows, no q box
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(full ? box : 2 * box)
+               : "memory");
+  if (full) ch0 = 0;
   const int t_lo = (r & 1) ? si.t0 + si.T - 1 : si.t0;      // route token at the lowest address
   const int p = route_pos(r, t_lo, H, W);
   if (r < 2) {
@@ -451,10 +465,11 @@ __device__ __forceinline__ void tma_stage(TcSmem& sm, const TcMaps& m, const Sta
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
             smem_u32(sm.yah)), "l"(reinterpret_cast<uint64_t>(&m.xr)), "r"(ch0), "r"(c1), "r"(bar)
         : "memory");
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            smem_u32(sm.yal)), "l"(reinterpret_cast<uint64_t>(&m.qr)), "r"(ch0), "r"(c1), "r"(bar)
-        : "memory");
+    if (!full)
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+              smem_u32(sm.yal)), "l"(reinterpret_cast<uint64_t>(&m.qr)), "r"(ch0), "r"(c1), "r"(bar)
+          : "memory");
   } else {
     const int i = p / W, j = p - i * W;
     const int c2 = b * H + i;
@@ -462,10 +477,11 @@ __device__ __forceinline__ void tma_stage(TcSmem& sm, const TcMaps& m, const Sta
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
             smem_u32(sm.yah)), "l"(reinterpret_cast<uint64_t>(&m.xc)), "r"(ch0), "r"(j), "r"(c2), "r"(bar)
         : "memory");
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-            smem_u32(sm.yal)), "l"(reinterpret_cast<uint64_t>(&m.qc)), "r"(ch0), "r"(j), "r"(c2), "r"(bar)
-        : "memory");
+    if (!full)
+      asm volatile(
+          "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+              smem_u32(sm.yal)), "l"(reinterpret_cast<uint64_t>(&m.qc)), "r"(ch0), "r"(j), "r"(c2), "r"(bar)
+          : "memory");
   }
 }
 
@@ -479,9 +495,22 @@ __device__ __forceinline__ bool stage_is_box(const StageInfo& si, int r, int H) 
 
 // Token warps (ht = 0..63): the staged boxes (64-byte rows, ascending raster order) into the
 // operand tiles in route order: x into rows t and 64 + t of the x tile, q into rows 64 + t of
-// the M1 A tile, for the stage's T tokens (the rows past them keep earlier tokens, which every
+// the M1 A tile (with the fused query: the other head's x channels into xo instead), for the
+// stage's T tokens (the rows past them keep earlier tokens, which every
 // consumer masks).  Reverse routes read the box backwards.
-__device__ __forceinline__ void unstage(TcSmem& sm, const StageInfo& si, int r, int ht) {
+__device__ __forceinline__ void unstage(TcSmem& sm, const StageInfo& si, int r, int ht, bool fused, int h) {
+  if (fused) {   // full-width rows (128 B): this head's channels to the x tile, the other head's to xo
+    for (int idx = ht; idx < si.T * 4; idx += 64) {
+      const int t = idx >> 2, part = idx & 3;
+      const int row = (r & 1) ? si.T - 1 - t : t;
+      const uint4 own = *reinterpret_cast<const uint4*>(sm.yah + row * 128 + h * 64 + part * 16);
+      const uint4 oth = *reinterpret_cast<const uint4*>(sm.yah + row * 128 + (1 - h) * 64 + part * 16);
+      *reinterpret_cast<uint4*>(sm.xa + umma_off(t, part * 8)) = own;
+      *reinterpret_cast<uint4*>(sm.xa + umma_off(64 + t, part * 8)) = own;
+      *reinterpret_cast<uint4*>(sm.xo + umma_off(t, part * 8)) = oth;
+    }
+    return;
+  }
   for (int idx = ht; idx < si.T * 4; idx += 64) {
     const int t = idx >> 2, part = idx & 3;
     const int row = (r & 1) ? si.T - 1 - t : t;
@@ -491,6 +520,44 @@ __device__ __forceinline__ void unstage(TcSmem& sm, const StageInfo& si, int r, 
     *reinterpret_cast<uint4*>(sm.xa + umma_off(64 + t, part * 8)) = xv;
     *reinterpret_cast<uint4*>(sm.a1h + umma_off(64 + t, part * 8)) = qv;
   }
+}
+
+// Token warps (ht = 0..63), fused query only: q_t = x_t W_q[h]^T for the staged stage (x of
+// channels 0..31 and 32..63 as the two K halves, this head's W_q rows in the Q_b tiles), on the
+// tensor cores into 32 columns of TMEM (lanes = tokens), then rounded to bf16 into rows 64 + t
+// of the M1 A tile, as the separate projection kernel would have left them.  The K order
+// (channels 0..31 first) is the projection kernel's.
+__device__ __forceinline__ void query_product(TcSmem& sm, uint32_t tmem, uint32_t tmem_lane, uint32_t col, int h,
+                                              int T, int ht, uint32_t& qpar) {
+  fence_async_smem();
+  tc_fence_before();
+  tok_bar();
+  if (ht == 0) {
+    tc_fence_after();
+    const uint32_t lo = smem_u32(h == 0 ? sm.xa : sm.xo), hi = smem_u32(h == 0 ? sm.xo : sm.xa);
+    mma_k32(tmem + col, lo, smem_u32(sm.qbh), idesc_bf16(32), false);
+    mma_k32(tmem + col, hi, smem_u32(sm.qbl), idesc_bf16(32), true);
+    mma_commit(&sm.mbar_q);
+  }
+  mbar_wait(&sm.mbar_q, qpar, &sm.wait_failed);
+  qpar ^= 1u;
+  float qv[kD];
+  SRNL_LD16(qv, tmem_lane + col);
+  SRNL_LD16(qv + 16, tmem_lane + col + 16);
+  tmem_wait_ld();
+  if (ht < T) {
+#pragma unroll
+    for (int c = 0; c < kD; c += 8) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(qv[c + 2 * e], qv[c + 2 * e + 1]);
+        w4[e] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(sm.a1h + umma_off(64 + ht, c)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+  fence_async_smem();
 }
 
 __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(const TcArgs a,
@@ -531,6 +598,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_y)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_c)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_x)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar_q)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -544,7 +612,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
     const int o = i / kD, kk = i % kD;
     store_split(sm.mh, sm.ml, o, kk, Msrc[i]);
     const float e = (o == kk) ? 1.f : 0.f;
-    store_split(sm.qbh, sm.qbl, o, kk, e);
+    if (!a.fuse_q) store_split(sm.qbh, sm.qbl, o, kk, e);   // fused: the tiles hold W_q instead
     store_split(sm.b1h, sm.b1l, 64 + o, kk, e);
     sm.qsT[o][kk] = e;
   }
@@ -557,18 +625,31 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
   const int nst = live_stages(N, L);
   if (tid == 32 && a.act_bf16) {   // the tensor maps into the descriptor cache before first use
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.xr)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.qr)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.xc)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.qc)) : "memory");
+    if (!a.fuse_q) {   // with the fused query the q maps are not encoded
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.qr)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.qc)) : "memory");
+    }
   }
   uint32_t xpar = 0;   // phase of mbar_x (token warps)
+  uint32_t qpar = 0;   // phase of mbar_q (token warps)
   if (is_k && nst > 0) {
     const StageInfo s0 = stage_info(0, N, L);
+    if (a.fuse_q) {   // this head's W_q rows (bf16), K halves in qbh / qbl
+      for (int i = tid - 128; i < kD * 64; i += 64) {
+        const int o = i >> 6, k = i & 63;
+        *reinterpret_cast<__nv_bfloat16*>((k < 32 ? sm.qbh : sm.qbl) + umma_off(o, k & 31)) =
+            a.Wqb[(int64_t)(ch0 + o) * a.C + k];
+      }
+    }
     if (a.act_bf16 && stage_is_box(s0, r, a.H)) {
       if (tid == 128) tma_stage(sm, maps, s0, r, b, ch0, a.H, a.W);
       mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
       xpar ^= 1u;
-      unstage(sm, s0, r, tid - 128);
+      unstage(sm, s0, r, tid - 128, a.fuse_q, h);
+      if (a.fuse_q)
+        query_product(sm, sm.tmem_base, sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16), 32u, h, s0.T, tid - 128,
+                      qpar);
     } else {
       tc_prefetch(sm, s0, a, r, tok0, ch0, tid - 128);
       cp_async_wait_all();
@@ -856,7 +937,10 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         // the Gen and M1 products have finished reading
         mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
         xpar ^= 1u;
-        unstage(sm, sn, r, gt);
+        unstage(sm, sn, r, gt, a.fuse_q, h);
+        // the next stage's queries, into columns 32..63 of its TMEM half (free once y of the
+        // previous stage has been drained above)
+        if (a.fuse_q) query_product(sm, tmem, tmem_lane, (uint32_t)((ne + 1) & 1) * 128u + 32u, h, sn.T, gt, qpar);
       } else {
         cp_async_wait_all();
       }
@@ -1081,23 +1165,23 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return g_encode;
 }
 
-// Row view: [B*H*W][C]; column view: [B*H][W][C].  bf16, boxes of 32 channels x box_r (row
+// Row view: [B*H*W][C]; column view: [B*H][W][C].  bf16, boxes of box_ch channels x box_r (row
 // view) or box_c (column view) tokens.
-bool encode_maps(const void* base, int B, int H, int W, int C, int box_r, int box_c, CUtensorMap* row,
+bool encode_maps(const void* base, int B, int H, int W, int C, int box_ch, int box_r, int box_c, CUtensorMap* row,
                  CUtensorMap* col) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint32_t estr[3] = {1, 1, 1};
   const cuuint64_t rdim[2] = {(cuuint64_t)C, (cuuint64_t)B * H * W};
   const cuuint64_t rstr[1] = {(cuuint64_t)C * 2};
-  const cuuint32_t rbox[2] = {(cuuint32_t)kD, (cuuint32_t)box_r};
+  const cuuint32_t rbox[2] = {(cuuint32_t)box_ch, (cuuint32_t)box_r};
   CUresult e = enc(row, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), rdim, rstr, rbox, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (e != CUDA_SUCCESS) return false;
   const cuuint64_t cdim[3] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)B * H};
   const cuuint64_t cstr[2] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2};
-  const cuuint32_t cbox[3] = {(cuuint32_t)kD, 1, (cuuint32_t)box_c};
+  const cuuint32_t cbox[3] = {(cuuint32_t)box_ch, 1, (cuuint32_t)box_c};
   e = enc(col, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), cdim, cstr, cbox, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1116,16 +1200,20 @@ cudaError_t launch_scan_chunkwise(const ScanGeom& g, const ScanParamsDev& p, con
   a.Lrow = g.Lrow; a.Lcol = g.Lcol; a.alpha = g.alpha; a.eps = g.eps;
   a.act_bf16 = g.act_bf16;
   a.hard_cap = g.hard_cap; a.binds = binds;
+  a.Wqb = static_cast<const __nv_bfloat16*>(p.Wqb);
+  a.fuse_q = scan_fuses_query(g, p);
   const unsigned nseq = (unsigned)g.routes * (unsigned)g.B * (unsigned)g.heads;
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
   if (g.act_bf16) {
     // a stage holds at most min(L, 64) tokens: the box covers that, rounded up to 8
     const int box_r = std::min(kStage, (g.Lrow + 7) / 8 * 8), box_c = std::min(kStage, (g.Lcol + 7) / 8 * 8);
-    maps.box_bytes_r = (uint32_t)box_r * kD * 2;
-    maps.box_bytes_c = (uint32_t)box_c * kD * 2;
-    if (!encode_maps(x, g.B, g.H, g.W, g.C, box_r, box_c, &maps.xr, &maps.xc) ||
-        !encode_maps(q, g.B, g.H, g.W, g.C, box_r, box_c, &maps.qr, &maps.qc))
+    const bool fuse = scan_fuses_query(g, p);
+    maps.box_ch = fuse ? g.C : kD;   // the fused query reads full-width x rows (128 B) and no q
+    maps.box_bytes_r = (uint32_t)box_r * maps.box_ch * 2;
+    maps.box_bytes_c = (uint32_t)box_c * maps.box_ch * 2;
+    if (!encode_maps(x, g.B, g.H, g.W, g.C, maps.box_ch, box_r, box_c, &maps.xr, &maps.xc) ||
+        (!fuse && !encode_maps(q, g.B, g.H, g.W, g.C, kD, box_r, box_c, &maps.qr, &maps.qc)))
       return cudaErrorInvalidValue;
   }
   srnl_scan_chunkwise_kernel<<<nseq, kThreadsTc, sizeof(TcSmem), s>>>(a, maps);
