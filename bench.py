@@ -61,6 +61,15 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------- work model
+def scan_fuses_query(cfg, gen):
+    """Whether the library's scan forms the queries itself (no projection launch): bf16
+    activations and generation, two 32-wide heads (C = 64), chunks of at most 64 tokens, column
+    chunks inside a column.  Mirrors the library's launch rule, for the launch count."""
+    lr, lc = cfg.chunk_row or cfg.W, cfg.chunk_col or cfg.H
+    return (cfg.act_dtype == "bf16" and gen == "bf16" and cfg.d == 32 and cfg.C == 64 and lr <= 64 and lc <= 64
+            and lc <= cfg.H and cfg.H % lc == 0)
+
+
 def work_model(cfg, gen_bf16=True):
     """Algorithmic bytes and flops of one forward (per launch)."""
     B, H, W, C, heads, d = cfg.B, cfg.H, cfg.W, cfg.C, cfg.heads, cfg.d
@@ -404,7 +413,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                   "note": "scan of one image (each sequence alone on an SM) over the full scan"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * elt),
                 "d2h_bytes_per_step": int(y.numel() * elt), "ms_per_step": e2e_ms / args.steps},
-        "gpu_launches": (3 if cfg.d >= 32 else 5) * args.steps,   # + pad x, unpad y below 32
+        # projection (unless the scan forms q), scan, fusion; + pad x, unpad y below 32
+        "gpu_launches": ((2 if scan_fuses_query(cfg, gen) else 3) + (0 if cfg.d >= 32 else 2)) * args.steps,
         "clocks": clocks.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
