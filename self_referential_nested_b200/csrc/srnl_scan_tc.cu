@@ -526,9 +526,9 @@ __device__ __forceinline__ void unstage(TcSmem& sm, const StageInfo& si, int r, 
 // channels 0..31 and 32..63 as the two K halves, this head's W_q rows in the Q_b tiles), on the
 // tensor cores into 32 columns of TMEM (lanes = tokens), then rounded to bf16 into rows 64 + t
 // of the M1 A tile, as the separate projection kernel would have left them.  The K order
-// (channels 0..31 first) is the projection kernel's.
-__device__ __forceinline__ void query_product(TcSmem& sm, uint32_t tmem, uint32_t tmem_lane, uint32_t col, int h,
-                                              int T, int ht, uint32_t& qpar) {
+// (channels 0..31 first) is the projection kernel's.  query_issue starts the product;
+// query_drain waits for it and stores q, so other work can sit between the two.
+__device__ __forceinline__ void query_issue(TcSmem& sm, uint32_t tmem, uint32_t col, int h, int ht) {
   fence_async_smem();
   tc_fence_before();
   tok_bar();
@@ -539,6 +539,10 @@ __device__ __forceinline__ void query_product(TcSmem& sm, uint32_t tmem, uint32_
     mma_k32(tmem + col, hi, smem_u32(sm.qbl), idesc_bf16(32), true);
     mma_commit(&sm.mbar_q);
   }
+}
+
+__device__ __forceinline__ void query_drain(TcSmem& sm, uint32_t tmem_lane, uint32_t col, int T, int ht,
+                                            uint32_t& qpar) {
   mbar_wait(&sm.mbar_q, qpar, &sm.wait_failed);
   qpar ^= 1u;
   float qv[kD];
@@ -647,9 +651,10 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
       xpar ^= 1u;
       unstage(sm, s0, r, tid - 128, a.fuse_q, h);
-      if (a.fuse_q)
-        query_product(sm, sm.tmem_base, sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16), 32u, h, s0.T, tid - 128,
-                      qpar);
+      if (a.fuse_q) {
+        query_issue(sm, sm.tmem_base, 32u, h, tid - 128);
+        query_drain(sm, sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16), 32u, s0.T, tid - 128, qpar);
+      }
     } else {
       tc_prefetch(sm, s0, a, r, tok0, ch0, tid - 128);
       cp_async_wait_all();
@@ -921,6 +926,17 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
       const StageInfo sn = stage_info(ne + 1 < nst ? ne + 1 : ne, N, L);
       const bool next_box = a.act_bf16 && ne + 1 < nst && stage_is_box(sn, r, a.H);
       if (!next_box && ne + 1 < nst) tc_prefetch(sm, sn, a, r, tok0, ch0, gt);
+      // the next stage's boxes (issued during the gates) into the operand tiles, which the Gen
+      // and M1 products have finished reading; with the fused query, its product starts here,
+      // into columns 32..63 of the next stage's TMEM half, and runs beside the y drain below
+      // (columns 0..31 of that half)
+      const uint32_t qcol = (uint32_t)((ne + 1) & 1) * 128u + 32u;
+      if (next_box) {
+        mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
+        xpar ^= 1u;
+        unstage(sm, sn, r, gt, a.fuse_q, h);
+        if (a.fuse_q) query_issue(sm, tmem, qcol, h, gt);
+      }
       if (pend) {  // y of the previous stage: the Y product was issued in (A)
         mbar_wait(&sm.mbar_y, (uint32_t)((ne - 1) & 1), &sm.wait_failed);
         float y[kD];
@@ -933,14 +949,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2) srnl_scan_chunkwise_kernel(cons
         }
       }
       if (next_box) {
-        // the next stage's boxes (issued at the end of the gates) into the operand tiles, which
-        // the Gen and M1 products have finished reading
-        mbar_wait(&sm.mbar_x, xpar, &sm.wait_failed);
-        xpar ^= 1u;
-        unstage(sm, sn, r, gt, a.fuse_q, h);
-        // the next stage's queries, into columns 32..63 of its TMEM half (free once y of the
-        // previous stage has been drained above)
-        if (a.fuse_q) query_product(sm, tmem, tmem_lane, (uint32_t)((ne + 1) & 1) * 128u + 32u, h, sn.T, gt, qpar);
+        if (a.fuse_q) query_drain(sm, tmem_lane, qcol, sn.T, gt, qpar);
       } else {
         cp_async_wait_all();
       }
