@@ -36,10 +36,10 @@ from srnl_inputs import CONFIGS, Sustain, make_inputs  # noqa: E402
 METRIC = "SRNL 4-dir scan tokens/s (fwd, 1xB200) and % of roofline at 56x56x64"
 
 # DRAM bytes (read + write) of one scan launch, from a 1-pass ncu capture of the current
-# chunkwise kernel on the full workload (profiles/scan_dram_hier_s1_56x56.md): 25.92 MB read +
-# 2.82 MB written (the bf16 route partials stay in L2 for the fusion).  Keyed by (workload, B,
-# generation dtype); absent entries report null.
-SCAN_TRAFFIC_BYTES = {("hier_s1_56x56", 32, "bf16"): 25.92e6 + 2.82e6}
+# chunkwise kernel on the full workload (profiles/scan_dram_hier_s1_56x56.md): 13.08 MB read (x
+# once; the scan forms q itself) + 2.17 MB written (the bf16 route partials stay in L2 for the
+# fusion).  Keyed by (workload, B, generation dtype); absent entries report null.
+SCAN_TRAFFIC_BYTES = {("hier_s1_56x56", 32, "bf16"): 13.08e6 + 2.17e6}
 UNIT = "route-tokens/s"
 DEFAULT_CONFIG = "hier_s1_56x56"
 L2_FLUSH_BYTES = 256 << 20
